@@ -1,0 +1,392 @@
+#!/usr/bin/env python
+"""Benchmark of one SpecOPD target-scoring step on B200.
+
+A step is one pass of the whole hot path over one batch of synthetic trees:
+mask build -> RoPE + tree-masked GQA attention -> fused overlap / E2E-TV loss /
+gradient.  The metric is supervised tokens (predictions contributing to the
+loss, sum_b W) scored per second.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2] [--impl reference]
+
+N > 1 runs under torchrun: each rank scores its own batch (weak scaling; the
+trees are independent problems, so the data path has no collective), the
+timed region is bracketed by barriers and the slowest rank's time is used.
+`--impl reference` times the fp64 CPU oracle on the host cores instead (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "supervised tokens/s scored (tree attn + E2E-TV) on 1 B200; % of roofline"
+WORKLOAD_DEFAULT = 2
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sustained=d.get("bf16_tflops_sustained"),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ----------------------------------------------------------------- workload figures
+def visible_pairs(case) -> int:
+    """sum over packed rows of |vis(r)|: trunk row j sees j+1 columns, sample
+    y_{b,i} sees a_b+1 trunk columns plus i samples."""
+    total = 0
+    a_off = 0
+    for T, B in zip(case.trunk_len, case.num_branches):
+        total += T * (T + 1) // 2
+        anc = case.anchors[a_off:a_off + B].astype(np.int64)
+        rpb = case.rows_per_branch
+        total += int(rpb * (anc + 1).sum()) + B * rpb * (rpb + 1) // 2
+        a_off += B
+    return total
+
+
+def case_figures(case):
+    pairs = visible_pairs(case)
+    flops = 4.0 * case.d * case.Hq * pairs
+    es = 2 if case.dtype == "bf16" else 4
+    R = case.num_predictions
+    ov_bytes = float(R) * case.vocab * (2 * es + 4)
+    return dict(pairs=pairs, flops=flops, ov_bytes=ov_bytes, R=R)
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# ----------------------------------------------------------------- CPU oracle timing
+def oracle_sample(case, rng, attn_rows: int, branches: int, mask_rows: int):
+    """Time the oracle on a bounded sample of one step; returns the estimated
+    seconds of a whole step and a description of the sample."""
+    from oracle import attention as OA
+    from oracle import overlap as OO
+    from oracle import tree as OT
+    from synthetic import to_f64
+
+    t0 = time.perf_counter()
+    pt = OT.pack(case.trunk_len, case.prompt_len, case.num_branches, case.anchors, case.W, case.pack_terminal)
+    OT.positions(pt)
+    OT.prediction_rows(pt)
+    t_struct = time.perf_counter() - t0
+    N = pt.num_rows
+    rows = rng.choice(N, size=min(mask_rows, N), replace=False)
+    t0 = time.perf_counter()
+    OT.compact_fields(pt, rows)
+    t_mask = (time.perf_counter() - t0) / len(rows) * N
+    rows = rng.choice(N, size=min(attn_rows, N), replace=False)
+    q, k, v = (to_f64(x, case.dtype) for x in (case.q, case.k, case.v))
+    t0 = time.perf_counter()
+    OA.tree_attention(pt, q, k, v, theta=case.theta, rows=rows)
+    t_attn = (time.perf_counter() - t0) / len(rows) * N
+    nb = int(sum(case.num_branches))
+    bs = rng.choice(nb, size=min(branches, nb), replace=False)
+    t0 = time.perf_counter()
+    for b in bs:
+        r = np.arange(b * case.W, (b + 1) * case.W)
+        z = to_f64(case.draft[r], case.dtype)
+        t = to_f64(case.teacher[r], case.dtype)
+        a = OO.overlap(z, t)
+        OO.e2e_tv_loss(a, case.W, count=nb * case.W)
+        OO.e2e_tv_grad_draft(z, t, case.W, count=nb * case.W)
+    t_ov = (time.perf_counter() - t0) / len(bs) * nb
+    total = t_struct + t_mask + t_attn + t_ov
+    desc = (f"oracle on {len(rows)} of {N} packed rows (attention, all {case.Hq} heads), {mask_rows} rows of "
+            f"mask fields, {len(bs)} of {nb} branches (overlap + loss + gradient over all {case.W} rows), "
+            f"scaled linearly to the full step")
+    return total, desc
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [x.get("num_threads", 1) for x in threadpool_info() if x.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(case, seconds_target: float = 15.0):
+    rng = np.random.default_rng(123)
+    # a first small sample fixes the cost per unit, then the sample is sized
+    # to about `seconds_target` of CPU work
+    t_step, _ = oracle_sample(case, rng, attn_rows=2, branches=1, mask_rows=8)
+    t0 = time.perf_counter()
+    est, desc = oracle_sample(case, rng, attn_rows=8, branches=1, mask_rows=32)
+    spent = time.perf_counter() - t0
+    if spent < seconds_target / 3:
+        scale = max(1, int(seconds_target / max(spent, 1e-3)))
+        est, desc = oracle_sample(case, rng, attn_rows=min(8 * scale, 256), branches=min(scale, 8),
+                                  mask_rows=min(32 * scale, 512))
+    value = case.num_predictions / est
+    return {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle", "sample": desc,
+            "est_step_s": est}
+
+
+# ----------------------------------------------------------------- GPU run
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    import synthetic as SY
+    from tree_attention_masked_b200.build import build
+    build()
+    from tree_attention_masked_b200 import specopd as S
+    from tree_attention_masked_b200.scoring import ScoringStep
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    case = SY.make_workload(args.workload, seed=args.seed + rank, workers=min(8, os.cpu_count() or 1))
+    figs = case_figures(case)
+    st = ScoringStep(case.trunk_len, case.prompt_len, case.num_branches, case.W, case.Hq, case.Hkv, case.d,
+                     torch.bfloat16 if case.dtype == "bf16" else torch.float32, case.vocab, device=dev,
+                     pack_terminal=case.pack_terminal, theta=case.theta)
+    st.load(case)
+    stream = torch.cuda.current_stream(dev)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    K, Wm = args.steps, args.warmup
+    marks = [[ev() for _ in range(4)] for _ in range(K)]
+
+    def step(i=None):
+        if i is not None:
+            marks[i][0].record(stream)
+        st.build_mask(stream)
+        if i is not None:
+            marks[i][1].record(stream)
+        st.attention(stream)
+        if i is not None:
+            marks[i][2].record(stream)
+        st.overlap(stream)
+        if i is not None:
+            marks[i][3].record(stream)
+
+    for _ in range(Wm):
+        step()
+    torch.cuda.synchronize()
+    if st.check_status() != 0:
+        raise RuntimeError(f"device status {st.check_status()}")
+
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    clocks.start()
+    time.sleep(0.3)
+    start, end = ev(), ev()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(K):
+        step(i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = start.elapsed_time(end)
+    clk = clocks.stop()
+    t_mask = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
+    t_attn = statistics.mean(m[1].elapsed_time(m[2]) for m in marks)
+    t_ov = statistics.mean(m[2].elapsed_time(m[3]) for m in marks)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    # ---- end to end through the public API with host buffers
+    pin = lambda x, dt: (torch.from_numpy(x).view(torch.bfloat16) if dt == "bf16" else torch.from_numpy(x)).pin_memory()
+    h_in = [torch.from_numpy(case.anchors).pin_memory(), pin(case.q, case.dtype), pin(case.k, case.dtype),
+            pin(case.v, case.dtype), pin(case.draft, case.dtype), pin(case.teacher, case.dtype)]
+    d_in = [st.anchors, st.q, st.k, st.v, st.draft, st.teacher]
+    h_loss = torch.empty(1, dtype=torch.float32).pin_memory()
+    h_alpha = torch.empty(st.R, dtype=torch.float32).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in h_in)
+    d2h = h_loss.numel() * 4 + h_alpha.numel() * 4
+
+    def e2e_step():
+        for h, d in zip(h_in, d_in):
+            d.copy_(h, non_blocking=True)
+        st.run(stream)
+        h_loss.copy_(st.loss, non_blocking=True)
+        h_alpha.copy_(st.alpha[:st.R], non_blocking=True)
+
+    for _ in range(max(1, Wm // 2)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_start, e_end = ev(), ev()
+    if world > 1:
+        dist.barrier()
+    e_start.record(stream)
+    for _ in range(K):
+        e2e_step()
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e_start.elapsed_time(e_end)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    status = st.check_status()
+
+    peaks = load_peaks()
+    attn_tflops = figs["flops"] / (t_attn * 1e-3) / 1e12
+    ov_gbs = figs["ov_bytes"] / (t_ov * 1e-3) / 1e9
+    kernels = {
+        "tree_attention": {"bound": "tensor", "ms": t_attn, "achieved": attn_tflops, "unit": "TFLOP/s",
+                           "peak": peaks["bf16"], "frac": attn_tflops / peaks["bf16"],
+                           "useful_flops": figs["flops"], "visible_pairs": figs["pairs"]},
+        "tv_overlap_e2e": {"bound": "hbm", "ms": t_ov, "achieved": ov_gbs, "unit": "GB/s", "peak": peaks["hbm"],
+                           "frac": ov_gbs / peaks["hbm"], "algorithmic_bytes": figs["ov_bytes"]},
+        "build_tree_mask": {"ms": t_mask},
+    }
+    dom = "tree_attention" if t_attn >= t_ov else "tv_overlap_e2e"
+    kd = kernels[dom]
+    roofline = {"bound": kd["bound"], "achieved": kd["achieved"], "peak": kd["peak"], "unit": kd["unit"],
+                "frac": kd["frac"], "traffic": None, "kernel": dom,
+                "peak_source": f"{peaks['source']} ({'bf16_tflops burst' if dom == 'tree_attention' else 'hbm_gbs'})"}
+    tokens = figs["R"] * world
+    value = tokens * K / (elapsed_ms * 1e-3)
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": Wm,
+        "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": case.dtype, "data": "synthetic (seeded; no datasets or weights)",
+        "config": {"workload": SY.WORKLOADS[args.workload], "supervised_tokens_per_step": figs["R"],
+                   "packed_rows": case.num_rows, "visible_pairs": figs["pairs"], "seed": args.seed,
+                   "l2": "inputs larger than L2 (%.2f GB per step > 126 MB); each step streams them from HBM" %
+                         ((case.q.nbytes + case.k.nbytes + case.v.nbytes + case.draft.nbytes + case.teacher.nbytes) / 1e9),
+                   "parallelism": f"dp{world} (independent tree batches per rank)"},
+        "roofline": roofline,
+        "kernels": kernels,
+        "clocks": clk,
+        "e2e": {"value": tokens * K / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K},
+        "gpu_launches": 5 * K,
+        "device_status": status,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(case)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import synthetic as SY
+    case = SY.make_workload(args.workload, seed=args.seed, workers=min(8, os.cpu_count() or 1))
+    figs = case_figures(case)
+    rng = np.random.default_rng(7)
+    for _ in range(args.warmup):
+        oracle_sample(case, rng, attn_rows=1, branches=1, mask_rows=4)
+    ests = []
+    t0 = time.perf_counter()
+    desc = ""
+    for _ in range(args.steps):
+        est, desc = oracle_sample(case, rng, attn_rows=2, branches=1, mask_rows=8)
+        ests.append(est)
+    wall = time.perf_counter() - t0
+    est = statistics.mean(ests)
+    value = figs["R"] / est
+    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+           "impl": "reference",
+           "config": {"workload": SY.WORKLOADS[args.workload], "supervised_tokens_per_step": figs["R"]},
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                            "sample": desc + f"; {args.steps} samples, {wall:.1f} s wall"},
+           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=WORKLOAD_DEFAULT)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    # at least three untimed warm-up steps, whatever was asked for
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

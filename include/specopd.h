@@ -1,0 +1,250 @@
+/*
+ * specopd.h -- C ABI of the SpecOPD branch-parallel target-scoring library
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The method: "SpecOPD: Branch-Parallel On-Policy Distillation for Speculative
+ * Decoding".  Draft branches sampled at reference anchors are packed after a
+ * shared reference trunk (Fig 2, step 3); one tree-masked attention pass scores
+ * every packed row (Fig 3); the full-vocabulary overlap alpha and the E2E-TV
+ * loss with its gradient complete the path (daiwk.github.io write-up of the
+ * paper, section "Equations").
+ *
+ * Conventions for every entry point:
+ *   - The caller owns every buffer.  Pointers named *_dev or documented as
+ *     "device" are device memory of the current CUDA device; "host" pointers
+ *     are ordinary host memory read during the call only.
+ *   - The library allocates nothing and never synchronises: every kernel is
+ *     enqueued on the given stream and the call returns at once.
+ *   - A negative return value (specopd_status) means an argument error found
+ *     on the host; nothing was enqueued.  SPECOPD_ERR_CUDA means a launch
+ *     failed.
+ *   - Errors that depend on device data (an anchor outside the reference,
+ *     a non-finite teacher logit, a bounded wait that ran out) are OR-ed as
+ *     SPECOPD_FLAG_* bits into the caller's device word `status`.  The word is
+ *     never cleared by the library: zero it before the calls you want to check
+ *     and read it after the stream has synchronised.
+ *   - Tensors are row-major with the innermost dimension contiguous.
+ *   - All entry points may be called from several host threads on different
+ *     streams, but calls that share a workspace or a status word must be
+ *     ordered on one stream.
+ */
+#ifndef SPECOPD_H_
+#define SPECOPD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t without pulling in the CUDA headers */
+typedef struct CUstream_st* specopd_stream_t;
+
+typedef enum {
+  SPECOPD_OK = 0,
+  SPECOPD_ERR_ARG = -1,        /* null pointer, bad count, bad tree description */
+  SPECOPD_ERR_SHAPE = -2,      /* sizes out of the supported range */
+  SPECOPD_ERR_DTYPE = -3,      /* dtype not supported for this entry point */
+  SPECOPD_ERR_CUDA = -4,       /* a CUDA launch or driver call failed */
+  SPECOPD_ERR_WORKSPACE = -5,  /* workspace missing, too small or misaligned */
+  SPECOPD_ERR_ALIGN = -6       /* a pointer or leading dimension breaks 16-byte alignment */
+} specopd_status;
+
+/* bits OR-ed into the device status word */
+#define SPECOPD_FLAG_ANCHOR 1u     /* an anchor lies outside [P, T-1]; it was clamped */
+#define SPECOPD_FLAG_NONFINITE 2u  /* a teacher logit is NaN/inf, or a draft logit is +inf */
+#define SPECOPD_FLAG_TIMEOUT 4u    /* a bounded in-kernel wait gave up; outputs are invalid */
+
+typedef enum { SPECOPD_F32 = 0, SPECOPD_BF16 = 1 } specopd_dtype;
+
+#define SPECOPD_MAX_TREES 512
+#define SPECOPD_MAX_W 64
+#define SPECOPD_TILE_ROWS 128
+
+/*
+ * A batch of proposal trees (Fig 2, step 3; Fig 3).
+ *
+ * Tree t has a trunk of trunk_len[t] tokens, the first prompt_len[t] of them
+ * the prompt and the rest the reference response, and num_branches[t]
+ * branches of W drafted samples y_{b,1..W}.  Branch b hangs off trunk token
+ * anchors[b] (zero-based within its tree, in [prompt_len, trunk_len-1]; the
+ * write-up's section "Inputs and code mapping" fixes zero-based anchors).
+ *
+ * Packing: tree t occupies packed rows [cu_rows[t], cu_rows[t+1]): the trunk
+ * first, then each branch's samples contiguously, branches in the order given.
+ * With pack_terminal = 1 every sample has a row (W rows per branch); with 0
+ * the terminal sample y_{b,W} gets none (W-1 rows per branch), since its
+ * prediction reads its predecessor's row and nothing reads its own (Fig 3).
+ *
+ * trunk_len, prompt_len, num_branches: host arrays [num_trees].
+ * anchors: DEVICE array [sum num_branches], tree-major.
+ */
+typedef struct {
+  int32_t num_trees;       /* 1 .. SPECOPD_MAX_TREES */
+  int32_t W;               /* 1 .. SPECOPD_MAX_W */
+  int32_t pack_terminal;   /* 0 or 1 */
+  const int32_t* trunk_len;
+  const int32_t* prompt_len;
+  const int32_t* num_branches;
+  const int32_t* anchors;  /* device */
+} specopd_tree_desc;
+
+/*
+ * Per query tile of up to SPECOPD_TILE_ROWS packed rows of one tree: the
+ * column ranges the rows of the tile can see.  All values are global packed
+ * indices.  Written by specopd_build_tree_mask, read by
+ * specopd_tree_attention.
+ */
+typedef struct {
+  int32_t row_start;   /* first row of the tile */
+  int32_t row_end;     /* one past its last row (same tree) */
+  int32_t tree_base;   /* first packed row of the tree */
+  int32_t trunk_hi;    /* one past the last trunk column any row of the tile sees */
+  int32_t trunk_full;  /* every row of the tile sees every trunk column < trunk_full */
+  int32_t br_lo;       /* first branch column any row sees (br_lo == br_hi: none) */
+  int32_t br_hi;       /* one past the last branch column any row sees */
+  int32_t reserved;
+} specopd_tile_meta;
+
+/* Number of packed rows N of the batch, or a negative specopd_status. */
+int64_t specopd_tree_packed_rows(const specopd_tree_desc* desc);
+/* Number of query tiles (tiles never straddle two trees), or a negative status. */
+int64_t specopd_tree_num_tiles(const specopd_tree_desc* desc);
+/* Number of predictions sum_b W, or a negative status. */
+int64_t specopd_tree_num_predictions(const specopd_tree_desc* desc);
+
+/*
+ * specopd_build_tree_mask -- tree packing and the compact tree mask.
+ *
+ * Fig 3 (each row sees itself and its ancestors; siblings are hidden), the
+ * write-up's section "Equations" (history (x_{<=a_b}, y_{b,<i}); semantic
+ * position a_b + i; the anchor row predicts the first sample and the row of
+ * y_{b,i-1} predicts y_{b,i}).
+ *
+ * Outputs (device, written in full):
+ *   pos[N]          semantic position: trunk token j -> j, y_{b,i} -> a_b + i
+ *   trunk_limit[N]  largest tree-local trunk index the row sees: j on the trunk, a_b on a branch
+ *   branch_of[N]    global branch index of the row, -1 on the trunk
+ *   anc_bits[N]     bit k-1 set iff the row sees y_{b,k} of its own branch (0 on the trunk)
+ *   pred_rows[P]    P = sum_b W; entry b*W + i-1 is the packed row whose query
+ *                   predicts y_{b,i} (b-major over the whole batch)
+ *   cu_rows[num_trees+1]
+ *   tile_meta[num_tiles]
+ * So row r sees column c iff c lies in r's tree and either c is a trunk
+ * column with tree-local index <= trunk_limit[r], or c = row of y_{b,k} of
+ * r's own branch with bit k-1 of anc_bits[r] set.
+ *
+ * An anchor outside [prompt_len, trunk_len-1] sets SPECOPD_FLAG_ANCHOR in
+ * *status and is clamped into range so later kernels stay in bounds.
+ */
+int specopd_build_tree_mask(const specopd_tree_desc* desc, int32_t* pos, int32_t* trunk_limit,
+                            int32_t* branch_of, uint64_t* anc_bits, int32_t* pred_rows,
+                            int32_t* cu_rows, specopd_tile_meta* tile_meta, int32_t* status,
+                            specopd_stream_t stream);
+
+/*
+ * specopd_rope -- rotate-half rotary embedding at semantic positions.
+ *
+ * The write-up's section "Equations": branch token y_{b,i} takes position
+ * a_b + i, not its packed offset.  Element k of each head pairs with element
+ * k + d/2 and both rotate by pos[r] * theta^(-2k/d); the angle is formed in
+ * fp64.  q [N, Hq, d] -> q_out, k [N, Hkv, d] -> k_out (same dtype, may not
+ * alias the inputs).  d even, d <= 256.
+ */
+int specopd_rope(const void* q, const void* k, void* q_out, void* k_out, specopd_dtype dtype, int64_t N,
+                 int Hq, int Hkv, int d, const int32_t* pos, float theta, specopd_stream_t stream);
+
+/* Bytes of workspace specopd_tree_attention needs (rotated Q and K). */
+size_t specopd_attention_workspace_bytes(specopd_dtype dtype, int64_t N, int Hq, int Hkv, int d);
+
+/*
+ * specopd_tree_attention -- one tree-masked GQA attention pass over all packed rows.
+ *
+ * Fig 3: packed queries share trunk keys/values; every row attends to itself
+ * and its ancestors only.  O[r, h] = sum_{c visible to r} softmax_c(q_r.k_c *
+ * scale) v_c with q, k rotated at pos (specopd_rope), query head h reading
+ * KV head h / (Hq / Hkv).
+ *
+ * q [N, Hq, d], k and v [N, Hkv, d], out [N, Hq, d]: device, dtype `dtype`,
+ * 16-byte aligned.  rope_theta > 0 rotates q and k at pos first (into the
+ * workspace); rope_theta <= 0 takes q and k as already rotated.
+ * softmax_scale <= 0 means 1/sqrt(d).  pos, trunk_limit, anc_bits, tile_meta:
+ * outputs of specopd_build_tree_mask for the same trees.
+ * bf16 with d = 128 runs the tcgen05/TMEM kernel; fp32 (any d) and bf16 with
+ * other d (multiple of 32, <= 256) run a SIMT kernel with fp32 arithmetic.
+ * Accumulation is fp32 in both.
+ * workspace: device, >= specopd_attention_workspace_bytes, 256-byte aligned
+ * (may be null when rope_theta <= 0).
+ * status: device word; SPECOPD_FLAG_TIMEOUT if an in-kernel wait gave up.
+ */
+int specopd_tree_attention(const void* q, const void* k, const void* v, void* out, specopd_dtype dtype,
+                           int64_t N, int Hq, int Hkv, int d, float rope_theta, float softmax_scale,
+                           const int32_t* pos, const int32_t* trunk_limit, const uint64_t* anc_bits,
+                           const specopd_tile_meta* tile_meta, int64_t num_tiles, void* workspace,
+                           size_t workspace_bytes, int32_t* status, specopd_stream_t stream);
+
+/* Bytes of workspace specopd_tv_overlap_e2e needs. */
+size_t specopd_overlap_workspace_bytes(int64_t rows, int64_t V, int64_t num_branches);
+
+/*
+ * specopd_tv_overlap -- per-row full-vocabulary overlap, unfused.
+ *
+ * The write-up's section "Equations": alpha = sum_v min(q(v), p(v)) with q the
+ * draft softmax and p the teacher softmax over the FULL vocabulary (teacher
+ * mass outside the draft support is kept, never renormalised).  Section
+ * "Inputs and code mapping": draft entries that are NaN or -inf are outside
+ * the draft support; the teacher must be finite; bf16 work is promoted to fp32.
+ *
+ * draft [rows, ld_draft], teacher [rows, ld_teacher]: device, dtype `dtype`;
+ * the first V entries of each row are used.  Rows must start on 16-byte
+ * boundaries (base pointer and ld * element size).
+ * alpha[rows] (fp32, device) is written; q_less[rows] = sum_v q_v [q_v < p_v],
+ * lse_draft[rows], lse_teacher[rows] (natural-log normalisers) are written
+ * when non-null.  A row with an empty draft support gets alpha = 0.
+ * A non-finite teacher logit or a +inf draft logit sets SPECOPD_FLAG_NONFINITE.
+ */
+int specopd_tv_overlap(const void* draft, const void* teacher, specopd_dtype dtype, int64_t rows, int64_t V,
+                       int64_t ld_draft, int64_t ld_teacher, float* alpha, float* q_less, float* lse_draft,
+                       float* lse_teacher, int32_t* status, specopd_stream_t stream);
+
+/*
+ * specopd_e2e_tv_loss -- E2E-TV loss from per-prediction overlaps, unfused.
+ *
+ * The write-up's section "Equations": L = 1 - (1/count) sum_b sum_{j<=W}
+ * prod_{i<=j} alpha_{b,i}.  alpha: device [num_branches * W], b-major.
+ * count <= 0 means num_branches * W.  loss: device scalar.  grad_alpha
+ * (nullable, device [num_branches * W]) receives dL/dalpha.  An empty batch
+ * writes loss = 0.
+ */
+int specopd_e2e_tv_loss(const float* alpha, int64_t num_branches, int W, double count, float* loss,
+                        float* grad_alpha, specopd_stream_t stream);
+
+/*
+ * specopd_tv_overlap_e2e -- fused overlap, E2E-TV loss and gradient.
+ *
+ * One pass computes alpha for every prediction row; the last row of each
+ * branch to finish forms that branch's prefix products and dL/dalpha, and the
+ * last branch forms L.  With grad_draft non-null a second streaming pass
+ * writes dL/dz = dL/dalpha * q (1[q < p] - sum_v q_v 1[q_v < p_v]) (zero on
+ * entries outside the draft support); samples and teacher are held fixed
+ * (write-up, section "Equations").
+ *
+ * Rows are predictions b-major: row b*W + i-1 holds the logits read out for
+ * y_{b,i}.  rows must equal num_branches * W.  count <= 0 means rows.
+ * grad_draft [rows, ld_grad] fp32 device (16-byte aligned rows).
+ * workspace: device, >= specopd_overlap_workspace_bytes, 256-byte aligned.
+ * alpha[rows] and loss (scalar) are device fp32 outputs.
+ */
+int specopd_tv_overlap_e2e(const void* draft, const void* teacher, specopd_dtype dtype, int64_t rows,
+                           int64_t V, int64_t ld_draft, int64_t ld_teacher, int64_t num_branches, int W,
+                           double count, float* alpha, float* loss, float* grad_draft, int64_t ld_grad,
+                           void* workspace, size_t workspace_bytes, int32_t* status, specopd_stream_t stream);
+
+/* Human-readable name of a specopd_status value. */
+const char* specopd_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPECOPD_H_ */

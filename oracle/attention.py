@@ -63,16 +63,16 @@ def tree_attention(pt: _tree.PackedTrees, q: np.ndarray, k: np.ndarray, v: np.nd
     if scale is None:
         scale = 1.0 / np.sqrt(d)
     pos = _tree.positions(pt)
-    qr = rope(q, pos, theta)
+    rows = list(range(N)) if rows is None else list(rows)
+    qr = rope(np.asarray(q)[rows], pos[rows], theta)
     kr = rope(k, pos, theta)
     vv = np.asarray(v, dtype=np.float64)
-    rows = list(range(N)) if rows is None else list(rows)
     out = np.zeros((len(rows), Hq, d), dtype=np.float64)
     for n, r in enumerate(rows):
         cols = _tree.visible(pt, r)
         for h in range(Hq):
             g = h // grp
-            out[n, h] = _softmax_attend(qr[r, h], kr[cols, g], vv[cols, g], scale)
+            out[n, h] = _softmax_attend(qr[n, h], kr[cols, g], vv[cols, g], scale)
     return out
 
 

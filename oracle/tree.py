@@ -127,8 +127,16 @@ def dense_mask(pt: PackedTrees) -> np.ndarray:
 
 def positions(pt: PackedTrees) -> np.ndarray:
     """Semantic position of each row = number of strict ancestors (its depth).
-    For trunk token j this is j; for y_{b,i} it is a_b + i."""
-    return np.asarray([len(ancestors(pt, r)) for r in range(pt.num_rows)], dtype=np.int64)
+    For trunk token j this is j; for y_{b,i} it is a_b + i.  Parents are
+    packed before their children, so one pass in packed order counts them:
+    depth(r) = depth(parent(r)) + 1, depth(root) = 0."""
+    depth = np.zeros(pt.num_rows, dtype=np.int64)
+    for r in range(pt.num_rows):
+        p = int(pt.parent[r])
+        if p >= 0:
+            assert p < r, "parents are packed before their children"
+            depth[r] = depth[p] + 1
+    return depth
 
 
 def prediction_rows(pt: PackedTrees) -> np.ndarray:

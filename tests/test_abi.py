@@ -1,0 +1,113 @@
+"""The C ABI library loads, exports every symbol include/specopd.h declares,
+and its host-side logic (counts, argument validation) is right.  No kernel is
+launched: everything here runs without a GPU."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import tree as T
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "specopd.h")
+
+
+@pytest.fixture(scope="module")
+def S():
+    from tree_attention_masked_b200.build import build
+    build()
+    from tree_attention_masked_b200 import specopd
+    return specopd
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(specopd_[a-z_0-9]+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ["specopd_build_tree_mask", "specopd_tree_attention", "specopd_tv_overlap", "specopd_e2e_tv_loss",
+              "specopd_tv_overlap_e2e", "specopd_rope"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(S):
+    lib = ctypes.CDLL(S.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert sorted(S.EXPORTED) == declared_functions()
+
+
+CASES = [
+    ([12], [3], [4], [3, 7, 11, 5], 3, True),
+    ([12], [3], [4], [3, 7, 11, 5], 3, False),
+    ([300, 129, 1], [10, 0, 0], [7, 2, 0], [10, 299, 50, 60, 70, 80, 90, 5, 128], 5, True),
+    ([10], [4], [5], [4, 9, 6, 5, 8], 1, False),
+]
+
+
+@pytest.mark.parametrize("trunk,prompt,nb,anc,W,ptf", CASES)
+def test_counts_match_oracle(S, trunk, prompt, nb, anc, W, ptf):
+    import torch
+    trees = S.Trees(trunk, prompt, nb, W, torch.zeros(0, dtype=torch.int32), ptf)
+    pt = T.pack(trunk, prompt, nb, anc, W, ptf)
+    assert S.specopd_tree_packed_rows(trees) == pt.num_rows
+    assert S.specopd_tree_num_predictions(trees) == len(T.prediction_rows(pt))
+    tiles = sum((int(pt.cu_rows[t + 1] - pt.cu_rows[t]) + 127) // 128 for t in range(len(trunk)))
+    assert S.specopd_tree_num_tiles(trees) == tiles
+
+
+@pytest.mark.parametrize("trunk,prompt,nb,W", [
+    ([12], [12], [1], 2),     # prompt covers the whole trunk: no reference position
+    ([0], [0], [0], 2),       # empty trunk
+    ([12], [3], [-1], 2),
+    ([12], [3], [1], 0),
+    ([12], [3], [1], 65),
+])
+def test_bad_descriptions_rejected(S, trunk, prompt, nb, W):
+    import torch
+    trees = S.Trees(trunk, prompt, nb, W, torch.zeros(0, dtype=torch.int32))
+    with pytest.raises(S.SpecopdError):
+        S.specopd_tree_packed_rows(trees)
+
+
+def test_too_many_trees_rejected(S):
+    import torch
+    n = S.MAX_TREES + 1
+    trees = S.Trees([4] * n, [0] * n, [0] * n, 2, torch.zeros(0, dtype=torch.int32))
+    with pytest.raises(S.SpecopdError):
+        S.specopd_tree_packed_rows(trees)
+
+
+def test_argument_errors_before_launch(S):
+    lib = S._c
+    # null logits with rows > 0, misaligned leading dimension, unknown dtype
+    assert lib["specopd_tv_overlap"](None, None, 1, 4, 10, 10, 10, None, None, None, None, None, None) == -1
+    assert lib["specopd_tv_overlap"](16, 16, 1, 4, 10, 12, 12, 16, None, None, None, 16, None) == -6
+    assert lib["specopd_tv_overlap"](16, 16, 7, 4, 10, 16, 16, 16, None, None, None, 16, None) == -3
+    # rows must be num_branches * W for the fused entry point
+    assert lib["specopd_tv_overlap_e2e"](16, 16, 1, 5, 8, 8, 8, 2, 2, 0.0, 16, 16, None, 0, 256, 1 << 20, 16,
+                                         None) == -2
+    # workspace too small
+    need = S.specopd_overlap_workspace_bytes(4, 8, 2)
+    assert lib["specopd_tv_overlap_e2e"](16, 16, 1, 4, 8, 8, 8, 2, 2, 0.0, 16, 16, None, 0, 256, need - 1, 16,
+                                         None) == -5
+    # attention: head count not a multiple of KV heads, d outside the range
+    assert lib["specopd_tree_attention"](16, 16, 16, 16, 1, 8, 3, 2, 128, 1e4, 0.0, 16, 16, 16, 16, 1, 256, 1 << 20,
+                                         16, None) == -2
+    assert lib["specopd_tree_attention"](16, 16, 16, 16, 1, 8, 4, 2, 48, 1e4, 0.0, 16, 16, 16, 16, 1, 256, 1 << 20,
+                                         16, None) == -2
+    assert lib["specopd_rope"](16, 16, 16, 16, 1, 4, 2, 2, 6, 16, 1e4, None) == -2
+    assert lib["specopd_e2e_tv_loss"](16, 2, 0, 0.0, 16, None, None) == -2
+    assert S._c["specopd_status_string"](-5) == b"workspace missing, too small or misaligned"
+
+
+def test_workspace_sizes(S):
+    assert S.specopd_attention_workspace_bytes(S.BF16, 100, 4, 2, 128) == (
+        (100 * 4 * 128 * 2 + 255) // 256 * 256 + (100 * 2 * 128 * 2 + 255) // 256 * 256)
+    ws = S.specopd_overlap_workspace_bytes(1024, 151936, 64)
+    assert ws >= 1024 * 151936 // 8 + 3 * 1024 * 4

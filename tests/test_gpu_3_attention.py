@@ -1,0 +1,111 @@
+"""Tree attention on the GPU against the oracle.
+
+fp32 (SIMT kernel): relative L2 <= 1e-5.  bf16 (tcgen05 kernel for d = 128,
+SIMT for other d): relative L2 <= 1e-2 over the whole output, and every row
+within 2e-2 so that a single wrong row cannot hide in the average.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synthetic as SY
+from tests.gpu_cases import oracle_attention_rows, packed, rel_l2, step_for, to_np
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-5, "bf16": 1e-2}
+ROW_TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def run_attention(case):
+    st = step_for(case, with_grad=False)
+    st.build_mask()
+    st.attention()
+    torch.cuda.synchronize()
+    return st
+
+
+def check(case, st, rows=None):
+    pt = packed(case)
+    if rows is None:
+        rows = list(range(pt.num_rows))
+    ref = oracle_attention_rows(case, pt, rows)
+    got = to_np(st.out)[rows].astype(np.float64)
+    assert np.all(np.isfinite(got))
+    assert rel_l2(got, ref) <= TOL[case.dtype], rel_l2(got, ref)
+    per_row = [rel_l2(got[i], ref[i]) for i in range(len(rows))]
+    worst = int(np.argmax(per_row))
+    assert per_row[worst] <= ROW_TOL[case.dtype], (rows[worst], per_row[worst])
+
+
+def test_tiny_fp32_workload():
+    case = SY.make_workload(1)
+    st = run_attention(case)
+    assert st.check_status() == 0
+    check(case, st)
+
+
+SIMT = [
+    dict(trees=[(100, 10, 5)], W=4, Hq=4, Hkv=2, d=64, dtype="f32"),
+    dict(trees=[(150, 20, 6), (40, 3, 2)], W=3, Hq=6, Hkv=2, d=32, dtype="f32", pack_terminal=False),
+    dict(trees=[(260, 30, 8)], W=5, Hq=4, Hkv=1, d=64, dtype="bf16"),
+    dict(trees=[(200, 30, 4)], W=2, Hq=2, Hkv=2, d=256, dtype="f32"),
+]
+
+
+@pytest.mark.parametrize("spec", SIMT, ids=range(len(SIMT)))
+def test_simt_kernel(spec):
+    spec = dict(spec)
+    case = SY.make_case("simt", spec.pop("trees"), vocab=0, seed=4, **spec)
+    st = run_attention(case)
+    assert st.check_status() == 0
+    check(case, st)
+
+
+TC = [
+    dict(trees=[(300, 40, 9)], W=4, Hq=4, Hkv=1),                      # 3 tiles + ragged tail
+    dict(trees=[(512, 64, 16)], W=8, Hq=8, Hkv=2),                     # tiles aligned with branches
+    dict(trees=[(700, 100, 20)], W=8, Hq=10, Hkv=2),                   # odd group size (5 heads per KV head)
+    dict(trees=[(129, 0, 5), (77, 70, 3), (400, 100, 17)], W=3, Hq=4, Hkv=2),   # ragged multi-tree
+    dict(trees=[(300, 10, 6)], W=1, Hq=2, Hkv=2, anchors=[10, 299, 299, 50, 10, 120]),  # W=1, a_b=P, T-1, dups
+    dict(trees=[(300, 40, 9)], W=4, Hq=4, Hkv=1, pack_terminal=False),
+    dict(trees=[(250, 30, 7)], W=6, Hq=4, Hkv=2, sort_anchors=False),
+    dict(trees=[(90, 5, 3)], W=64, Hq=2, Hkv=1, anchors=[60, 5, 89]),  # full-width branches
+    dict(trees=[(1100, 200, 40)], W=16, Hq=4, Hkv=1),                  # 9 trunk tiles, 5 branch tiles
+]
+
+
+@pytest.mark.parametrize("spec", TC, ids=range(len(TC)))
+def test_tcgen05_kernel(spec):
+    spec = dict(spec)
+    case = SY.make_case("tc", spec.pop("trees"), d=128, dtype="bf16", vocab=0, seed=5, **spec)
+    st = run_attention(case)
+    assert st.check_status() == 0
+    check(case, st)
+
+
+def test_tcgen05_deterministic():
+    case = SY.make_case("det", [(700, 100, 20)], W=8, Hq=8, Hkv=2, d=128, dtype="bf16", vocab=0, seed=6)
+    st = run_attention(case)
+    o1 = st.out.clone()
+    st.attention()
+    torch.cuda.synchronize()
+    assert torch.equal(o1, st.out)
+
+
+@pytest.mark.parametrize("wl", [2, 3, 4, 5])
+def test_full_size_sampled_rows(wl):
+    case = SY.make_workload(wl, with_logits=False)
+    st = run_attention(case)
+    assert st.check_status() == 0
+    pt = packed(case)
+    N = pt.num_rows
+    rng = np.random.default_rng(wl)
+    # rows from every kind of tile: first/last trunk rows, branch rows, the tail
+    rows = {0, 127, 128, N - 1}
+    for t in range(len(case.trunk_len)):
+        base, T = int(pt.cu_rows[t]), case.trunk_len[t]
+        rows |= {base + T - 1, base + T, int(pt.cu_rows[t + 1]) - 1}
+    rows |= set(rng.choice(N, size=24, replace=False).tolist())
+    check(case, st, sorted(rows))
+    assert torch.isfinite(st.out.float()).all()

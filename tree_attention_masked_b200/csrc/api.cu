@@ -1,0 +1,292 @@
+// C ABI of the library (include/specopd.h): host-side validation, workspace
+// carving and kernel launches.  Nothing here allocates or synchronises.
+#include <cmath>
+#include <cstring>
+
+#include "internal.h"
+
+using namespace specopd;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Validate a tree description and fill the per-tree layout.  Returns a status.
+int tree_params(const specopd_tree_desc* d, TreeParams* p) {
+  if (!d || !d->trunk_len || !d->prompt_len || !d->num_branches) return SPECOPD_ERR_ARG;
+  if (d->num_trees < 1 || d->num_trees > SPECOPD_MAX_TREES) return SPECOPD_ERR_ARG;
+  if (d->W < 1 || d->W > SPECOPD_MAX_W) return SPECOPD_ERR_ARG;
+  if (d->pack_terminal != 0 && d->pack_terminal != 1) return SPECOPD_ERR_ARG;
+  std::memset(p, 0, sizeof(*p));
+  p->num_trees = d->num_trees;
+  p->W = d->W;
+  p->rows_per_branch = d->pack_terminal ? d->W : d->W - 1;
+  long long rows = 0, branches = 0, tiles = 0;
+  for (int t = 0; t < d->num_trees; ++t) {
+    const long long T = d->trunk_len[t], P = d->prompt_len[t], B = d->num_branches[t];
+    if (T < 1 || P < 0 || P > T - 1 || B < 0) return SPECOPD_ERR_ARG;
+    const long long n = T + B * p->rows_per_branch;
+    p->row_base[t] = (int32_t)rows;
+    p->trunk_len[t] = (int32_t)T;
+    p->prompt_len[t] = (int32_t)P;
+    p->branch_base[t] = (int32_t)branches;
+    p->tile_base[t] = (int32_t)tiles;
+    rows += n;
+    branches += B;
+    tiles += (n + SPECOPD_TILE_ROWS - 1) / SPECOPD_TILE_ROWS;
+    if (rows > (1LL << 30) || branches * d->W > (1LL << 30)) return SPECOPD_ERR_SHAPE;
+  }
+  p->row_base[d->num_trees] = (int32_t)rows;
+  p->branch_base[d->num_trees] = (int32_t)branches;
+  p->tile_base[d->num_trees] = (int32_t)tiles;
+  p->total_branches = (int32_t)branches;
+  p->num_tiles = (int32_t)tiles;
+  return SPECOPD_OK;
+}
+
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? SPECOPD_OK : SPECOPD_ERR_CUDA; }
+
+size_t elem_size(specopd_dtype dt) { return dt == SPECOPD_BF16 ? 2 : 4; }
+
+struct OverlapLayout {
+  size_t mbits, lz2, ql, g, cnt, bsum, total;
+  int64_t mbits_ld;
+};
+
+OverlapLayout overlap_layout(int64_t rows, int64_t V, int64_t nb) {
+  OverlapLayout L;
+  L.mbits_ld = ((V + 7) / 8 + 15) / 16 * 16;
+  size_t off = 0;
+  L.mbits = off;
+  off = align_up(off + (size_t)rows * L.mbits_ld);
+  L.lz2 = off;
+  off = align_up(off + (size_t)rows * 4);
+  L.ql = off;
+  off = align_up(off + (size_t)rows * 4);
+  L.g = off;
+  off = align_up(off + (size_t)rows * 4);
+  L.cnt = off;
+  off = align_up(off + (size_t)(nb + 1) * 4);
+  L.bsum = off;
+  off = align_up(off + (size_t)nb * 8);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t specopd_tree_packed_rows(const specopd_tree_desc* desc) {
+  TreeParams p;
+  const int s = tree_params(desc, &p);
+  return s != SPECOPD_OK ? s : (int64_t)p.row_base[p.num_trees];
+}
+
+int64_t specopd_tree_num_tiles(const specopd_tree_desc* desc) {
+  TreeParams p;
+  const int s = tree_params(desc, &p);
+  return s != SPECOPD_OK ? s : (int64_t)p.num_tiles;
+}
+
+int64_t specopd_tree_num_predictions(const specopd_tree_desc* desc) {
+  TreeParams p;
+  const int s = tree_params(desc, &p);
+  return s != SPECOPD_OK ? s : (int64_t)p.total_branches * p.W;
+}
+
+int specopd_build_tree_mask(const specopd_tree_desc* desc, int32_t* pos, int32_t* trunk_limit,
+                            int32_t* branch_of, uint64_t* anc_bits, int32_t* pred_rows, int32_t* cu_rows,
+                            specopd_tile_meta* tile_meta, int32_t* status, specopd_stream_t stream) {
+  TreeParams local;
+  const int s = tree_params(desc, &local);
+  if (s != SPECOPD_OK) return s;
+  if (!pos || !trunk_limit || !branch_of || !anc_bits || !cu_rows || !tile_meta || !status) return SPECOPD_ERR_ARG;
+  if (local.total_branches > 0 && (!desc->anchors || !pred_rows)) return SPECOPD_ERR_ARG;
+  return cuda_status(launch_tree_mask(local, desc->anchors, pos, trunk_limit, branch_of, anc_bits, pred_rows,
+                                      cu_rows, tile_meta, status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int specopd_rope(const void* q, const void* k, void* q_out, void* k_out, specopd_dtype dtype, int64_t N, int Hq,
+                 int Hkv, int d, const int32_t* pos, float theta, specopd_stream_t stream) {
+  if (dtype != SPECOPD_F32 && dtype != SPECOPD_BF16) return SPECOPD_ERR_DTYPE;
+  if (N < 0 || Hq < 1 || Hkv < 1 || d < 4 || d > 256 || d % 4) return SPECOPD_ERR_SHAPE;
+  if (N > 0 && (!q || !k || !q_out || !k_out || !pos)) return SPECOPD_ERR_ARG;
+  if (!(theta > 0.f) || !std::isfinite(theta)) return SPECOPD_ERR_ARG;
+  return cuda_status(
+      launch_rope(q, k, q_out, k_out, dtype, N, Hq, Hkv, d, pos, theta, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t specopd_attention_workspace_bytes(specopd_dtype dtype, int64_t N, int Hq, int Hkv, int d) {
+  if (N <= 0 || Hq < 1 || Hkv < 1 || d < 1) return 0;
+  const size_t e = elem_size(dtype);
+  return align_up((size_t)N * Hq * d * e) + align_up((size_t)N * Hkv * d * e);
+}
+
+int specopd_tree_attention(const void* q, const void* k, const void* v, void* out, specopd_dtype dtype,
+                           int64_t N, int Hq, int Hkv, int d, float rope_theta, float softmax_scale,
+                           const int32_t* pos, const int32_t* trunk_limit, const uint64_t* anc_bits,
+                           const specopd_tile_meta* tile_meta, int64_t num_tiles, void* workspace,
+                           size_t workspace_bytes, int32_t* status, specopd_stream_t stream) {
+  if (dtype != SPECOPD_F32 && dtype != SPECOPD_BF16) return SPECOPD_ERR_DTYPE;
+  if (N < 0 || num_tiles < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv) return SPECOPD_ERR_SHAPE;
+  if (d < 32 || d > 256 || d % 32) return SPECOPD_ERR_SHAPE;
+  if (N == 0) return SPECOPD_OK;
+  if (num_tiles < (N + SPECOPD_TILE_ROWS - 1) / SPECOPD_TILE_ROWS || num_tiles > N) return SPECOPD_ERR_SHAPE;
+  if (!q || !k || !v || !out || !pos || !trunk_limit || !anc_bits || !tile_meta || !status) return SPECOPD_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SPECOPD_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const void* qr = q;
+  const void* kr = k;
+  if (rope_theta > 0.f) {
+    if (!std::isfinite(rope_theta)) return SPECOPD_ERR_ARG;
+    const size_t need = specopd_attention_workspace_bytes(dtype, N, Hq, Hkv, d);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) % kAlign))
+      return SPECOPD_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    void* qo = ws;
+    void* ko = ws + align_up((size_t)N * Hq * d * elem_size(dtype));
+    const int rs = specopd_rope(q, k, qo, ko, dtype, N, Hq, Hkv, d, pos, rope_theta, stream);
+    if (rs != SPECOPD_OK) return rs;
+    qr = qo;
+    kr = ko;
+  }
+  AttnArgs a;
+  a.q = qr;
+  a.k = kr;
+  a.v = v;
+  a.out = out;
+  a.N = N;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.d = d;
+  a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)d);
+  a.pos = pos;
+  a.trunk_limit = trunk_limit;
+  a.anc_bits = anc_bits;
+  a.meta = tile_meta;
+  a.num_tiles = num_tiles;
+  a.status = status;
+  if (dtype == SPECOPD_BF16 && d == 128) return cuda_status(launch_tree_attention_sm100(a, st));
+  return cuda_status(launch_tree_attention_simt(a, dtype, st));
+}
+
+size_t specopd_overlap_workspace_bytes(int64_t rows, int64_t V, int64_t num_branches) {
+  if (rows < 0 || V < 1 || num_branches < 0) return 0;
+  return overlap_layout(rows, V, num_branches).total;
+}
+
+static int check_logits(const void* draft, const void* teacher, specopd_dtype dtype, int64_t rows, int64_t V,
+                        int64_t ld_draft, int64_t ld_teacher) {
+  if (dtype != SPECOPD_F32 && dtype != SPECOPD_BF16) return SPECOPD_ERR_DTYPE;
+  if (rows < 0 || V < 1 || ld_draft < V || ld_teacher < V) return SPECOPD_ERR_SHAPE;
+  if (V > (1LL << 20)) return SPECOPD_ERR_SHAPE;
+  if (rows > 0 && (!draft || !teacher)) return SPECOPD_ERR_ARG;
+  const size_t e = elem_size(dtype);
+  if (!aligned16(draft) || !aligned16(teacher) || (ld_draft * e) % 16 || (ld_teacher * e) % 16)
+    return SPECOPD_ERR_ALIGN;
+  return SPECOPD_OK;
+}
+
+int specopd_tv_overlap(const void* draft, const void* teacher, specopd_dtype dtype, int64_t rows, int64_t V,
+                       int64_t ld_draft, int64_t ld_teacher, float* alpha, float* q_less, float* lse_draft,
+                       float* lse_teacher, int32_t* status, specopd_stream_t stream) {
+  const int c = check_logits(draft, teacher, dtype, rows, V, ld_draft, ld_teacher);
+  if (c != SPECOPD_OK) return c;
+  if (rows == 0) return SPECOPD_OK;
+  if (!alpha || !status) return SPECOPD_ERR_ARG;
+  OverlapArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.draft = draft;
+  a.teacher = teacher;
+  a.ld_draft = ld_draft;
+  a.ld_teacher = ld_teacher;
+  a.rows = rows;
+  a.V = V;
+  a.alpha = alpha;
+  a.q_less = q_less;
+  a.lse_draft = lse_draft;
+  a.lse_teacher = lse_teacher;
+  a.status = status;
+  return cuda_status(launch_tv_stats(a, dtype, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int specopd_e2e_tv_loss(const float* alpha, int64_t num_branches, int W, double count, float* loss,
+                        float* grad_alpha, specopd_stream_t stream) {
+  if (num_branches < 0 || W < 1 || W > SPECOPD_MAX_W) return SPECOPD_ERR_SHAPE;
+  if (!loss || (num_branches > 0 && !alpha)) return SPECOPD_ERR_ARG;
+  if (!(count <= 0.0) && !std::isfinite(count)) return SPECOPD_ERR_ARG;
+  const double n = count > 0.0 ? count : (double)num_branches * W;
+  const double inv = n > 0.0 ? 1.0 / n : 0.0;
+  return cuda_status(
+      launch_e2e_loss(alpha, num_branches, W, inv, loss, grad_alpha, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int specopd_tv_overlap_e2e(const void* draft, const void* teacher, specopd_dtype dtype, int64_t rows, int64_t V,
+                           int64_t ld_draft, int64_t ld_teacher, int64_t num_branches, int W, double count,
+                           float* alpha, float* loss, float* grad_draft, int64_t ld_grad, void* workspace,
+                           size_t workspace_bytes, int32_t* status, specopd_stream_t stream) {
+  const int c = check_logits(draft, teacher, dtype, rows, V, ld_draft, ld_teacher);
+  if (c != SPECOPD_OK) return c;
+  if (W < 1 || W > SPECOPD_MAX_W || num_branches < 0 || rows != num_branches * W) return SPECOPD_ERR_SHAPE;
+  if (!loss || !status) return SPECOPD_ERR_ARG;
+  if (!(count <= 0.0) && !std::isfinite(count)) return SPECOPD_ERR_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (rows == 0) return cuda_status(cudaMemsetAsync(loss, 0, sizeof(float), st));
+  if (!alpha) return SPECOPD_ERR_ARG;
+  if (grad_draft && (ld_grad < V || !aligned16(grad_draft) || (ld_grad * 4) % 16)) return SPECOPD_ERR_ALIGN;
+  const OverlapLayout L = overlap_layout(rows, V, num_branches);
+  if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) % kAlign))
+    return SPECOPD_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const double n = count > 0.0 ? count : (double)rows;
+  OverlapArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.draft = draft;
+  a.teacher = teacher;
+  a.ld_draft = ld_draft;
+  a.ld_teacher = ld_teacher;
+  a.rows = rows;
+  a.V = V;
+  a.alpha = alpha;
+  a.mbits = grad_draft ? ws + L.mbits : nullptr;
+  a.mbits_ld = L.mbits_ld;
+  a.lz2 = reinterpret_cast<float*>(ws + L.lz2);
+  a.ql = reinterpret_cast<float*>(ws + L.ql);
+  a.g = reinterpret_cast<float*>(ws + L.g);
+  a.branch_cnt = reinterpret_cast<uint32_t*>(ws + L.cnt);
+  a.branch_sum = reinterpret_cast<double*>(ws + L.bsum);
+  a.loss = loss;
+  a.W = W;
+  a.num_branches = num_branches;
+  a.inv_count = 1.0 / n;
+  a.grad = grad_draft;
+  a.ld_grad = ld_grad;
+  a.status = status;
+  cudaError_t e = cudaMemsetAsync(a.branch_cnt, 0, (size_t)(num_branches + 1) * 4, st);
+  if (e != cudaSuccess) return SPECOPD_ERR_CUDA;
+  e = launch_tv_stats(a, dtype, st);
+  if (e != cudaSuccess) return SPECOPD_ERR_CUDA;
+  if (grad_draft) {
+    e = launch_tv_grad(a, dtype, st);
+    if (e != cudaSuccess) return SPECOPD_ERR_CUDA;
+  }
+  return SPECOPD_OK;
+}
+
+const char* specopd_status_string(int status) {
+  switch (status) {
+    case SPECOPD_OK: return "ok";
+    case SPECOPD_ERR_ARG: return "invalid argument";
+    case SPECOPD_ERR_SHAPE: return "unsupported shape";
+    case SPECOPD_ERR_DTYPE: return "unsupported dtype";
+    case SPECOPD_ERR_CUDA: return "CUDA launch failed";
+    case SPECOPD_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case SPECOPD_ERR_ALIGN: return "pointer or leading dimension not 16-byte aligned";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,85 @@
+// Internal launch interfaces shared by the kernel files and the C ABI layer.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/specopd.h"
+
+namespace specopd {
+
+// Per-tree layout of a batch, computed on the host and passed by value.
+struct TreeParams {
+  int32_t num_trees;
+  int32_t W;
+  int32_t rows_per_branch;
+  int32_t total_branches;
+  int32_t num_tiles;
+  int32_t row_base[SPECOPD_MAX_TREES + 1];     // first packed row of each tree
+  int32_t trunk_len[SPECOPD_MAX_TREES];
+  int32_t prompt_len[SPECOPD_MAX_TREES];
+  int32_t branch_base[SPECOPD_MAX_TREES + 1];  // first global branch id of each tree
+  int32_t tile_base[SPECOPD_MAX_TREES + 1];    // first query tile of each tree
+};
+
+cudaError_t launch_tree_mask(const TreeParams& p, const int32_t* anchors, int32_t* pos, int32_t* trunk_limit,
+                             int32_t* branch_of, uint64_t* anc_bits, int32_t* pred_rows, int32_t* cu_rows,
+                             specopd_tile_meta* tile_meta, int32_t* status, cudaStream_t stream);
+
+cudaError_t launch_rope(const void* q, const void* k, void* q_out, void* k_out, specopd_dtype dtype, int64_t N,
+                        int Hq, int Hkv, int d, const int32_t* pos, float theta, cudaStream_t stream);
+
+struct AttnArgs {
+  const void* q;  // rotated
+  const void* k;  // rotated
+  const void* v;
+  void* out;
+  int64_t N;
+  int Hq, Hkv, d;
+  float scale;
+  const int32_t* pos;
+  const int32_t* trunk_limit;
+  const uint64_t* anc_bits;
+  const specopd_tile_meta* meta;
+  int64_t num_tiles;
+  int32_t* status;
+};
+
+// tcgen05 kernel: bf16, d = 128.
+cudaError_t launch_tree_attention_sm100(const AttnArgs& a, cudaStream_t stream);
+// SIMT kernel: fp32 or bf16, d multiple of 32 up to 256.
+cudaError_t launch_tree_attention_simt(const AttnArgs& a, specopd_dtype dtype, cudaStream_t stream);
+
+struct OverlapArgs {
+  const void* draft;
+  const void* teacher;
+  int64_t ld_draft, ld_teacher;
+  int64_t rows, V;
+  // outputs of the statistics pass
+  float* alpha;
+  float* q_less;     // nullable
+  float* lse_draft;  // nullable (natural log)
+  float* lse_teacher;
+  // fused path (all null in the unfused entry point)
+  uint8_t* mbits;    // [rows, mbits_ld] strict-less bits
+  int64_t mbits_ld;
+  float* lz2;        // [rows] draft normaliser, log2 units
+  float* ql;         // [rows] q_less
+  float* g;          // [rows] dL/dalpha
+  uint32_t* branch_cnt;  // [num_branches + 1], zero on entry
+  double* branch_sum;    // [num_branches]
+  float* loss;
+  int W;
+  int64_t num_branches;
+  double inv_count;
+  // gradient output (fused path)
+  float* grad;
+  int64_t ld_grad;
+  int32_t* status;
+};
+
+cudaError_t launch_tv_stats(const OverlapArgs& a, specopd_dtype dtype, cudaStream_t stream);
+cudaError_t launch_tv_grad(const OverlapArgs& a, specopd_dtype dtype, cudaStream_t stream);
+cudaError_t launch_e2e_loss(const float* alpha, int64_t num_branches, int W, double inv_count, float* loss,
+                            float* grad_alpha, cudaStream_t stream);
+
+}  // namespace specopd

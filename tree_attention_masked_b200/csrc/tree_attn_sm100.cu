@@ -1,0 +1,397 @@
+// K3: tree-masked GQA attention on the 5th-generation tensor cores (sm_100a).
+//
+// SpecOPD listing, Fig 3: one packed pass scores every row of a proposal tree;
+// packed queries share the trunk's keys and values while each row attends only
+// to itself and its ancestors.  The pages give no kernel; this design is new:
+//
+//  * a CTA owns one 128-row query tile of one tree and two query heads that
+//    read the same KV head (GQA), so every K/V tile it loads feeds two heads;
+//  * the columns it visits are the tile's trunk span [tree_base, trunk_hi)
+//    followed by its branch span [br_lo, br_hi) (both from the mask builder);
+//    column blocks outside them are never loaded.  Trunk blocks below
+//    `trunk_full` are seen by every row and skip masking entirely;
+//  * warp 0 issues TMA tile loads (no multicast) into a 4-slot K/V ring,
+//    one thread of warp 1 issues tcgen05.mma: S = Q K^T into TMEM, then
+//    O += P V with P read straight from TMEM;
+//  * warps 4-7 and 8-11 (one warpgroup per query head) own one query row per
+//    thread: they read S from TMEM, mask, run the online softmax in base 2,
+//    write P (bf16) back over S, and rescale O in TMEM only when the running
+//    maximum grows by more than 2^8 (the stale maximum is exact: the same
+//    reference enters numerator and denominator);
+//  * TMEM: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512) fp32 columns;
+//    P_t occupies the first 64 columns of S_t as packed bf16 pairs.
+//
+// All waits are bounded (see ptx.cuh); a wait that gives up sets
+// SPECOPD_FLAG_TIMEOUT, and the CTA drains its copies and MMAs, frees TMEM
+// and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace specopd {
+namespace {
+
+constexpr int kBM = 128;             // query rows per tile
+constexpr int kBN = 128;             // key columns per block
+constexpr int kHD = 128;             // head dim
+constexpr int kSlots = 4;            // K/V ring slots
+constexpr int kBoxBytes = 128 * 64 * 2;   // one [128 rows][64 elems] swizzled box
+constexpr int kTileBytes = 2 * kBoxBytes; // [128][128] bf16
+constexpr int kThreads = 384;
+constexpr float kRescaleLog2 = 8.0f;
+
+struct __align__(1024) Smem {
+  uint8_t q[2][kTileBytes];
+  uint8_t kv[kSlots][kTileBytes];
+  uint64_t q_full;
+  uint64_t kv_full[kSlots];
+  uint64_t kv_empty[kSlots];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_done[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct Params {
+  __nv_bfloat16* out;
+  const int32_t* pos;
+  const int32_t* trunk_limit;
+  const uint64_t* anc_bits;
+  const specopd_tile_meta* meta;
+  int num_tiles;
+  int Hq, Hkv, G, pairs;
+  float scale_log2;
+  int32_t* status;
+};
+
+// bounded wait used only to drain in-flight work before exit: ignores the
+// abort flag, still gives up after the time limit.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitLimitCycles) return;
+  }
+}
+
+__device__ __forceinline__ int block_col(const specopd_tile_meta& m, int n_trunk, int j) {
+  return j < n_trunk ? m.tree_base + j * kBN : m.br_lo + (j - n_trunk) * kBN;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    tree_attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                           const __grid_constant__ CUtensorMap tmV, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem* sm = reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item: (tile, kv head, head pair); expensive tiles (late rows) first
+  const int items_per_tile = p.Hkv * p.pairs;
+  const int w = blockIdx.x;
+  const int tile = p.num_tiles - 1 - w / items_per_tile;
+  const int rem = w % items_per_tile;
+  const int kvh = rem / p.pairs;
+  const int pair = rem % p.pairs;
+  const int h0 = kvh * p.G + 2 * pair;
+  const int nq = (2 * pair + 1 < p.G) ? 2 : 1;
+  const specopd_tile_meta m = p.meta[tile];
+  const int n_trunk = (m.trunk_hi - m.tree_base + kBN - 1) / kBN;
+  const int n_br = (m.br_hi > m.br_lo) ? (m.br_hi - m.br_lo + kBN - 1) / kBN : 0;
+  const int nblk = n_trunk + n_br;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sm->q_full, 1);
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(&sm->kv_full[s], 1);
+      mbar_init(&sm->kv_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&sm->s_full[t], 1);
+      mbar_init(&sm->p_full[t], 128);
+      mbar_init(&sm->o_done[t], 1);
+    }
+    mbar_init(&sm->mma_done, 1);
+    sm->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(&sm->tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 32) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm->tmem_base;
+  volatile int* abort_flag = &sm->abort_flag;
+
+  if (warp == 0) {
+    // ================= TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&sm->q_full, nq * kTileBytes);
+      for (int t = 0; t < nq; ++t)
+        for (int hx = 0; hx < 2; ++hx)
+          tma_load_3d(sm->q[t] + hx * kBoxBytes, &tmQ, hx * 64, h0 + t, m.row_start, &sm->q_full);
+      int last_n[kSlots] = {-1, -1, -1, -1};
+      for (int n = 0; n < 2 * nblk; ++n) {
+        const int slot = n % kSlots;
+        if (n >= kSlots && !mbar_wait(&sm->kv_empty[slot], ((n / kSlots) - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&sm->kv_full[slot], kTileBytes);
+        const int c0 = block_col(m, n_trunk, n >> 1);
+        const CUtensorMap* tm = (n & 1) ? &tmV : &tmK;
+        tma_load_3d(sm->kv[slot], tm, 0, kvh, c0, &sm->kv_full[slot]);
+        tma_load_3d(sm->kv[slot] + kBoxBytes, tm, 64, kvh, c0, &sm->kv_full[slot]);
+        last_n[slot] = n;
+      }
+      // every issued copy must land before the CTA may exit
+      drain_wait(&sm->q_full, 0);
+      for (int s = 0; s < kSlots; ++s)
+        if (last_n[s] >= 0) drain_wait(&sm->kv_full[s], (last_n[s] / kSlots) & 1);
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer (one thread)
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, kHD, true);
+      auto issue_s = [&](int j, int t) {
+        const uint32_t kb = smem_u32(sm->kv[(2 * j) % kSlots]);
+        const uint32_t qb = smem_u32(sm->q[t]);
+#pragma unroll
+        for (int s = 0; s < kHD / 16; ++s) {
+          const uint32_t off = (s >> 2) * kBoxBytes + (s & 3) * 32;
+          mma_ss(tmem + t * 128, smem_desc_sw128(qb + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024),
+                 idesc_qk, s > 0);
+        }
+        mma_commit(&sm->s_full[t]);
+      };
+      auto issue_pv = [&](int j, int t) {
+        const uint32_t vb = smem_u32(sm->kv[(2 * j + 1) % kSlots]);
+#pragma unroll
+        for (int s = 0; s < kBN / 16; ++s) {
+          mma_ts(tmem + 256 + t * 128, tmem + t * 128 + s * 8, smem_desc_sw128(vb + s * 2048, kBoxBytes, 1024),
+                 idesc_pv, (j > 0 || s > 0) ? 1u : 0u);
+        }
+        mma_commit(&sm->o_done[t]);
+      };
+      bool ok = mbar_wait(&sm->q_full, 0, abort_flag);
+      if (ok) ok = mbar_wait(&sm->kv_full[0], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < nq; ++t) issue_s(0, t);
+        mma_commit(&sm->kv_empty[0]);
+      }
+      for (int j = 0; ok && j < nblk; ++j) {
+        const int nv = 2 * j + 1;
+        if (!mbar_wait(&sm->kv_full[nv % kSlots], (nv / kSlots) & 1, abort_flag)) break;
+        const bool next = j + 1 < nblk;
+        const int nk = 2 * (j + 1);
+        for (int t = 0; t < nq; ++t) {
+          if (!mbar_wait(&sm->p_full[t], j & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(j, t);
+          if (next) {
+            if (t == 0 && !mbar_wait(&sm->kv_full[nk % kSlots], (nk / kSlots) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(j + 1, t);
+          }
+        }
+        if (!ok) break;
+        mma_commit(&sm->kv_empty[nv % kSlots]);
+        if (next) mma_commit(&sm->kv_empty[nk % kSlots]);
+      }
+      // all MMAs must finish before TMEM and shared memory are released
+      mma_commit(&sm->mma_done);
+      drain_wait(&sm->mma_done, 0);
+    }
+  } else if (warp >= 4) {
+    // ================= softmax: one warpgroup per query head, one row per thread
+    const int t = (warp - 4) >> 2;
+    if (t < nq) {
+      const int quad = warp & 3;
+      const int rloc = quad * 32 + lane;
+      const int r = m.row_start + rloc;
+      const bool valid = r < m.row_end;
+      int lim = m.tree_base, bstart = 0;
+      uint64_t bits = 0;
+      if (valid) {
+        const int tl = p.trunk_limit[r];
+        lim = m.tree_base + tl;
+        bstart = r - (p.pos[r] - tl) + 1;
+        bits = p.anc_bits[r];
+      }
+      const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+      const uint32_t s_col = t * 128;
+      const uint32_t o_col = 256 + t * 128;
+      float m_use = -INFINITY;
+      float l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < nblk; ++j) {
+        if (!mbar_wait_warp(&sm->s_full[t], j & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sr[128];
+        tmem_ld32(trow + s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(trow + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld32(trow + s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+        tmem_ld32(trow + s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+        tmem_ld_wait();
+        float* s = reinterpret_cast<float*>(sr);
+        const int c0 = block_col(m, n_trunk, j);
+        const bool trunk = j < n_trunk;
+        if (!(trunk && c0 + kBN <= m.trunk_full)) {
+          if (trunk) {
+#pragma unroll
+            for (int e = 0; e < 128; ++e)
+              if (c0 + e > lim) s[e] = -INFINITY;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 128; ++e) {
+              const unsigned off = (unsigned)(c0 + e - bstart);
+              const bool vis = off < 64u && ((bits >> off) & 1ull);
+              if (!vis) s[e] = -INFINITY;
+            }
+          }
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 128; ++e) mx = fmaxf(mx, s[e]);
+        const float m_new = fmaxf(m_use, mx * p.scale_log2);
+        float corr = 1.f;
+        bool rescale = false;
+        if (m_use == -INFINITY || m_new > m_use + kRescaleLog2) {
+          corr = ex2(m_use - m_new);
+          m_use = m_new;
+          rescale = j > 0;
+        }
+        const float m_eff = (m_use == -INFINITY) ? 0.f : m_use;
+        float rowsum = 0.f;
+        uint32_t pk[64];
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+          const float p0 = ex2(fmaf(s[2 * e], p.scale_log2, -m_eff));
+          const float p1 = ex2(fmaf(s[2 * e + 1], p.scale_log2, -m_eff));
+          rowsum += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        l = l * corr + rowsum;
+        tmem_st32(trow + s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+        tmem_st32(trow + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        tmem_st_wait();
+        if (__any_sync(0xffffffffu, rescale)) {
+          // O may be touched only after the previous P.V has finished
+          if (!mbar_wait_warp(&sm->o_done[t], (j - 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t orr[32];
+            tmem_ld32(trow + o_col + c * 32, orr);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * corr);
+            tmem_st32(trow + o_col + c * 32, orr);
+          }
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        mbar_arrive(&sm->p_full[t]);
+      }
+      if (ok && mbar_wait_warp(&sm->o_done[t], (nblk - 1) & 1, abort_flag)) {
+        tc_fence_after();
+        const float inv = 1.f / l;
+        __nv_bfloat16* orow = p.out + ((long long)r * p.Hq + h0 + t) * kHD;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t orr[32];
+          tmem_ld32(trow + o_col + c * 32, orr);
+          tmem_ld_wait();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv, __uint_as_float(orr[2 * e + 1]) * inv);
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0 && sm->abort_flag) atomicOr(reinterpret_cast<unsigned*>(p.status), SPECOPD_FLAG_TIMEOUT);
+}
+
+// ------------------------------------------------------------------ host side
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn get_encode() {
+  static EncodeFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(ptr);
+  }
+  return fn;
+}
+
+// [N, H, 128] bf16 -> 3-D map, box [64 elems][1 head][128 rows], 128-byte swizzle
+bool make_map(CUtensorMap* tm, const void* ptr, int64_t N, int H) {
+  EncodeFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kHD, (cuuint64_t)H, (cuuint64_t)N};
+  cuuint64_t strides[2] = {(cuuint64_t)kHD * 2, (cuuint64_t)H * kHD * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_tree_attention_sm100(const AttnArgs& a, cudaStream_t stream) {
+  if (a.num_tiles == 0) return cudaSuccess;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, a.q, a.N, a.Hq) || !make_map(&tk, a.k, a.N, a.Hkv) || !make_map(&tv, a.v, a.N, a.Hkv))
+    return cudaErrorInvalidValue;
+  Params p;
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.pos = a.pos;
+  p.trunk_limit = a.trunk_limit;
+  p.anc_bits = a.anc_bits;
+  p.meta = a.meta;
+  p.num_tiles = (int)a.num_tiles;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.G = a.Hq / a.Hkv;
+  p.pairs = (p.G + 1) / 2;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.status = a.status;
+  const size_t smem = sizeof(Smem) + 1024;
+  cudaError_t e =
+      cudaFuncSetAttribute(tree_attn_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const long long grid = (long long)a.num_tiles * p.Hkv * p.pairs;
+  tree_attn_sm100_kernel<<<(unsigned)grid, kThreads, smem, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace specopd

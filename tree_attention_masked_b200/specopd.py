@@ -1,0 +1,203 @@
+"""ctypes binding of libspecopd.so (include/specopd.h).
+
+Argument marshalling only: every function here forwards torch tensors' device
+pointers and the current CUDA stream to the C ABI of the same name and raises
+if the call returns an error.  All arithmetic runs in the library's kernels.
+Importing this module without a built library raises immediately; there is no
+fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libspecopd.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m tree_attention_masked_b200.build`")
+_lib = ctypes.CDLL(LIB_PATH)
+
+F32, BF16 = 0, 1
+TILE_ROWS = 128
+MAX_W = 64
+MAX_TREES = 512
+FLAG_ANCHOR, FLAG_NONFINITE, FLAG_TIMEOUT = 1, 2, 4
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int32
+_int = ctypes.c_int
+_f32 = ctypes.c_float
+_f64 = ctypes.c_double
+_sz = ctypes.c_size_t
+
+
+class TreeDesc(ctypes.Structure):
+    _fields_ = [("num_trees", _i32), ("W", _i32), ("pack_terminal", _i32),
+                ("trunk_len", ctypes.POINTER(_i32)), ("prompt_len", ctypes.POINTER(_i32)),
+                ("num_branches", ctypes.POINTER(_i32)), ("anchors", _vp)]
+
+
+_desc_p = ctypes.POINTER(TreeDesc)
+
+
+def _sig(name, res, *args):
+    f = getattr(_lib, name)
+    f.restype = res
+    f.argtypes = list(args)
+    return f
+
+
+_c = {
+    "specopd_tree_packed_rows": _sig("specopd_tree_packed_rows", _i64, _desc_p),
+    "specopd_tree_num_tiles": _sig("specopd_tree_num_tiles", _i64, _desc_p),
+    "specopd_tree_num_predictions": _sig("specopd_tree_num_predictions", _i64, _desc_p),
+    "specopd_build_tree_mask": _sig("specopd_build_tree_mask", _int, _desc_p, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                    _vp, _vp),
+    "specopd_rope": _sig("specopd_rope", _int, _vp, _vp, _vp, _vp, _int, _i64, _int, _int, _int, _vp, _f32, _vp),
+    "specopd_attention_workspace_bytes": _sig("specopd_attention_workspace_bytes", _sz, _int, _i64, _int, _int,
+                                              _int),
+    "specopd_tree_attention": _sig("specopd_tree_attention", _int, _vp, _vp, _vp, _vp, _int, _i64, _int, _int, _int,
+                                   _f32, _f32, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp, _vp),
+    "specopd_overlap_workspace_bytes": _sig("specopd_overlap_workspace_bytes", _sz, _i64, _i64, _i64),
+    "specopd_tv_overlap": _sig("specopd_tv_overlap", _int, _vp, _vp, _int, _i64, _i64, _i64, _i64, _vp, _vp, _vp,
+                               _vp, _vp, _vp),
+    "specopd_e2e_tv_loss": _sig("specopd_e2e_tv_loss", _int, _vp, _i64, _int, _f64, _vp, _vp, _vp),
+    "specopd_tv_overlap_e2e": _sig("specopd_tv_overlap_e2e", _int, _vp, _vp, _int, _i64, _i64, _i64, _i64, _i64,
+                                   _int, _f64, _vp, _vp, _vp, _i64, _vp, _sz, _vp, _vp),
+    "specopd_status_string": _sig("specopd_status_string", ctypes.c_char_p, _int),
+}
+
+EXPORTED = sorted(_c)
+
+
+class SpecopdError(RuntimeError):
+    pass
+
+
+def _check(name: str, rc: int) -> None:
+    if rc != 0:
+        raise SpecopdError(f"{name}: {_c['specopd_status_string'](rc).decode()} ({rc})")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise SpecopdError(f"unsupported dtype {t.dtype}")
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise SpecopdError("tensors must be contiguous")
+
+
+class Trees:
+    """A batch of proposal trees: host shape arrays plus the device anchors."""
+
+    def __init__(self, trunk_len: Sequence[int], prompt_len: Sequence[int], num_branches: Sequence[int], W: int,
+                 anchors: torch.Tensor, pack_terminal: bool = True):
+        n = len(trunk_len)
+        self._t = (_i32 * n)(*trunk_len)
+        self._p = (_i32 * n)(*prompt_len)
+        self._b = (_i32 * n)(*num_branches)
+        self.anchors = anchors
+        self.desc = TreeDesc(n, W, 1 if pack_terminal else 0, self._t, self._p, self._b,
+                             anchors.data_ptr() if anchors.numel() else None)
+        self.W = W
+        self.num_trees = n
+
+    def ref(self):
+        return ctypes.byref(self.desc)
+
+
+def specopd_tree_packed_rows(trees: Trees) -> int:
+    n = _c["specopd_tree_packed_rows"](trees.ref())
+    if n < 0:
+        _check("specopd_tree_packed_rows", n)
+    return n
+
+
+def specopd_tree_num_tiles(trees: Trees) -> int:
+    n = _c["specopd_tree_num_tiles"](trees.ref())
+    if n < 0:
+        _check("specopd_tree_num_tiles", n)
+    return n
+
+
+def specopd_tree_num_predictions(trees: Trees) -> int:
+    n = _c["specopd_tree_num_predictions"](trees.ref())
+    if n < 0:
+        _check("specopd_tree_num_predictions", n)
+    return n
+
+
+def specopd_build_tree_mask(trees: Trees, pos, trunk_limit, branch_of, anc_bits, pred_rows, cu_rows, tile_meta,
+                            status, stream=None) -> None:
+    _contig(pos, trunk_limit, branch_of, anc_bits, pred_rows, cu_rows, tile_meta, status)
+    _check("specopd_build_tree_mask", _c["specopd_build_tree_mask"](
+        trees.ref(), _ptr(pos), _ptr(trunk_limit), _ptr(branch_of), _ptr(anc_bits), _ptr(pred_rows),
+        _ptr(cu_rows), _ptr(tile_meta), _ptr(status), _stream(stream)))
+
+
+def specopd_rope(q, k, q_out, k_out, pos, theta: float, stream=None) -> None:
+    _contig(q, k, q_out, k_out, pos)
+    N, Hq, d = q.shape
+    _check("specopd_rope", _c["specopd_rope"](
+        _ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), _dtype(q), N, Hq, k.shape[1], d, _ptr(pos), theta,
+        _stream(stream)))
+
+
+def specopd_attention_workspace_bytes(dtype: int, N: int, Hq: int, Hkv: int, d: int) -> int:
+    return _c["specopd_attention_workspace_bytes"](dtype, N, Hq, Hkv, d)
+
+
+def specopd_tree_attention(q, k, v, out, pos, trunk_limit, anc_bits, tile_meta, num_tiles: int, rope_theta: float,
+                           softmax_scale: float, workspace, status, stream=None) -> None:
+    _contig(q, k, v, out, pos, trunk_limit, anc_bits, tile_meta, status)
+    N, Hq, d = q.shape
+    wb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("specopd_tree_attention", _c["specopd_tree_attention"](
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype(q), N, Hq, k.shape[1], d, rope_theta, softmax_scale,
+        _ptr(pos), _ptr(trunk_limit), _ptr(anc_bits), _ptr(tile_meta), num_tiles, _ptr(workspace), wb,
+        _ptr(status), _stream(stream)))
+
+
+def specopd_overlap_workspace_bytes(rows: int, V: int, num_branches: int) -> int:
+    return _c["specopd_overlap_workspace_bytes"](rows, V, num_branches)
+
+
+def specopd_tv_overlap(draft, teacher, V: int, alpha, q_less, lse_draft, lse_teacher, status, stream=None) -> None:
+    _check("specopd_tv_overlap", _c["specopd_tv_overlap"](
+        _ptr(draft), _ptr(teacher), _dtype(draft), draft.shape[0], V, draft.stride(0), teacher.stride(0),
+        _ptr(alpha), _ptr(q_less), _ptr(lse_draft), _ptr(lse_teacher), _ptr(status), _stream(stream)))
+
+
+def specopd_e2e_tv_loss(alpha, num_branches: int, W: int, count: float, loss, grad_alpha=None, stream=None) -> None:
+    _check("specopd_e2e_tv_loss", _c["specopd_e2e_tv_loss"](
+        _ptr(alpha), num_branches, W, count, _ptr(loss), _ptr(grad_alpha), _stream(stream)))
+
+
+def specopd_tv_overlap_e2e(draft, teacher, V: int, num_branches: int, W: int, count: float, alpha, loss, grad,
+                           workspace, status, stream=None) -> None:
+    wb = workspace.numel() * workspace.element_size()
+    _check("specopd_tv_overlap_e2e", _c["specopd_tv_overlap_e2e"](
+        _ptr(draft), _ptr(teacher), _dtype(draft), draft.shape[0], V, draft.stride(0), teacher.stride(0),
+        num_branches, W, count, _ptr(alpha), _ptr(loss), _ptr(grad), grad.stride(0) if grad is not None else 0,
+        _ptr(workspace), wb, _ptr(status), _stream(stream)))
