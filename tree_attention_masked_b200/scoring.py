@@ -57,11 +57,15 @@ class ScoringStep:
         ldt = S.BF16 if dtype == torch.bfloat16 else S.F32
         ws = S.specopd_attention_workspace_bytes(ldt, N, Hq, Hkv, d)
         self.attn_ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
-        self.draft = torch.empty(R, vocab, dtype=dtype, device=dev)
-        self.teacher = torch.empty(R, vocab, dtype=dtype, device=dev)
+        # logit rows start on 16-byte boundaries: pad the row stride when needed
+        es = torch.tensor([], dtype=dtype).element_size()
+        ld = -(-vocab * es // 16) * 16 // es
+        ldg = -(-vocab // 4) * 4
+        self.draft = torch.empty(R, ld, dtype=dtype, device=dev)[:, :vocab]
+        self.teacher = torch.empty(R, ld, dtype=dtype, device=dev)[:, :vocab]
         self.alpha = torch.empty(max(R, 1), dtype=torch.float32, device=dev)
         self.loss = torch.zeros(1, dtype=torch.float32, device=dev)
-        self.grad = torch.empty(R, vocab, dtype=torch.float32, device=dev) if with_grad else None
+        self.grad = torch.empty(R, ldg, dtype=torch.float32, device=dev)[:, :vocab] if with_grad else None
         ows = S.specopd_overlap_workspace_bytes(R, vocab, nb)
         self.ov_ws = torch.empty(max(ows, 256), dtype=torch.uint8, device=dev)
 
