@@ -51,10 +51,16 @@ inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? SPECOPD_OK : S
 size_t elem_size(specopd_dtype dt) { return dt == SPECOPD_BF16 ? 2 : 4; }
 
 struct OverlapLayout {
-  size_t mbits, lz2, ql, g, cnt, bsum, total;
+  size_t mbits, lz2, ql, g, counters, bsum, total;
+  size_t counters_bytes;
   int64_t mbits_ld;
 };
 
+// Workspace of the fused overlap pass (all regions 256-byte aligned):
+//   mbits     [rows][mbits_ld]  one bit per logit, [q < p]
+//   lz2, ql, g [rows]           draft normaliser (base 2), q_less, dL/dalpha
+//   counters  branch arrivals [nb] + branches done [1]
+//   bsum      [nb] doubles      each branch's share of L
 OverlapLayout overlap_layout(int64_t rows, int64_t V, int64_t nb) {
   OverlapLayout L;
   L.mbits_ld = ((V + 7) / 8 + 15) / 16 * 16;
@@ -67,8 +73,9 @@ OverlapLayout overlap_layout(int64_t rows, int64_t V, int64_t nb) {
   off = align_up(off + (size_t)rows * 4);
   L.g = off;
   off = align_up(off + (size_t)rows * 4);
-  L.cnt = off;
-  off = align_up(off + (size_t)(nb + 1) * 4);
+  L.counters = off;
+  L.counters_bytes = (size_t)(nb + 1) * 4;
+  off = align_up(off + L.counters_bytes);
   L.bsum = off;
   off = align_up(off + (size_t)nb * 8);
   L.total = off;
@@ -256,7 +263,8 @@ int specopd_tv_overlap_e2e(const void* draft, const void* teacher, specopd_dtype
   a.lz2 = reinterpret_cast<float*>(ws + L.lz2);
   a.ql = reinterpret_cast<float*>(ws + L.ql);
   a.g = reinterpret_cast<float*>(ws + L.g);
-  a.branch_cnt = reinterpret_cast<uint32_t*>(ws + L.cnt);
+  uint32_t* counters = reinterpret_cast<uint32_t*>(ws + L.counters);
+  a.branch_cnt = counters;  // [nb] arrivals per branch, then [1] branches done
   a.branch_sum = reinterpret_cast<double*>(ws + L.bsum);
   a.loss = loss;
   a.W = W;
@@ -265,7 +273,7 @@ int specopd_tv_overlap_e2e(const void* draft, const void* teacher, specopd_dtype
   a.grad = grad_draft;
   a.ld_grad = ld_grad;
   a.status = status;
-  cudaError_t e = cudaMemsetAsync(a.branch_cnt, 0, (size_t)(num_branches + 1) * 4, st);
+  cudaError_t e = cudaMemsetAsync(counters, 0, L.counters_bytes, st);
   if (e != cudaSuccess) return SPECOPD_ERR_CUDA;
   e = launch_tv_stats(a, dtype, st);
   if (e != cudaSuccess) return SPECOPD_ERR_CUDA;

@@ -78,6 +78,9 @@ struct OverlapArgs {
 };
 
 cudaError_t launch_tv_stats(const OverlapArgs& a, specopd_dtype dtype, cudaStream_t stream);
+// bf16 kernels (tv_bf16.cu); launch_tv_stats / launch_tv_grad route bf16 here
+cudaError_t launch_tv_stats_bf16(const OverlapArgs& a, cudaStream_t stream);
+cudaError_t launch_tv_grad_bf16(const OverlapArgs& a, cudaStream_t stream);
 cudaError_t launch_tv_grad(const OverlapArgs& a, specopd_dtype dtype, cudaStream_t stream);
 cudaError_t launch_e2e_loss(const float* alpha, int64_t num_branches, int W, double inv_count, float* loss,
                             float* grad_alpha, cudaStream_t stream);

@@ -1,0 +1,60 @@
+// Device helpers shared by the overlap kernels: base-2 log-sum-exp merging
+// and the per-row E2E-TV epilogue.
+#pragma once
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace specopd {
+
+// (m, s) pairs of a base-2 log-sum-exp: value = m + log2(s)
+__device__ __forceinline__ void lse_merge(float& m, float& s, float m2, float s2) {
+  const float mn = fmaxf(m, m2);
+  if (mn == -INFINITY) return;
+  s = s * ex2(m - mn) + s2 * ex2(m2 - mn);
+  m = mn;
+}
+
+// Row results and the E2E-TV epilogue.  Called by one thread per row after
+// the row's alpha and q_less are final: writes the per-row outputs, then the
+// last row of the branch to arrive forms the branch's prefix products,
+// dL/dalpha and its share of L, and the last branch forms L from the shares
+// in branch order.
+__device__ inline void row_epilogue(const OverlapArgs& a, long long row, float alpha, float qless, float lz2, float lt2) {
+  a.alpha[row] = alpha;
+  if (a.q_less) a.q_less[row] = qless;
+  if (a.lse_draft) a.lse_draft[row] = lz2 * 0.6931471805599453f;
+  if (a.lse_teacher) a.lse_teacher[row] = lt2 * 0.6931471805599453f;
+  if (a.lz2) a.lz2[row] = lz2;
+  if (a.ql) a.ql[row] = qless;
+  if (!a.branch_cnt) return;
+  const int W = a.W;
+  const long long b = row / W;
+  __threadfence();
+  const unsigned old = atomicAdd(&a.branch_cnt[b], 1u);
+  if (old != (unsigned)(W - 1)) return;
+  __threadfence();
+  const float* al_b = a.alpha + b * W;
+  double pre[SPECOPD_MAX_W + 1];
+  pre[0] = 1.0;
+  double share = 0.0;
+  for (int i = 1; i <= W; ++i) {
+    pre[i] = pre[i - 1] * (double)__ldcg(al_b + i - 1);
+    share += pre[i];
+  }
+  // S_i = 1 + alpha_{i+1} S_{i+1}, S_W = 1; g_i = -(1/count) pre_{i-1} S_i
+  double S = 1.0;
+  for (int i = W; i >= 1; --i) {
+    a.g[b * W + i - 1] = (float)(-a.inv_count * pre[i - 1] * S);
+    S = 1.0 + (double)__ldcg(al_b + i - 1) * S;
+  }
+  a.branch_sum[b] = share;
+  __threadfence();
+  const unsigned done = atomicAdd(&a.branch_cnt[a.num_branches], 1u);
+  if (done != (unsigned)(a.num_branches - 1)) return;
+  __threadfence();
+  double total = 0.0;
+  for (long long k = 0; k < a.num_branches; ++k) total += __ldcg(a.branch_sum + k);
+  *a.loss = (float)(1.0 - total * a.inv_count);
+}
+
+}  // namespace specopd

@@ -1,4 +1,5 @@
-// K4/K5: full-vocabulary overlap, E2E-TV loss and its gradient.
+// K4/K5: full-vocabulary overlap, E2E-TV loss and its gradient -- the generic
+// kernels, used for fp32 logits (bf16 logits take the kernels in tv_bf16.cu).
 //
 // daiwk.github.io write-up of SpecOPD, section "Equations":
 //   alpha_{b,i} = sum_v min(q(v), p(v)),
@@ -25,7 +26,10 @@
 //   dL/dz = g q (bit - q_less), zero outside the draft support.
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "internal.h"
+#include "overlap_common.cuh"
 #include "ptx.cuh"
 
 namespace specopd {
@@ -61,14 +65,6 @@ struct Elem<__nv_bfloat16> {
   }
   __device__ static float one(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 };
-
-// (m, s) pairs of a base-2 log-sum-exp: value = m + log2(s)
-__device__ __forceinline__ void lse_merge(float& m, float& s, float m2, float s2) {
-  const float mn = fmaxf(m, m2);
-  if (mn == -INFINITY) return;
-  s = s * ex2(m - mn) + s2 * ex2(m2 - mn);
-  m = mn;
-}
 
 struct StatSmem {
   float part[8];      // this CTA's partials, read by the cluster
@@ -286,46 +282,7 @@ __global__ void __launch_bounds__(kStatThreads) tv_stats_kernel(const OverlapArg
     }
     if (flags & 1) atomicOr(reinterpret_cast<unsigned*>(a.status), SPECOPD_FLAG_NONFINITE);
     if (flags & 2) atomicOr(reinterpret_cast<unsigned*>(a.status), SPECOPD_FLAG_TIMEOUT);
-    a.alpha[row] = x;
-    if (a.q_less) a.q_less[row] = y;
-    if (a.lse_draft) a.lse_draft[row] = lz2 * 0.6931471805599453f;
-    if (a.lse_teacher) a.lse_teacher[row] = lt2 * 0.6931471805599453f;
-    if (a.lz2) a.lz2[row] = lz2;
-    if (a.ql) a.ql[row] = y;
-
-    if (a.branch_cnt) {
-      // ---- E2E-TV epilogue: the last row of the branch to arrive finishes it
-      const int W = a.W;
-      const long long b = row / W;
-      __threadfence();
-      const unsigned old = atomicAdd(&a.branch_cnt[b], 1u);
-      if (old == (unsigned)(W - 1)) {
-        __threadfence();
-        const float* al_b = a.alpha + b * W;
-        double pre[SPECOPD_MAX_W + 1];
-        pre[0] = 1.0;
-        double share = 0.0;
-        for (int i = 1; i <= W; ++i) {
-          pre[i] = pre[i - 1] * (double)__ldcg(al_b + i - 1);
-          share += pre[i];
-        }
-        // S_i = 1 + alpha_{i+1} S_{i+1}, S_W = 1; g_i = -(1/count) pre_{i-1} S_i
-        double S = 1.0;
-        for (int i = W; i >= 1; --i) {
-          a.g[b * W + i - 1] = (float)(-a.inv_count * pre[i - 1] * S);
-          S = 1.0 + (double)__ldcg(al_b + i - 1) * S;
-        }
-        a.branch_sum[b] = share;
-        __threadfence();
-        const unsigned done = atomicAdd(&a.branch_cnt[a.num_branches], 1u);
-        if (done == (unsigned)(a.num_branches - 1)) {
-          __threadfence();
-          double total = 0.0;
-          for (long long k = 0; k < a.num_branches; ++k) total += __ldcg(a.branch_sum + k);
-          *a.loss = (float)(1.0 - total * a.inv_count);
-        }
-      }
-    }
+    row_epilogue(a, row, x, y, lz2, lt2);
   }
   // keep this CTA's shared memory alive until rank 0 has read it, and make
   // sure no bulk copy into it is still in flight (matters only after a timeout)
@@ -407,14 +364,16 @@ __global__ void __launch_bounds__(1024) e2e_loss_kernel(const float* __restrict_
   if (threadIdx.x == 0) *loss = (nb == 0) ? 0.f : (float)(1.0 - red[0] * inv_count);
 }
 
-int pick_cluster(long long V, size_t elem, int* seg_len, size_t* smem_bytes) {
+// Cluster size: the smallest C in {1,2,4,8,16} whose per-CTA share of the
+// row (draft + teacher) fits `target` bytes, so several CTAs fit on an SM.
+int pick_cluster(long long V, size_t elem, size_t extra, size_t target, int* seg_len, size_t* smem_bytes) {
   const int choices[5] = {1, 2, 4, 8, 16};
   for (int i = 0; i < 5; ++i) {
     const int C = choices[i];
     long long seg = (V + C - 1) / C;
     seg = (seg + 7) / 8 * 8;
-    const size_t bytes = 2 * (size_t)seg * elem + kMaxChunks * 8 + sizeof(StatSmem) + 128;
-    if ((bytes <= 100 * 1024 || C == 16) && seg <= (long long)kChunkElems * kMaxChunks) {
+    const size_t bytes = 2 * (size_t)seg * elem + kMaxChunks * 8 + extra + 128;
+    if ((bytes <= target || C == 16) && seg <= (long long)kChunkElems * kMaxChunks) {
       if (bytes > 227 * 1024) return 0;
       *seg_len = (int)seg;
       *smem_bytes = bytes;
@@ -424,16 +383,12 @@ int pick_cluster(long long V, size_t elem, int* seg_len, size_t* smem_bytes) {
   return 0;
 }
 
-template <typename T>
-cudaError_t launch_stats_t(const OverlapArgs& a, cudaStream_t stream) {
-  int seg_len = 0;
-  size_t smem = 0;
-  const int C = pick_cluster(a.V, sizeof(T), &seg_len, &smem);
-  if (C == 0) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(tv_stats_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+template <typename K>
+cudaError_t launch_cluster(K kernel, const OverlapArgs& a, int C, int seg_len, size_t smem, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if (C > 8) {
-    e = cudaFuncSetAttribute(tv_stats_kernel<T>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
   cudaLaunchConfig_t cfg = {};
@@ -448,9 +403,18 @@ cudaError_t launch_stats_t(const OverlapArgs& a, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, tv_stats_kernel<T>, a, C, seg_len);
+  e = cudaLaunchKernelEx(&cfg, kernel, a, C, seg_len);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_stats_t(const OverlapArgs& a, cudaStream_t stream) {
+  int seg_len = 0;
+  size_t smem = 0;
+  const int C = pick_cluster(a.V, sizeof(T), sizeof(StatSmem), 100 * 1024, &seg_len, &smem);
+  if (C == 0) return cudaErrorInvalidValue;
+  return launch_cluster(tv_stats_kernel<T>, a, C, seg_len, smem, stream);
 }
 
 template <typename T>
@@ -466,12 +430,12 @@ cudaError_t launch_grad_t(const OverlapArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_tv_stats(const OverlapArgs& a, specopd_dtype dtype, cudaStream_t stream) {
   if (a.rows == 0) return cudaSuccess;
-  return dtype == SPECOPD_BF16 ? launch_stats_t<__nv_bfloat16>(a, stream) : launch_stats_t<float>(a, stream);
+  return dtype == SPECOPD_BF16 ? launch_tv_stats_bf16(a, stream) : launch_stats_t<float>(a, stream);
 }
 
 cudaError_t launch_tv_grad(const OverlapArgs& a, specopd_dtype dtype, cudaStream_t stream) {
   if (a.rows == 0) return cudaSuccess;
-  return dtype == SPECOPD_BF16 ? launch_grad_t<__nv_bfloat16>(a, stream) : launch_grad_t<float>(a, stream);
+  return dtype == SPECOPD_BF16 ? launch_tv_grad_bf16(a, stream) : launch_grad_t<float>(a, stream);
 }
 
 cudaError_t launch_e2e_loss(const float* alpha, int64_t num_branches, int W, double inv_count, float* loss,
