@@ -241,6 +241,36 @@ int specopd_tv_overlap_e2e(const void* draft, const void* teacher, specopd_dtype
                            double count, float* alpha, float* loss, float* grad_draft, int64_t ld_grad,
                            void* workspace, size_t workspace_bytes, int32_t* status, specopd_stream_t stream);
 
+/*
+ * specopd_tv_overlap_e2e_static -- specopd_tv_overlap_e2e without a workspace.
+ *
+ * The paper has no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory for a workspace: programs whose device
+ * memory belongs to another allocator they must not bypass, and hot loops
+ * that must not call cudaMalloc/cudaFree because those calls can stall the
+ * whole device.  The scratch is a fixed array of SPECOPD_STATIC_SCRATCH_BYTES
+ * inside the library; every GPU that loads the library holds it until the
+ * process exits.  Arguments, outputs and results are those of
+ * specopd_tv_overlap_e2e minus the workspace; the call allocates nothing.
+ *
+ * Limits and caveats:
+ *   - a batch whose specopd_overlap_workspace_bytes(rows, V, num_branches)
+ *     exceeds SPECOPD_STATIC_SCRATCH_BYTES is rejected with
+ *     SPECOPD_ERR_WORKSPACE before anything is enqueued (32 MiB holds, e.g.,
+ *     1,600 rows of a 151,936-entry vocabulary);
+ *   - the first call on a device looks up the array's device address; make
+ *     that first call before starting any stream capture;
+ *   - all calls on a device share the one array and it keeps the previous
+ *     call's contents (the call clears what must start at zero itself), so
+ *     calls that may run at the same time on the GPU -- e.g. on two streams --
+ *     race and corrupt each other: order them on one stream.
+ */
+#define SPECOPD_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
+int specopd_tv_overlap_e2e_static(const void* draft, const void* teacher, specopd_dtype dtype, int64_t rows,
+                                  int64_t V, int64_t ld_draft, int64_t ld_teacher, int64_t num_branches, int W,
+                                  double count, float* alpha, float* loss, float* grad_draft, int64_t ld_grad,
+                                  int32_t* status, specopd_stream_t stream);
+
 /* Human-readable name of a specopd_status value. */
 const char* specopd_status_string(int status);
 

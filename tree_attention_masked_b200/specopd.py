@@ -69,8 +69,12 @@ _c = {
     "specopd_e2e_tv_loss": _sig("specopd_e2e_tv_loss", _int, _vp, _i64, _int, _f64, _vp, _vp, _vp),
     "specopd_tv_overlap_e2e": _sig("specopd_tv_overlap_e2e", _int, _vp, _vp, _int, _i64, _i64, _i64, _i64, _i64,
                                    _int, _f64, _vp, _vp, _vp, _i64, _vp, _sz, _vp, _vp),
+    "specopd_tv_overlap_e2e_static": _sig("specopd_tv_overlap_e2e_static", _int, _vp, _vp, _int, _i64, _i64,
+                                          _i64, _i64, _i64, _int, _f64, _vp, _vp, _vp, _i64, _vp, _vp),
     "specopd_status_string": _sig("specopd_status_string", ctypes.c_char_p, _int),
 }
+
+STATIC_SCRATCH_BYTES = 32 << 20
 
 EXPORTED = sorted(_c)
 
@@ -201,3 +205,13 @@ def specopd_tv_overlap_e2e(draft, teacher, V: int, num_branches: int, W: int, co
         _ptr(draft), _ptr(teacher), _dtype(draft), draft.shape[0], V, draft.stride(0), teacher.stride(0),
         num_branches, W, count, _ptr(alpha), _ptr(loss), _ptr(grad), grad.stride(0) if grad is not None else 0,
         _ptr(workspace), wb, _ptr(status), _stream(stream)))
+
+
+def specopd_tv_overlap_e2e_static(draft, teacher, V: int, num_branches: int, W: int, count: float, alpha, loss,
+                                  grad, status, stream=None) -> None:
+    """specopd_tv_overlap_e2e with the library's own fixed scratch instead of a
+    caller workspace, for callers that cannot allocate device memory."""
+    _check("specopd_tv_overlap_e2e_static", _c["specopd_tv_overlap_e2e_static"](
+        _ptr(draft), _ptr(teacher), _dtype(draft), draft.shape[0], V, draft.stride(0), teacher.stride(0),
+        num_branches, W, count, _ptr(alpha), _ptr(loss), _ptr(grad), grad.stride(0) if grad is not None else 0,
+        _ptr(status), _stream(stream)))
