@@ -1,5 +1,5 @@
-// K4/K5 for bf16 logits: per-row overlap statistics (cluster kernel) and the
-// streaming gradient.
+// K4/K5 for bf16 logits: per-row overlap statistics (persistent ring kernel)
+// and the streaming gradient.
 //
 // daiwk.github.io write-up of SpecOPD, section "Equations": alpha = sum_v
 // min(q(v), p(v)); L = 1 - (1/(B W)) sum_b sum_j prod_{i<=j} alpha_{b,i};
@@ -7,22 +7,14 @@
 // draft support kept.  Section "Inputs and code mapping": NaN padding marks
 // inactive draft entries, the teacher must be finite, bf16 work promotes to fp32.
 //
-// Statistics: one thread-block cluster of C CTAs per prediction row, the row's
-// draft and teacher logits split over the CTAs and bulk-copied (no multicast)
-// into shared memory, where they stay for both passes.  The per-row latency
-// (load -> pass 1 -> exchange -> pass 2 -> exchange) bounds the bandwidth
-// (bytes in flight / latency), so the chain is kept short:
-//   * copies are issued before the cluster start barrier, whose wait is
-//     deferred until after pass 1;
-//   * pass 1 is a single online base-2 (max, sum) pass over packed bf16x2
-//     data as the copy chunks land;
-//   * every CTA pushes its partials into the shared memory of the CTAs that
-//     need them before a cluster barrier, so all reads after it are local and
-//     CTAs other than rank 0 exit right after the second barrier;
-//   * reductions use fixed shuffle trees, so every CTA derives bitwise
-//     identical normalisers and the results are reproducible run to run.
-// Gradient: dL/dz = g q ([q < p] - q_less) from the draft logits and the bits
-// written by pass 2; every warp access is contiguous.
+// Statistics need two passes over a row (the normalisers before alpha).  A
+// row's logits are read from HBM once: the second pass re-reads them while
+// they are still in the L2 (one row in flight per SM is a small part of it),
+// and every copy goes through a ring of shared-memory slots fed by one
+// producer thread, so HBM reads run ahead of the arithmetic and through the
+// reductions between the passes.  Gradient: dL/dz = g q ([q < p] - q_less)
+// from the draft logits and the bits written by pass 2; every warp access is
+// contiguous.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -32,11 +24,6 @@
 namespace specopd {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
-constexpr int kChunkElems = 4096;
-constexpr int kMaxChunks = 32;
-constexpr int kMaxCluster = 16;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kNegInf2 = 0xFF80FF80u;  // two bf16 -inf
 
@@ -54,281 +41,328 @@ __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w <<
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 __device__ __forceinline__ bool nonfinite(float x) { return !(fabsf(x) < INFINITY); }
 
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
 }
-__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
-__device__ __forceinline__ void st_cluster_v4(uint32_t caddr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(caddr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
-// try_wait that lets the hardware suspend the thread for up to `ns`
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  const long long t0 = clock64();
-  while (!mbar_try_wait_sleep(bar, parity, 20000u)) {
-    if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
-      *abort_flag = 1;
-      return false;
-    }
-  }
-  return true;
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
 }
 
-struct Smem {
-  float lse_in[kMaxCluster][4];  // (mz, sz, mt, st) pushed by each CTA of the cluster, by rank
-  float al_in[kMaxCluster][4];   // (alpha, q_less, flags) pushed to rank 0, by rank
-  float red[kWarps][4];
+// pass-1 update for 8 draft and 8 teacher logits
+__device__ __forceinline__ void p1_group(const uint4& zw, const uint4& tw, float& mz, float& sz, float& mt, float& st,
+                                         uint32_t& tmn) {
+  const uint32_t zm = bmax2(bmax2(zw.x, zw.y), bmax2(zw.z, zw.w));
+  const uint32_t tm = bmax2(bmax2(tw.x, tw.y), bmax2(tw.z, tw.w));
+  tmn = bmin2_nan(tmn, bmin2_nan(bmin2_nan(tw.x, tw.y), bmin2_nan(tw.z, tw.w)));
+  const float gz = fmaxf(bf_lo(zm), bf_hi(zm)) * kLog2e;
+  const float gt = fmaxf(bf_lo(tm), bf_hi(tm)) * kLog2e;
+  if (gz > mz) {
+    sz *= ex2(mz - gz);
+    mz = gz;
+  }
+  if (gt > mt) {
+    st *= ex2(mt - gt);
+    mt = gt;
+  }
+  const float mze = (mz == -INFINITY) ? 0.f : mz;
+  const float2 l2e = make_float2(kLog2e, kLog2e);
+  const float2 nmz = make_float2(-mze, -mze), nmt = make_float2(-mt, -mt);
+  const uint32_t zs[4] = {zw.x, zw.y, zw.z, zw.w};
+  const uint32_t ts[4] = {tw.x, tw.y, tw.z, tw.w};
+  float2 az = make_float2(0.f, 0.f), at = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t zc = bmax2(zs[k], kNegInf2);  // NaN (inactive) -> -inf -> adds 0
+    const float2 ea = __ffma2_rn(make_float2(bf_lo(zc), bf_hi(zc)), l2e, nmz);
+    const float2 eb = __ffma2_rn(make_float2(bf_lo(ts[k]), bf_hi(ts[k])), l2e, nmt);
+    az = __fadd2_rn(az, make_float2(ex2(ea.x), ex2(ea.y)));
+    at = __fadd2_rn(at, make_float2(ex2(eb.x), ex2(eb.y)));
+  }
+  sz += az.x + az.y;
+  st += at.x + at.y;
+}
+
+// pass-2 update for 8 logit pairs: alpha and q_less shares, one byte of bits
+__device__ __forceinline__ uint32_t p2_group(const uint4& zw, const uint4& tw, float2 nlz, float2 nlt, float2& acc_a,
+                                             float2& acc_q) {
+  const float2 l2e = make_float2(kLog2e, kLog2e);
+  const uint32_t zs[4] = {zw.x, zw.y, zw.z, zw.w};
+  const uint32_t ts[4] = {tw.x, tw.y, tw.z, tw.w};
+  uint32_t byte = 0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t zc = bmax2(zs[k], kNegInf2);
+    const float2 da = __ffma2_rn(make_float2(bf_lo(zc), bf_hi(zc)), l2e, nlz);
+    const float2 db = __ffma2_rn(make_float2(bf_lo(ts[k]), bf_hi(ts[k])), l2e, nlt);
+    const float e0 = ex2(fminf(da.x, db.x)), e1 = ex2(fminf(da.y, db.y));
+    const bool c0 = da.x < db.x, c1 = da.y < db.y;
+    acc_a = __fadd2_rn(acc_a, make_float2(e0, e1));
+    acc_q = __fadd2_rn(acc_q, make_float2(c0 ? e0 : 0.f, c1 ? e1 : 0.f));
+    byte |= (c0 ? 1u : 0u) << (2 * k) | (c1 ? 1u : 0u) << (2 * k + 1);
+  }
+  return byte;
+}
+
+// ---------------- statistics: persistent ring kernel
+// One CTA owns one prediction row at a time (rows blockIdx.x, + gridDim.x,
+// ...) and reads it twice through a ring of shared-memory slots:
+//   pass 1 -- the row's draft and teacher logits from HBM (L2 policy
+//             evict_last) into the online base-2 (max, sum) of both softmaxes;
+//   pass 2 -- the same bytes again, an L2 hit (one row per SM is a small part
+//             of the L2), for alpha, q_less and the [q < p] bits.
+// Warp 0 is the producer: one thread walks the chunk sequence
+// P1(row), P2(row), P1(next row), ... and bulk-copies each chunk of draft and
+// teacher logits into the next free slot (no multicast).  The other warps
+// consume the slots in the same order, so the copies run ahead through the
+// reductions between the passes.  Per-row reductions use fixed shuffle trees
+// (reproducible results).  All waits are bounded; the consumer warps always
+// pass the same named barriers, whatever happened, so none can be left behind.
+constexpr int kRProd = 32;                       // producer warp
+constexpr int kRCons = 512;                      // consumer threads (16 warps)
+constexpr int kRThreads = kRProd + kRCons;
+constexpr int kRWarps = kRCons / 32;
+constexpr int kRChunk = 8192;                    // logits per chunk and array
+constexpr int kRSlots = 6;
+constexpr int kRGroups = kRChunk / 8;            // 16-byte groups per chunk and array
+constexpr uint32_t kRSlotBytes = 2u * kRChunk * 2u;
+
+struct RingCtl {
+  uint64_t full[kRSlots];
+  uint64_t empty[kRSlots];
+  float red[kRWarps][4];
   float bcast[2];
-  int bad;
   int abort_flag;
 };
 
-__global__ void __launch_bounds__(kThreads) tv_stats_bf16_kernel(const OverlapArgs a, int C, int seg_len) {
+__device__ __forceinline__ void bulk_g2s_policy(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                                uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void cons_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kRCons) : "memory"); }
+
+struct RingRed {
+  float r1[kRWarps][4];  // pass-1 partials (mz, sz, mt, st) by consumer warp
+  float r2[kRWarps][2];  // pass-2 partials (alpha, q_less)
+  int bad[kRWarps];
+};
+
+__device__ __forceinline__ void ring_drain_wait(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitLimitCycles) return;
+  }
+}
+
+__global__ void __launch_bounds__(kRThreads, 1) tv_stats_bf16_ring_kernel(const OverlapArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
-  uint32_t* zb = reinterpret_cast<uint32_t*>(smem);  // bf16 pairs
-  uint32_t* tb = zb + seg_len / 2;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(tb + seg_len / 2);
-  Smem* ss = reinterpret_cast<Smem*>(bars + kMaxChunks);
-
+  uint8_t* ring = smem;
+  RingCtl* ctl = reinterpret_cast<RingCtl*>(ring + kRSlots * kRSlotBytes);
+  RingRed* rr = reinterpret_cast<RingRed*>(ctl + 1);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int rank = (int)cluster_ctarank();
-  const long long row = blockIdx.x / C;
-  const long long s0 = (long long)rank * seg_len;
-  const int len = (int)max(0LL, min((long long)a.V, s0 + seg_len) - s0);
-  const int len8 = len & ~7;
-  const int tail = len - len8;
-  const int nch = (len8 + kChunkElems - 1) / kChunkElems;
-  const __nv_bfloat16* zrow = static_cast<const __nv_bfloat16*>(a.draft) + row * a.ld_draft + s0;
-  const __nv_bfloat16* trow = static_cast<const __nv_bfloat16*>(a.teacher) + row * a.ld_teacher + s0;
-
+  const int len8 = (int)(a.V & ~7LL);
+  const int tail = (int)(a.V - len8);
+  const int nch = (len8 + kRChunk - 1) / kRChunk;
   if (tid == 0) {
-    for (int c = 0; c < nch; ++c) mbar_init(&bars[c], 1);
-    ss->bad = 0;
-    ss->abort_flag = 0;
+    for (int s = 0; s < kRSlots; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], kRWarps);
+    }
+    ctl->abort_flag = 0;
     fence_barrier_init();
   }
   __syncthreads();
-  if (tid == 0) {
-    for (int c = 0; c < nch; ++c) {
-      const int e0 = c * kChunkElems, e1 = min(len8, e0 + kChunkElems);
-      const uint32_t bytes = (uint32_t)(e1 - e0) * 2u;
-      mbar_arrive_expect_tx(&bars[c], 2 * bytes);
-      bulk_g2s(zb + e0 / 2, zrow + e0, bytes, &bars[c]);
-      bulk_g2s(tb + e0 / 2, trow + e0, bytes, &bars[c]);
-    }
-  }
-  cluster_arrive_relaxed();  // every CTA of the cluster has started (waited below)
-  volatile int* abort_flag = &ss->abort_flag;
+  volatile int* abort_flag = &ctl->abort_flag;
 
-  // ---- pass 1: online base-2 log-sum-exp of draft (active) and teacher
-  float mz = -INFINITY, sz = 0.f, mt = -INFINITY, st = 0.f;
-  uint32_t tmn = 0u;  // NaN-aware running min of the teacher: NaN or -inf wins
-  const float2 l2e = make_float2(kLog2e, kLog2e);
-  for (int c = 0; c < nch; ++c) {
-    if (!mbar_wait_sleep(&bars[c], 0, abort_flag)) break;
-    const int g1 = min(len8, (c + 1) * kChunkElems) / 8;
-    for (int g = c * (kChunkElems / 8) + tid; g < g1; g += kThreads) {
-      const uint4 zw = reinterpret_cast<const uint4*>(zb)[g];
-      const uint4 tw = reinterpret_cast<const uint4*>(tb)[g];
-      const uint32_t zm = bmax2(bmax2(zw.x, zw.y), bmax2(zw.z, zw.w));
-      const uint32_t tm = bmax2(bmax2(tw.x, tw.y), bmax2(tw.z, tw.w));
-      tmn = bmin2_nan(tmn, bmin2_nan(bmin2_nan(tw.x, tw.y), bmin2_nan(tw.z, tw.w)));
-      const float gz = fmaxf(bf_lo(zm), bf_hi(zm)) * kLog2e;
-      const float gt = fmaxf(bf_lo(tm), bf_hi(tm)) * kLog2e;
-      if (gz > mz) {
-        sz *= ex2(mz - gz);
-        mz = gz;
-      }
-      if (gt > mt) {
-        st *= ex2(mt - gt);
-        mt = gt;
-      }
-      const float mze = (mz == -INFINITY) ? 0.f : mz;
-      const float2 nmz = make_float2(-mze, -mze), nmt = make_float2(-mt, -mt);
-      const uint32_t zs[4] = {zw.x, zw.y, zw.z, zw.w};
-      const uint32_t ts[4] = {tw.x, tw.y, tw.z, tw.w};
-      float2 az = make_float2(0.f, 0.f), at = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t zc = bmax2(zs[k], kNegInf2);  // NaN (inactive) -> -inf -> adds 0
-        const float2 ea = __ffma2_rn(make_float2(bf_lo(zc), bf_hi(zc)), l2e, nmz);
-        const float2 eb = __ffma2_rn(make_float2(bf_lo(ts[k]), bf_hi(ts[k])), l2e, nmt);
-        az = __fadd2_rn(az, make_float2(ex2(ea.x), ex2(ea.y)));
-        at = __fadd2_rn(at, make_float2(ex2(eb.x), ex2(eb.y)));
-      }
-      sz += az.x + az.y;
-      st += at.x + at.y;
-    }
-  }
-  bool bad = nonfinite(bf_lo(tmn)) || nonfinite(bf_hi(tmn)) || mz == INFINITY || mt == INFINITY;
-  float ztail = -INFINITY, ttail = 0.f;
-  if (tid < tail) {  // fewer than 8 logits at the very end of the row
-    ztail = __bfloat162float(zrow[len8 + tid]);
-    ttail = __bfloat162float(trow[len8 + tid]);
-    bad |= nonfinite(ttail) || ztail == INFINITY;
-    if (ztail == ztail && ztail != -INFINITY) lse_merge(mz, sz, ztail * kLog2e, 1.f);
-    lse_merge(mt, st, ttail * kLog2e, 1.f);
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const float om1 = __shfl_xor_sync(0xffffffffu, mz, off), os1 = __shfl_xor_sync(0xffffffffu, sz, off);
-    const float om2 = __shfl_xor_sync(0xffffffffu, mt, off), os2 = __shfl_xor_sync(0xffffffffu, st, off);
-    lse_merge(mz, sz, om1, os1);
-    lse_merge(mt, st, om2, os2);
-  }
-  if (__any_sync(0xffffffffu, bad) && lane == 0) ss->bad = 1;
-  if (lane == 0) {
-    ss->red[warp][0] = mz;
-    ss->red[warp][1] = sz;
-    ss->red[warp][2] = mt;
-    ss->red[warp][3] = st;
-  }
-  __syncthreads();
-  cluster_wait();  // all CTAs have started: remote shared memory may be written
   if (warp == 0) {
-    float m1 = -INFINITY, s1 = 0.f, m2 = -INFINITY, s2 = 0.f;
-    if (lane < kWarps) {
-      m1 = ss->red[lane][0];
-      s1 = ss->red[lane][1];
-      m2 = ss->red[lane][2];
-      s2 = ss->red[lane][3];
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float o1 = __shfl_xor_sync(0xffffffffu, m1, off), p1 = __shfl_xor_sync(0xffffffffu, s1, off);
-      const float o2 = __shfl_xor_sync(0xffffffffu, m2, off), p2 = __shfl_xor_sync(0xffffffffu, s2, off);
-      lse_merge(m1, s1, o1, p1);
-      lse_merge(m2, s2, o2, p2);
-    }
-    // lane q pushes this CTA's partial into CTA q's slot for this rank
-    if (lane < C) st_cluster_v4(map_cluster(smem_u32(&ss->lse_in[rank][0]), lane), m1, s1, m2, s2);
-  }
-  cluster_sync();
-  if (warp == 0) {
-    float m1 = -INFINITY, s1 = 0.f, m2 = -INFINITY, s2 = 0.f;
-    if (lane < C) {
-      m1 = ss->lse_in[lane][0];
-      s1 = ss->lse_in[lane][1];
-      m2 = ss->lse_in[lane][2];
-      s2 = ss->lse_in[lane][3];
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float o1 = __shfl_xor_sync(0xffffffffu, m1, off), p1 = __shfl_xor_sync(0xffffffffu, s1, off);
-      const float o2 = __shfl_xor_sync(0xffffffffu, m2, off), p2 = __shfl_xor_sync(0xffffffffu, s2, off);
-      lse_merge(m1, s1, o1, p1);
-      lse_merge(m2, s2, o2, p2);
-    }
+    // ================= producer: chunk sequence P1(row), P2(row), P1(next row), ...
     if (lane == 0) {
-      ss->bcast[0] = (s1 > 0.f) ? m1 + log2f(s1) : -INFINITY;
-      ss->bcast[1] = m2 + log2f(s2);
+      const uint64_t pol_keep = l2_policy_evict_last();
+      const uint64_t pol_drop = l2_policy_evict_first();
+      long long n = 0;  // chunks issued
+      bool ok = true;
+      for (long long row = blockIdx.x; ok && row < a.rows; row += gridDim.x) {
+        const __nv_bfloat16* zrow = static_cast<const __nv_bfloat16*>(a.draft) + row * a.ld_draft;
+        const __nv_bfloat16* trow = static_cast<const __nv_bfloat16*>(a.teacher) + row * a.ld_teacher;
+        for (int pass = 0; ok && pass < 2; ++pass) {
+          for (int c = 0; c < nch; ++c, ++n) {
+            const int slot = (int)(n % kRSlots);
+            if (n >= kRSlots && !mbar_wait(&ctl->empty[slot], (uint32_t)((n / kRSlots) - 1) & 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            const int e0 = c * kRChunk;
+            const uint32_t bytes = (uint32_t)(min(len8, e0 + kRChunk) - e0) * 2u;
+            uint8_t* dz = ring + slot * kRSlotBytes;
+            mbar_arrive_expect_tx(&ctl->full[slot], 2u * bytes);
+            bulk_g2s_policy(dz, zrow + e0, bytes, &ctl->full[slot], pass ? pol_drop : pol_keep);
+            bulk_g2s_policy(dz + kRChunk * 2, trow + e0, bytes, &ctl->full[slot], pass ? pol_drop : pol_keep);
+          }
+        }
+      }
+      // every issued copy must land before the CTA may exit
+      for (long long k = (n > kRSlots ? n - kRSlots : 0); k < n; ++k)
+        ring_drain_wait(&ctl->full[k % kRSlots], (uint32_t)(k / kRSlots) & 1u);
+      if (ctl->abort_flag) atomicOr(reinterpret_cast<unsigned*>(a.status), SPECOPD_FLAG_TIMEOUT);
     }
+    return;
   }
-  __syncthreads();
-  const float lz2 = ss->bcast[0];
-  const float lt2 = ss->bcast[1];
 
-  // ---- pass 2: alpha, q_less and the strict-less bits
-  float2 acc_a = make_float2(0.f, 0.f), acc_q = make_float2(0.f, 0.f);
-  uint8_t* mrow = a.mbits ? a.mbits + row * a.mbits_ld + s0 / 8 : nullptr;
-  if (lz2 != -INFINITY) {
-    const float2 nlz = make_float2(-lz2, -lz2), nlt = make_float2(-lt2, -lt2);
-    for (int g = tid; g < len8 / 8; g += kThreads) {
-      const uint4 zw = reinterpret_cast<const uint4*>(zb)[g];
-      const uint4 tw = reinterpret_cast<const uint4*>(tb)[g];
-      const uint32_t zs[4] = {zw.x, zw.y, zw.z, zw.w};
-      const uint32_t ts[4] = {tw.x, tw.y, tw.z, tw.w};
-      uint32_t byte = 0;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t zc = bmax2(zs[k], kNegInf2);
-        const float2 da = __ffma2_rn(make_float2(bf_lo(zc), bf_hi(zc)), l2e, nlz);
-        const float2 db = __ffma2_rn(make_float2(bf_lo(ts[k]), bf_hi(ts[k])), l2e, nlt);
-        const float e0 = ex2(fminf(da.x, db.x)), e1 = ex2(fminf(da.y, db.y));
-        const bool c0 = da.x < db.x, c1 = da.y < db.y;
-        acc_a = __fadd2_rn(acc_a, make_float2(e0, e1));
-        acc_q = __fadd2_rn(acc_q, make_float2(c0 ? e0 : 0.f, c1 ? e1 : 0.f));
-        byte |= (c0 ? 1u : 0u) << (2 * k) | (c1 ? 1u : 0u) << (2 * k + 1);
-      }
-      if (mrow) mrow[g] = (uint8_t)byte;
-    }
-  }
-  float al = acc_a.x + acc_a.y, ql = acc_q.x + acc_q.y;
-  if (tail > 0 && warp == 0) {
-    bool lt = false;
-    if (tid < tail && lz2 != -INFINITY && ztail == ztail && ztail != -INFINITY) {
-      const float da = fmaf(ztail, kLog2e, -lz2), db = fmaf(ttail, kLog2e, -lt2);
-      const float e = ex2(fminf(da, db));
-      lt = da < db;
-      al += e;
-      if (lt) ql += e;
-    }
-    const unsigned bits = __ballot_sync(0xffffffffu, lt) & ((1u << tail) - 1u);
-    if (mrow && tid == 0) mrow[len8 / 8] = (uint8_t)bits;
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    al += __shfl_xor_sync(0xffffffffu, al, off);
-    ql += __shfl_xor_sync(0xffffffffu, ql, off);
-  }
-  if (lane == 0) {
-    ss->red[warp][0] = al;
-    ss->red[warp][1] = ql;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    float x = (lane < kWarps) ? ss->red[lane][0] : 0.f;
-    float y = (lane < kWarps) ? ss->red[lane][1] : 0.f;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      x += __shfl_xor_sync(0xffffffffu, x, off);
-      y += __shfl_xor_sync(0xffffffffu, y, off);
-    }
-    if (lane == 0) {
-      const float flags = (float)((ss->bad ? 1 : 0) | (ss->abort_flag ? 2 : 0));
-      st_cluster_v4(map_cluster(smem_u32(&ss->al_in[rank][0]), 0), x, y, flags, 0.f);
-    }
-  }
-  // drain before this CTA may exit (copies only remain in flight after a timeout)
-  if (tid == 0 && ss->abort_flag) {
-    for (int c = 0; c < nch; ++c) {
-      const long long t0 = clock64();
-      while (!mbar_try_wait(&bars[c], 0) && clock64() - t0 < kWaitLimitCycles) {
+  // ================= consumers (16 warps, one or two 16-byte groups per chunk each)
+  const int ct = tid - kRProd;
+  const int cw = ct >> 5;
+  long long n = 0;  // chunks consumed
+  bool ok = true;   // uniform per warp; a failed wait only skips work, never a barrier
+  for (long long row = blockIdx.x; row < a.rows; row += gridDim.x) {
+    const __nv_bfloat16* zrow = static_cast<const __nv_bfloat16*>(a.draft) + row * a.ld_draft;
+    const __nv_bfloat16* trow = static_cast<const __nv_bfloat16*>(a.teacher) + row * a.ld_teacher;
+
+    // ---- pass 1
+    float mz = -INFINITY, sz = 0.f, mt = -INFINITY, st = 0.f;
+    uint32_t tmn = 0u;  // NaN-aware running min of the teacher: NaN or -inf wins
+    for (int c = 0; c < nch; ++c, ++n) {
+      const int slot = (int)(n % kRSlots);
+      if (ok) ok = mbar_wait_warp(&ctl->full[slot], (uint32_t)(n / kRSlots) & 1u, abort_flag);
+      if (ok) {
+        const int ngc = (min(len8, (c + 1) * kRChunk) - c * kRChunk) / 8;
+        const uint4* zs = reinterpret_cast<const uint4*>(ring + slot * kRSlotBytes);
+        const uint4* ts = zs + kRGroups;
+        if (ct + kRCons < ngc) {
+          const uint4 z0 = zs[ct], t0 = ts[ct], z1 = zs[ct + kRCons], t1 = ts[ct + kRCons];
+          p1_group(z0, t0, mz, sz, mt, st, tmn);
+          p1_group(z1, t1, mz, sz, mt, st, tmn);
+        } else if (ct < ngc) {
+          p1_group(zs[ct], ts[ct], mz, sz, mt, st, tmn);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->empty[slot]);
       }
     }
-  }
-  cluster_sync();
-  if (rank == 0 && warp == 0) {
-    float x = 0.f, y = 0.f;
-    int f = 0;
-    if (lane < C) {
-      x = ss->al_in[lane][0];
-      y = ss->al_in[lane][1];
-      f = (int)ss->al_in[lane][2];
+    bool bad = nonfinite(bf_lo(tmn)) || nonfinite(bf_hi(tmn)) || mz == INFINITY || mt == INFINITY;
+    float ztail = -INFINITY, ttail = 0.f;
+    if (ct < tail) {  // fewer than 8 logits at the very end of the row
+      ztail = __bfloat162float(zrow[len8 + ct]);
+      ttail = __bfloat162float(trow[len8 + ct]);
+      bad |= nonfinite(ttail) || ztail == INFINITY;
+      if (ztail == ztail && ztail != -INFINITY) lse_merge(mz, sz, ztail * kLog2e, 1.f);
+      lse_merge(mt, st, ttail * kLog2e, 1.f);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
-      x += __shfl_xor_sync(0xffffffffu, x, off);
-      y += __shfl_xor_sync(0xffffffffu, y, off);
-      f |= __shfl_xor_sync(0xffffffffu, f, off);
+      const float om1 = __shfl_xor_sync(0xffffffffu, mz, off), os1 = __shfl_xor_sync(0xffffffffu, sz, off);
+      const float om2 = __shfl_xor_sync(0xffffffffu, mt, off), os2 = __shfl_xor_sync(0xffffffffu, st, off);
+      lse_merge(mz, sz, om1, os1);
+      lse_merge(mt, st, om2, os2);
+    }
+    const bool wbad = __any_sync(0xffffffffu, bad);
+    if (lane == 0) {
+      rr->r1[cw][0] = mz;
+      rr->r1[cw][1] = sz;
+      rr->r1[cw][2] = mt;
+      rr->r1[cw][3] = st;
+      rr->bad[cw] = wbad ? 1 : 0;
+    }
+    cons_bar();
+    // every warp merges the 16 partials with the same shuffle tree: identical bits
+    float lz2, lt2;
+    bool row_bad = false;
+    {
+      float m1 = -INFINITY, s1 = 0.f, m2 = -INFINITY, s2 = 0.f;
+      if (lane < kRWarps) {
+        m1 = rr->r1[lane][0];
+        s1 = rr->r1[lane][1];
+        m2 = rr->r1[lane][2];
+        s2 = rr->r1[lane][3];
+        row_bad = rr->bad[lane] != 0;
+      }
+      row_bad = __any_sync(0xffffffffu, row_bad);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float o1 = __shfl_xor_sync(0xffffffffu, m1, off), p1 = __shfl_xor_sync(0xffffffffu, s1, off);
+        const float o2 = __shfl_xor_sync(0xffffffffu, m2, off), p2 = __shfl_xor_sync(0xffffffffu, s2, off);
+        lse_merge(m1, s1, o1, p1);
+        lse_merge(m2, s2, o2, p2);
+      }
+      lz2 = (s1 > 0.f) ? m1 + log2f(s1) : -INFINITY;
+      lt2 = m2 + log2f(s2);
+    }
+
+    // ---- pass 2: alpha, q_less and the strict-less bits (L2 re-read)
+    const bool live = lz2 != -INFINITY;
+    const float2 nlz = make_float2(live ? -lz2 : 0.f, live ? -lz2 : 0.f), nlt = make_float2(-lt2, -lt2);
+    float2 acc_a = make_float2(0.f, 0.f), acc_q = make_float2(0.f, 0.f);
+    uint8_t* mrow = a.mbits ? a.mbits + row * a.mbits_ld : nullptr;
+    for (int c = 0; c < nch; ++c, ++n) {
+      const int slot = (int)(n % kRSlots);
+      if (ok) ok = mbar_wait_warp(&ctl->full[slot], (uint32_t)(n / kRSlots) & 1u, abort_flag);
+      if (ok) {
+        const int ngc = (min(len8, (c + 1) * kRChunk) - c * kRChunk) / 8;
+        const uint4* zs = reinterpret_cast<const uint4*>(ring + slot * kRSlotBytes);
+        const uint4* ts = zs + kRGroups;
+        uint8_t* mc = mrow ? mrow + (long long)c * kRGroups : nullptr;
+        if (live) {
+          if (ct + kRCons < ngc) {
+            const uint4 z0 = zs[ct], t0 = ts[ct], z1 = zs[ct + kRCons], t1 = ts[ct + kRCons];
+            const uint32_t b0 = p2_group(z0, t0, nlz, nlt, acc_a, acc_q);
+            const uint32_t b1 = p2_group(z1, t1, nlz, nlt, acc_a, acc_q);
+            if (mc) {
+              mc[ct] = (uint8_t)b0;
+              mc[ct + kRCons] = (uint8_t)b1;
+            }
+          } else if (ct < ngc) {
+            const uint32_t b0 = p2_group(zs[ct], ts[ct], nlz, nlt, acc_a, acc_q);
+            if (mc) mc[ct] = (uint8_t)b0;
+          }
+        } else if (mc) {  // no active draft logit: q = 0 everywhere
+          for (int g = ct; g < ngc; g += kRCons) mc[g] = 0;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->empty[slot]);
+      }
+    }
+    float al = acc_a.x + acc_a.y, ql = acc_q.x + acc_q.y;
+    if (tail > 0 && cw == 0) {
+      bool lt = false;
+      if (ct < tail && live && ztail == ztail && ztail != -INFINITY) {
+        const float da = fmaf(ztail, kLog2e, -lz2), db = fmaf(ttail, kLog2e, -lt2);
+        const float e = ex2(fminf(da, db));
+        lt = da < db;
+        al += e;
+        if (lt) ql += e;
+      }
+      const unsigned bits = __ballot_sync(0xffffffffu, lt) & ((1u << tail) - 1u);
+      if (mrow && ct == 0) mrow[len8 / 8] = (uint8_t)bits;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      al += __shfl_xor_sync(0xffffffffu, al, off);
+      ql += __shfl_xor_sync(0xffffffffu, ql, off);
     }
     if (lane == 0) {
-      if (f & 1) atomicOr(reinterpret_cast<unsigned*>(a.status), SPECOPD_FLAG_NONFINITE);
-      if (f & 2) atomicOr(reinterpret_cast<unsigned*>(a.status), SPECOPD_FLAG_TIMEOUT);
-      if (lz2 == -INFINITY) x = y = 0.f;
-      row_epilogue(a, row, x, y, lz2, lt2);
+      rr->r2[cw][0] = al;
+      rr->r2[cw][1] = ql;
+    }
+    cons_bar();
+    if (cw == 0) {
+      float x = (lane < kRWarps) ? rr->r2[lane][0] : 0.f;
+      float y = (lane < kRWarps) ? rr->r2[lane][1] : 0.f;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        x += __shfl_xor_sync(0xffffffffu, x, off);
+        y += __shfl_xor_sync(0xffffffffu, y, off);
+      }
+      if (lane == 0) {
+        if (row_bad) atomicOr(reinterpret_cast<unsigned*>(a.status), SPECOPD_FLAG_NONFINITE);
+        if (!live) x = y = 0.f;
+        row_epilogue(a, row, x, y, lz2, lt2);
+      }
     }
   }
 }
@@ -393,41 +427,21 @@ __global__ void __launch_bounds__(kGradThreads) tv_grad_bf16_kernel(const Overla
 
 }  // namespace
 
-// Cluster size: the smallest C in {1,2,4,8,16} whose per-CTA share of the
-// row (draft + teacher) fits about 48 KB, so four or five CTAs share an SM.
+// Persistent ring statistics kernel: one CTA per SM (about 194 KB of ring),
+// at most one CTA per row.
 cudaError_t launch_tv_stats_bf16(const OverlapArgs& a, cudaStream_t stream) {
   if (a.rows == 0) return cudaSuccess;
-  int C = 0;
-  long long seg = 0;
-  const int choices[5] = {1, 2, 4, 8, 16};
-  for (int i = 0; i < 5 && !C; ++i) {
-    seg = (a.V + choices[i] - 1) / choices[i];
-    seg = (seg + 7) / 8 * 8;
-    if (4 * seg <= 48 * 1024 || choices[i] == kMaxCluster) C = choices[i];
-  }
-  if (seg > (long long)kChunkElems * kMaxChunks) return cudaErrorInvalidValue;
-  const size_t smem = (size_t)4 * seg + kMaxChunks * 8 + sizeof(Smem) + 128;
-  if (smem > 227 * 1024) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(tv_stats_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (a.V > 0x7fffffffLL - kRChunk) return cudaErrorInvalidValue;
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (C > 8) {
-    e = cudaFuncSetAttribute(tv_stats_bf16_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(a.rows * C), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, tv_stats_bf16_kernel, a, C, (int)seg);
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
+  const size_t smem = (size_t)kRSlots * kRSlotBytes + sizeof(RingCtl) + sizeof(RingRed);
+  e = cudaFuncSetAttribute(tv_stats_bf16_ring_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const long long grid = a.rows < sms ? a.rows : sms;
+  tv_stats_bf16_ring_kernel<<<(unsigned)grid, kRThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
