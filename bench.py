@@ -196,6 +196,7 @@ def run_gpu(args):
     build()
     from tree_attention_masked_b200 import specopd as S
     from tree_attention_masked_b200.scoring import ScoringStep
+    from tree_attention_masked_b200 import parallel as PAR
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -256,10 +257,7 @@ def run_gpu(args):
     t_mask = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
     t_attn = statistics.mean(m[1].elapsed_time(m[2]) for m in marks)
     t_ov = statistics.mean(m[2].elapsed_time(m[3]) for m in marks)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = PAR.max_time_ms(elapsed_ms, device=dev)  # slowest rank (identity at N = 1)
 
     # ---- end to end through the public API with host buffers
     pin = lambda x, dt: (torch.from_numpy(x).view(torch.bfloat16) if dt == "bf16" else torch.from_numpy(x)).pin_memory()
@@ -291,10 +289,7 @@ def run_gpu(args):
     e_end.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e_start.elapsed_time(e_end)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = PAR.max_time_ms(e2e_ms, device=dev)
     status = st.check_status()
 
     peaks = load_peaks()
