@@ -52,12 +52,20 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   return p;
 }
 
-// pass-1 update for 8 draft and 8 teacher logits
-__device__ __forceinline__ void p1_group(const uint4& zw, const uint4& tw, float& mz, float& sz, float& mt, float& st,
-                                         uint32_t& tmn) {
-  const uint32_t zm = bmax2(bmax2(zw.x, zw.y), bmax2(zw.z, zw.w));
-  const uint32_t tm = bmax2(bmax2(tw.x, tw.y), bmax2(tw.z, tw.w));
-  tmn = bmin2_nan(tmn, bmin2_nan(bmin2_nan(tw.x, tw.y), bmin2_nan(tw.z, tw.w)));
+// pass-1 update for the G 16-byte groups a thread owns in one chunk: one
+// maximum over all of them, then the exponentials of every group against that
+// single reference (independent, so they overlap).  Groups with valid[k]
+// false hold -inf logits and do not enter the teacher finiteness check.
+template <int G>
+__device__ __forceinline__ void p1_chunk(const uint4 (&zw)[G], const uint4 (&tw)[G], const bool (&valid)[G], float& mz,
+                                         float& sz, float& mt, float& st, uint32_t& tmn) {
+  uint32_t zm = kNegInf2, tm = kNegInf2;
+#pragma unroll
+  for (int k = 0; k < G; ++k) {
+    zm = bmax2(zm, bmax2(bmax2(zw[k].x, zw[k].y), bmax2(zw[k].z, zw[k].w)));
+    tm = bmax2(tm, bmax2(bmax2(tw[k].x, tw[k].y), bmax2(tw[k].z, tw[k].w)));
+    if (valid[k]) tmn = bmin2_nan(tmn, bmin2_nan(bmin2_nan(tw[k].x, tw[k].y), bmin2_nan(tw[k].z, tw[k].w)));
+  }
   const float gz = fmaxf(bf_lo(zm), bf_hi(zm)) * kLog2e;
   const float gt = fmaxf(bf_lo(tm), bf_hi(tm)) * kLog2e;
   if (gz > mz) {
@@ -69,18 +77,22 @@ __device__ __forceinline__ void p1_group(const uint4& zw, const uint4& tw, float
     mt = gt;
   }
   const float mze = (mz == -INFINITY) ? 0.f : mz;
+  const float mte = (mt == -INFINITY) ? 0.f : mt;
   const float2 l2e = make_float2(kLog2e, kLog2e);
-  const float2 nmz = make_float2(-mze, -mze), nmt = make_float2(-mt, -mt);
-  const uint32_t zs[4] = {zw.x, zw.y, zw.z, zw.w};
-  const uint32_t ts[4] = {tw.x, tw.y, tw.z, tw.w};
+  const float2 nmz = make_float2(-mze, -mze), nmt = make_float2(-mte, -mte);
   float2 az = make_float2(0.f, 0.f), at = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const uint32_t zc = bmax2(zs[k], kNegInf2);  // NaN (inactive) -> -inf -> adds 0
-    const float2 ea = __ffma2_rn(make_float2(bf_lo(zc), bf_hi(zc)), l2e, nmz);
-    const float2 eb = __ffma2_rn(make_float2(bf_lo(ts[k]), bf_hi(ts[k])), l2e, nmt);
-    az = __fadd2_rn(az, make_float2(ex2(ea.x), ex2(ea.y)));
-    at = __fadd2_rn(at, make_float2(ex2(eb.x), ex2(eb.y)));
+  for (int k = 0; k < G; ++k) {
+    const uint32_t zs[4] = {zw[k].x, zw[k].y, zw[k].z, zw[k].w};
+    const uint32_t ts[4] = {tw[k].x, tw[k].y, tw[k].z, tw[k].w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t zc = bmax2(zs[q], kNegInf2);  // NaN (inactive) -> -inf -> adds 0
+      const float2 ea = __ffma2_rn(make_float2(bf_lo(zc), bf_hi(zc)), l2e, nmz);
+      const float2 eb = __ffma2_rn(make_float2(bf_lo(ts[q]), bf_hi(ts[q])), l2e, nmt);
+      az = __fadd2_rn(az, make_float2(ex2(ea.x), ex2(ea.y)));
+      at = __fadd2_rn(at, make_float2(ex2(eb.x), ex2(eb.y)));
+    }
   }
   sz += az.x + az.y;
   st += at.x + at.y;
@@ -125,8 +137,8 @@ constexpr int kRProd = 32;                       // producer warp
 constexpr int kRCons = 512;                      // consumer threads (16 warps)
 constexpr int kRThreads = kRProd + kRCons;
 constexpr int kRWarps = kRCons / 32;
-constexpr int kRChunk = 8192;                    // logits per chunk and array
-constexpr int kRSlots = 6;
+constexpr int kRChunk = 12288;                   // logits per chunk and array (3 groups per consumer)
+constexpr int kRSlots = 4;                        // 4 x 48 KB ring
 constexpr int kRGroups = kRChunk / 8;            // 16-byte groups per chunk and array
 constexpr uint32_t kRSlotBytes = 2u * kRChunk * 2u;
 
@@ -215,7 +227,7 @@ __global__ void __launch_bounds__(kRThreads, 1) tv_stats_bf16_ring_kernel(const 
     return;
   }
 
-  // ================= consumers (16 warps, one or two 16-byte groups per chunk each)
+  // ================= consumers (16 warps, three 16-byte groups of each array per chunk each)
   const int ct = tid - kRProd;
   const int cw = ct >> 5;
   long long n = 0;  // chunks consumed
@@ -234,13 +246,16 @@ __global__ void __launch_bounds__(kRThreads, 1) tv_stats_bf16_ring_kernel(const 
         const int ngc = (min(len8, (c + 1) * kRChunk) - c * kRChunk) / 8;
         const uint4* zs = reinterpret_cast<const uint4*>(ring + slot * kRSlotBytes);
         const uint4* ts = zs + kRGroups;
-        if (ct + kRCons < ngc) {
-          const uint4 z0 = zs[ct], t0 = ts[ct], z1 = zs[ct + kRCons], t1 = ts[ct + kRCons];
-          p1_group(z0, t0, mz, sz, mt, st, tmn);
-          p1_group(z1, t1, mz, sz, mt, st, tmn);
-        } else if (ct < ngc) {
-          p1_group(zs[ct], ts[ct], mz, sz, mt, st, tmn);
+        constexpr int G = kRGroups / kRCons;
+        uint4 zw[G], tw[G];
+        bool valid[G];
+#pragma unroll
+        for (int k = 0; k < G; ++k) {
+          valid[k] = ct + k * kRCons < ngc;
+          zw[k] = valid[k] ? zs[ct + k * kRCons] : make_uint4(kNegInf2, kNegInf2, kNegInf2, kNegInf2);
+          tw[k] = valid[k] ? ts[ct + k * kRCons] : make_uint4(kNegInf2, kNegInf2, kNegInf2, kNegInf2);
         }
+        p1_chunk<G>(zw, tw, valid, mz, sz, mt, st, tmn);
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->empty[slot]);
       }
@@ -308,17 +323,13 @@ __global__ void __launch_bounds__(kRThreads, 1) tv_stats_bf16_ring_kernel(const 
         const uint4* ts = zs + kRGroups;
         uint8_t* mc = mrow ? mrow + (long long)c * kRGroups : nullptr;
         if (live) {
-          if (ct + kRCons < ngc) {
-            const uint4 z0 = zs[ct], t0 = ts[ct], z1 = zs[ct + kRCons], t1 = ts[ct + kRCons];
-            const uint32_t b0 = p2_group(z0, t0, nlz, nlt, acc_a, acc_q);
-            const uint32_t b1 = p2_group(z1, t1, nlz, nlt, acc_a, acc_q);
-            if (mc) {
-              mc[ct] = (uint8_t)b0;
-              mc[ct + kRCons] = (uint8_t)b1;
+#pragma unroll
+          for (int k = 0; k < kRGroups / kRCons; ++k) {
+            const int g = ct + k * kRCons;
+            if (g < ngc) {
+              const uint32_t b0 = p2_group(zs[g], ts[g], nlz, nlt, acc_a, acc_q);
+              if (mc) mc[g] = (uint8_t)b0;
             }
-          } else if (ct < ngc) {
-            const uint32_t b0 = p2_group(zs[ct], ts[ct], nlz, nlt, acc_a, acc_q);
-            if (mc) mc[ct] = (uint8_t)b0;
           }
         } else if (mc) {  // no active draft logit: q = 0 everywhere
           for (int g = ct; g < ngc; g += kRCons) mc[g] = 0;
@@ -427,7 +438,7 @@ __global__ void __launch_bounds__(kGradThreads) tv_grad_bf16_kernel(const Overla
 
 }  // namespace
 
-// Persistent ring statistics kernel: one CTA per SM (about 194 KB of ring),
+// Persistent ring statistics kernel: one CTA per SM (192 KB of ring),
 // at most one CTA per row.
 cudaError_t launch_tv_stats_bf16(const OverlapArgs& a, cudaStream_t stream) {
   if (a.rows == 0) return cudaSuccess;
