@@ -14,7 +14,8 @@
 //    one thread of warp 1 issues tcgen05.mma: S = Q K^T into TMEM, then
 //    O += P V with P read straight from TMEM;
 //  * warps 4-7 and 8-11 (one warpgroup per query head) own one query row per
-//    thread: they read S from TMEM, mask, run the online softmax in base 2,
+//    thread, with 216 registers each (the TMA/MMA warpgroup gives up its
+//    share): they read S from TMEM, mask, run the online softmax in base 2,
 //    write P (bf16) back over S, and rescale O in TMEM only when the running
 //    maximum grows by more than 2^8 (the stale maximum is exact: the same
 //    reference enters numerator and denominator);
@@ -77,6 +78,12 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ int block_col(const specopd_tile_meta& m, int n_trunk, int j) {
   return j < n_trunk ? m.tree_base + j * kBN : m.br_lo + (j - n_trunk) * kBN;
 }
@@ -133,7 +140,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm->tmem_base;
   volatile int* abort_flag = &sm->abort_flag;
 
-  if (warp == 0) {
+  // Registers: the TMA/MMA warpgroup needs few, the two softmax warpgroups
+  // (a query row of 128 scores per thread) many; 128 x 72 + 256 x 216 equals
+  // the 384 x 168 the block is launched with.
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
+    if (warp == 0) {
     // ================= TMA producer
     if (lane == 0) {
       mbar_arrive_expect_tx(&sm->q_full, nq * kTileBytes);
@@ -156,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < kSlots; ++s)
         if (last_n[s] >= 0) drain_wait(&sm->kv_full[s], (last_n[s] / kSlots) & 1);
     }
-  } else if (warp == 1) {
+    } else if (warp == 1) {
     // ================= MMA issuer (one thread)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
@@ -211,7 +223,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(&sm->mma_done);
       drain_wait(&sm->mma_done, 0);
     }
-  } else if (warp >= 4) {
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 216;");
     // ================= softmax: one warpgroup per query head, one row per thread
     const int t = (warp - 4) >> 2;
     if (t < nq) {
@@ -259,9 +273,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        float mx = -INFINITY;
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-        for (int e = 0; e < 128; ++e) mx = fmaxf(mx, s[e]);
+        for (int e = 4; e < 128; e += 8) {
+          mx0 = fmax3(mx0, s[e], s[e + 1]);
+          mx1 = fmax3(mx1, s[e + 2], s[e + 3]);
+          mx2 = fmax3(mx2, s[e + 4], s[e + 5]);
+          mx3 = fmax3(mx3, s[e + 6], s[e + 7]);
+        }
+        const float mx = fmax3(fmaxf(mx0, mx1), mx2, mx3);
         const float m_new = fmaxf(m_use, mx * p.scale_log2);
         float corr = 1.f;
         bool rescale = false;
@@ -271,16 +291,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           rescale = j > 0;
         }
         const float m_eff = (m_use == -INFINITY) ? 0.f : m_use;
-        float rowsum = 0.f;
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 nm2 = make_float2(-m_eff, -m_eff);
+        float2 acc[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) acc[a] = make_float2(0.f, 0.f);
         uint32_t pk[64];
 #pragma unroll
         for (int e = 0; e < 64; ++e) {
-          const float p0 = ex2(fmaf(s[2 * e], p.scale_log2, -m_eff));
-          const float p1 = ex2(fmaf(s[2 * e + 1], p.scale_log2, -m_eff));
-          rowsum += p0 + p1;
-          pk[e] = pack_bf16x2(p0, p1);
+          const float2 x = __ffma2_rn(make_float2(s[2 * e], s[2 * e + 1]), sc2, nm2);
+          const float2 pe = make_float2(ex2(x.x), ex2(x.y));
+          acc[e & 3] = __fadd2_rn(acc[e & 3], pe);
+          pk[e] = pack_bf16x2(pe.x, pe.y);
         }
-        l = l * corr + rowsum;
+        acc[0] = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+        l = l * corr + (acc[0].x + acc[0].y);
         tmem_st32(trow + s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
         tmem_st32(trow + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
         tmem_st_wait();
