@@ -32,6 +32,13 @@ sys.path.insert(0, ROOT)
 METRIC = "supervised tokens/s scored (tree attn + E2E-TV) on 1 B200; % of roofline"
 WORKLOAD_DEFAULT = 2
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per step of a
+# step's kernels, from one ncu capture of each kernel on the gqa8b workload.
+# They hold only for the kernels they were taken on; a workload without a
+# capture reports null.  Overlap pass: statistics 652.701184 + 19.878656 MB,
+# gradient 330.643712 + 563.444992 MB.  Attention: 63.078144 + 6.784256 MB.
+MEASURED_TRAFFIC = {2: {"tv_overlap_e2e": 1566.668544e6, "tree_attention": 69.8624e6}}
+
 
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -306,7 +313,7 @@ def run_gpu(args):
     dom = "tree_attention" if t_attn >= t_ov else "tv_overlap_e2e"
     kd = kernels[dom]
     roofline = {"bound": kd["bound"], "achieved": kd["achieved"], "peak": kd["peak"], "unit": kd["unit"],
-                "frac": kd["frac"], "traffic": None, "kernel": dom,
+                "frac": kd["frac"], "traffic": MEASURED_TRAFFIC.get(args.workload, {}).get(dom), "kernel": dom,
                 "peak_source": f"{peaks['source']} ({'bf16_tflops burst' if dom == 'tree_attention' else 'hbm_gbs'})"}
     tokens = figs["R"] * world
     value = tokens * K / (elapsed_ms * 1e-3)
