@@ -6,6 +6,15 @@
 
 namespace specopd {
 
+// atomic add at GPU scope with acquire-release ordering: the caller's earlier
+// writes are visible to whoever reads the new count, and writes released by
+// earlier adders are visible to the caller
+__device__ __forceinline__ unsigned atomic_add_acq_rel(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 // (m, s) pairs of a base-2 log-sum-exp: value = m + log2(s)
 __device__ __forceinline__ void lse_merge(float& m, float& s, float m2, float s2) {
   const float mn = fmaxf(m, m2);
@@ -29,31 +38,49 @@ __device__ inline void row_epilogue(const OverlapArgs& a, long long row, float a
   if (!a.branch_cnt) return;
   const int W = a.W;
   const long long b = row / W;
-  __threadfence();
-  const unsigned old = atomicAdd(&a.branch_cnt[b], 1u);
+  // release: this row's alpha precedes the count; acquire for the last row:
+  // every other row's alpha is visible to it
+  const unsigned old = atomic_add_acq_rel(&a.branch_cnt[b], 1u);
   if (old != (unsigned)(W - 1)) return;
-  __threadfence();
+  // the branch's alphas, fetched in batches of independent loads (one L2
+  // round trip per batch instead of one per alpha)
   const float* al_b = a.alpha + b * W;
+  float al[SPECOPD_MAX_W];
+  for (int i0 = 0; i0 < W; i0 += 16) {
+    float v[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) v[u] = (i0 + u < W) ? __ldcg(al_b + i0 + u) : 0.f;
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+      if (i0 + u < W) al[i0 + u] = v[u];
+  }
   double pre[SPECOPD_MAX_W + 1];
   pre[0] = 1.0;
   double share = 0.0;
   for (int i = 1; i <= W; ++i) {
-    pre[i] = pre[i - 1] * (double)__ldcg(al_b + i - 1);
+    pre[i] = pre[i - 1] * (double)al[i - 1];
     share += pre[i];
   }
   // S_i = 1 + alpha_{i+1} S_{i+1}, S_W = 1; g_i = -(1/count) pre_{i-1} S_i
   double S = 1.0;
   for (int i = W; i >= 1; --i) {
     a.g[b * W + i - 1] = (float)(-a.inv_count * pre[i - 1] * S);
-    S = 1.0 + (double)__ldcg(al_b + i - 1) * S;
+    S = 1.0 + (double)al[i - 1] * S;
   }
   a.branch_sum[b] = share;
-  __threadfence();
-  const unsigned done = atomicAdd(&a.branch_cnt[a.num_branches], 1u);
+  const unsigned done = atomic_add_acq_rel(&a.branch_cnt[a.num_branches], 1u);
   if (done != (unsigned)(a.num_branches - 1)) return;
-  __threadfence();
+  // the shares in branch order (the same additions, in the same order, as one
+  // at a time), fetched in batches of independent loads
   double total = 0.0;
-  for (long long k = 0; k < a.num_branches; ++k) total += __ldcg(a.branch_sum + k);
+  for (long long k0 = 0; k0 < a.num_branches; k0 += 32) {
+    double v[32];
+#pragma unroll
+    for (int u = 0; u < 32; ++u) v[u] = (k0 + u < a.num_branches) ? __ldcg(a.branch_sum + k0 + u) : 0.0;
+#pragma unroll
+    for (int u = 0; u < 32; ++u)
+      if (k0 + u < a.num_branches) total += v[u];
+  }
   *a.loss = (float)(1.0 - total * a.inv_count);
 }
 

@@ -126,14 +126,15 @@ __device__ __forceinline__ uint32_t p2_group(const uint4& zw, const uint4& tw, f
 //             evict_last) into the online base-2 (max, sum) of both softmaxes;
 //   pass 2 -- the same bytes again, an L2 hit (one row per SM is a small part
 //             of the L2), for alpha, q_less and the [q < p] bits.
-// Warp 0 is the producer: one thread walks the chunk sequence
-// P1(row), P2(row), P1(next row), ... and bulk-copies each chunk of draft and
-// teacher logits into the next free slot (no multicast).  The other warps
-// consume the slots in the same order, so the copies run ahead through the
-// reductions between the passes.  Per-row reductions use fixed shuffle trees
+// Warp 0 is the producer and warp 1 the row epilogue.  The producer walks the
+// chunk sequence P1(row), P2(row), P1(next row), ... and bulk-copies each
+// chunk of draft and teacher logits into the next free slot (no multicast);
+// the epilogue warp takes each row's results from a two-entry queue and runs
+// the E2E-TV row epilogue.  The other warps consume the slots in the same
+// order, so the copies run ahead through the reductions between the passes.  Per-row reductions use fixed shuffle trees
 // (reproducible results).  All waits are bounded; the consumer warps always
 // pass the same named barriers, whatever happened, so none can be left behind.
-constexpr int kRProd = 32;                       // producer warp
+constexpr int kRProd = 64;                       // producer warp, epilogue warp
 constexpr int kRCons = 512;                      // consumer threads (16 warps)
 constexpr int kRThreads = kRProd + kRCons;
 constexpr int kRWarps = kRCons / 32;
@@ -145,8 +146,10 @@ constexpr uint32_t kRSlotBytes = 2u * kRChunk * 2u;
 struct RingCtl {
   uint64_t full[kRSlots];
   uint64_t empty[kRSlots];
-  float red[kRWarps][4];
-  float bcast[2];
+  uint64_t epi_full[2];   // a row's results are queued for the epilogue lane
+  uint64_t epi_empty[2];  // the epilogue lane has taken them
+  float epi[2][4];        // (alpha, q_less, lz2, lt2) of the queued row
+  int epi_bad[2];
   int abort_flag;
 };
 
@@ -187,15 +190,19 @@ __global__ void __launch_bounds__(kRThreads, 1) tv_stats_bf16_ring_kernel(const 
       mbar_init(&ctl->full[s], 1);
       mbar_init(&ctl->empty[s], kRWarps);
     }
+    for (int e = 0; e < 2; ++e) {
+      mbar_init(&ctl->epi_full[e], 1);
+      mbar_init(&ctl->epi_empty[e], 1);
+    }
     ctl->abort_flag = 0;
     fence_barrier_init();
   }
   __syncthreads();
   volatile int* abort_flag = &ctl->abort_flag;
 
-  if (warp == 0) {
+  if (warp < kRProd / 32) {
     // ================= producer: chunk sequence P1(row), P2(row), P1(next row), ...
-    if (lane == 0) {
+    if (warp == 0 && lane == 0) {
       const uint64_t pol_keep = l2_policy_evict_last();
       const uint64_t pol_drop = l2_policy_evict_first();
       long long n = 0;  // chunks issued
@@ -223,6 +230,20 @@ __global__ void __launch_bounds__(kRThreads, 1) tv_stats_bf16_ring_kernel(const 
       for (long long k = (n > kRSlots ? n - kRSlots : 0); k < n; ++k)
         ring_drain_wait(&ctl->full[k % kRSlots], (uint32_t)(k / kRSlots) & 1u);
       if (ctl->abort_flag) atomicOr(reinterpret_cast<unsigned*>(a.status), SPECOPD_FLAG_TIMEOUT);
+    } else if (warp == 1 && lane == 0) {
+      // ================= row epilogue in a warp of its own, off the
+      // consumers' and the producer's paths (its atomics and the branch's
+      // last-arriver loads are long round trips)
+      int i = 0;
+      for (long long row = blockIdx.x; row < a.rows; row += gridDim.x, ++i) {
+        const int e = i & 1;
+        if (!mbar_wait(&ctl->epi_full[e], (uint32_t)(i >> 1) & 1u, abort_flag)) break;
+        const float x = ctl->epi[e][0], y = ctl->epi[e][1], lz2 = ctl->epi[e][2], lt2 = ctl->epi[e][3];
+        const int bad = ctl->epi_bad[e];
+        mbar_arrive(&ctl->epi_empty[e]);
+        if (bad) atomicOr(reinterpret_cast<unsigned*>(a.status), SPECOPD_FLAG_NONFINITE);
+        row_epilogue(a, row, x, y, lz2, lt2);
+      }
     }
     return;
   }
@@ -232,7 +253,8 @@ __global__ void __launch_bounds__(kRThreads, 1) tv_stats_bf16_ring_kernel(const 
   const int cw = ct >> 5;
   long long n = 0;  // chunks consumed
   bool ok = true;   // uniform per warp; a failed wait only skips work, never a barrier
-  for (long long row = blockIdx.x; row < a.rows; row += gridDim.x) {
+  long long irow = 0;  // rows of this CTA so far
+  for (long long row = blockIdx.x; row < a.rows; row += gridDim.x, ++irow) {
     const __nv_bfloat16* zrow = static_cast<const __nv_bfloat16*>(a.draft) + row * a.ld_draft;
     const __nv_bfloat16* trow = static_cast<const __nv_bfloat16*>(a.teacher) + row * a.ld_teacher;
 
@@ -369,10 +391,16 @@ __global__ void __launch_bounds__(kRThreads, 1) tv_stats_bf16_ring_kernel(const 
         x += __shfl_xor_sync(0xffffffffu, x, off);
         y += __shfl_xor_sync(0xffffffffu, y, off);
       }
-      if (lane == 0) {
-        if (row_bad) atomicOr(reinterpret_cast<unsigned*>(a.status), SPECOPD_FLAG_NONFINITE);
-        if (!live) x = y = 0.f;
-        row_epilogue(a, row, x, y, lz2, lt2);
+      if (lane == 0) {  // queue the row's results for the epilogue lane
+        const int e = (int)(irow & 1);
+        if (irow < 2 || mbar_wait(&ctl->epi_empty[e], (uint32_t)((irow >> 1) - 1) & 1u, abort_flag)) {
+          ctl->epi[e][0] = live ? x : 0.f;
+          ctl->epi[e][1] = live ? y : 0.f;
+          ctl->epi[e][2] = lz2;
+          ctl->epi[e][3] = lt2;
+          ctl->epi_bad[e] = row_bad ? 1 : 0;
+          mbar_arrive(&ctl->epi_full[e]);
+        }
       }
     }
   }
