@@ -35,9 +35,9 @@ WORKLOAD_DEFAULT = 2
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per step of a
 # step's kernels, from one ncu capture of each kernel on the gqa8b workload.
 # They hold only for the kernels they were taken on; a workload without a
-# capture reports null.  Overlap pass: statistics 652.701184 + 19.878656 MB,
-# gradient 330.643712 + 563.444992 MB.  Attention: 63.078144 + 6.784256 MB.
-MEASURED_TRAFFIC = {2: {"tv_overlap_e2e": 1566.668544e6, "tree_attention": 69.8624e6}}
+# capture reports null.  Overlap pass: statistics 660.049664 + 19.913472 MB,
+# gradient 330.666240 + 566.113536 MB.  Attention: 63.078144 + 6.784256 MB.
+MEASURED_TRAFFIC = {2: {"tv_overlap_e2e": 1576.742912e6, "tree_attention": 69.8624e6}}
 
 
 def load_peaks():
