@@ -35,9 +35,9 @@ WORKLOAD_DEFAULT = 2
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per step of a
 # step's kernels, from one ncu capture of each kernel on the gqa8b workload.
 # They hold only for the kernels they were taken on; a workload without a
-# capture reports null.  Overlap pass: statistics 660.049664 + 19.913472 MB,
-# gradient 330.666240 + 566.113536 MB.  Attention: 63.078144 + 6.784256 MB.
-MEASURED_TRAFFIC = {2: {"tv_overlap_e2e": 1576.742912e6, "tree_attention": 69.8624e6}}
+# capture reports null.  Overlap pass (statistics + gradient in one launch):
+# 1193.076 + 585.014272 MB.  Attention: 63.078144 + 6.784256 MB.
+MEASURED_TRAFFIC = {2: {"tv_overlap_e2e": 1778.090272e6, "tree_attention": 69.8624e6}}
 
 
 def load_peaks():
@@ -331,7 +331,7 @@ def run_gpu(args):
         "clocks": clk,
         "e2e": {"value": tokens * Ke / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / Ke, "steps": Ke},
-        "gpu_launches": 5 * K,
+        "gpu_launches": 4 * K,  # mask, RoPE, attention, fused overlap (statistics + gradient)
         "device_status": status,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -228,7 +228,10 @@ int specopd_e2e_tv_loss(const float* alpha, int64_t num_branches, int W, double 
  * last branch forms L.  With grad_draft non-null a second streaming pass
  * writes dL/dz = dL/dalpha * q (1[q < p] - sum_v q_v 1[q_v < p_v]) (zero on
  * entries outside the draft support); samples and teacher are held fixed
- * (write-up, section "Equations").
+ * (write-up, section "Equations").  For bf16 with a gradient, both passes run
+ * in one cooperative launch with one CTA per SM (the gradient of a branch
+ * starts on the SMs as soon as its dL/dalpha is final); if the device
+ * refuses the cooperative launch the call returns SPECOPD_ERR_CUDA.
  *
  * Rows are predictions b-major: row b*W + i-1 holds the logits read out for
  * y_{b,i}.  rows must equal num_branches * W.  count <= 0 means rows.

@@ -212,6 +212,8 @@ int specopd_tv_overlap(const void* draft, const void* teacher, specopd_dtype dty
   a.ld_teacher = ld_teacher;
   a.rows = rows;
   a.V = V;
+  a.row_begin = 0;
+  a.row_end = rows;
   a.alpha = alpha;
   a.q_less = q_less;
   a.lse_draft = lse_draft;
@@ -257,6 +259,8 @@ int specopd_tv_overlap_e2e(const void* draft, const void* teacher, specopd_dtype
   a.ld_teacher = ld_teacher;
   a.rows = rows;
   a.V = V;
+  a.row_begin = 0;
+  a.row_end = rows;
   a.alpha = alpha;
   a.mbits = grad_draft ? ws + L.mbits : nullptr;
   a.mbits_ld = L.mbits_ld;
@@ -275,9 +279,15 @@ int specopd_tv_overlap_e2e(const void* draft, const void* teacher, specopd_dtype
   a.status = status;
   cudaError_t e = cudaMemsetAsync(counters, 0, L.counters_bytes, st);
   if (e != cudaSuccess) return SPECOPD_ERR_CUDA;
+  if (dtype == SPECOPD_BF16 && grad_draft) {
+    e = launch_tv_fused_bf16(a, st);
+    return e == cudaSuccess ? SPECOPD_OK : SPECOPD_ERR_CUDA;
+  }
   e = launch_tv_stats(a, dtype, st);
   if (e != cudaSuccess) return SPECOPD_ERR_CUDA;
   if (grad_draft) {
+    a.grad_begin = 0;
+    a.grad_end = rows;
     e = launch_tv_grad(a, dtype, st);
     if (e != cudaSuccess) return SPECOPD_ERR_CUDA;
   }

@@ -54,6 +54,11 @@ struct OverlapArgs {
   const void* teacher;
   int64_t ld_draft, ld_teacher;
   int64_t rows, V;
+  // one launch computes the statistics of rows [row_begin, row_end) and the
+  // gradient of rows [grad_begin, grad_end) (an empty range: no gradient);
+  // per-row and per-branch outputs are indexed by the global row
+  int64_t row_begin, row_end;
+  int64_t grad_begin, grad_end;
   // outputs of the statistics pass
   float* alpha;
   float* q_less;     // nullable
@@ -78,9 +83,10 @@ struct OverlapArgs {
 };
 
 cudaError_t launch_tv_stats(const OverlapArgs& a, specopd_dtype dtype, cudaStream_t stream);
-// bf16 kernels (tv_bf16.cu); launch_tv_stats / launch_tv_grad route bf16 here
+// bf16 kernels (tv_bf16.cu); launch_tv_stats routes bf16 here
 cudaError_t launch_tv_stats_bf16(const OverlapArgs& a, cudaStream_t stream);
-cudaError_t launch_tv_grad_bf16(const OverlapArgs& a, cudaStream_t stream);
+// bf16 statistics + gradient in one cooperative launch (the only bf16 gradient path)
+cudaError_t launch_tv_fused_bf16(OverlapArgs a, cudaStream_t stream);
 cudaError_t launch_tv_grad(const OverlapArgs& a, specopd_dtype dtype, cudaStream_t stream);
 cudaError_t launch_e2e_loss(const float* alpha, int64_t num_branches, int W, double inv_count, float* loss,
                             float* grad_alpha, cudaStream_t stream);

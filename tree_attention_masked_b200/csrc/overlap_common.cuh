@@ -15,6 +15,14 @@ __device__ __forceinline__ unsigned atomic_add_acq_rel(unsigned* p, unsigned v) 
   return old;
 }
 
+// load at GPU scope with acquire ordering: writes released before the value
+// was stored are visible to the caller's later reads
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // (m, s) pairs of a base-2 log-sum-exp: value = m + log2(s)
 __device__ __forceinline__ void lse_merge(float& m, float& s, float m2, float s2) {
   const float mn = fmaxf(m, m2);
@@ -67,6 +75,9 @@ __device__ inline void row_epilogue(const OverlapArgs& a, long long row, float a
     a.g[b * W + i - 1] = (float)(-a.inv_count * pre[i - 1] * S);
     S = 1.0 + (double)al[i - 1] * S;
   }
+  // publish the branch's dL/dalpha: its count becomes W + 1 (release), which
+  // gradient warps of the same launch wait for (acquire)
+  atomic_add_acq_rel(&a.branch_cnt[b], 1u);
   a.branch_sum[b] = share;
   const unsigned done = atomic_add_acq_rel(&a.branch_cnt[a.num_branches], 1u);
   if (done != (unsigned)(a.num_branches - 1)) return;

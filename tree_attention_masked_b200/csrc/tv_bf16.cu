@@ -1,5 +1,5 @@
-// K4/K5 for bf16 logits: per-row overlap statistics (persistent ring kernel)
-// and the streaming gradient.
+// K4/K5 for bf16 logits: per-row overlap statistics and the gradient with
+// respect to the draft logits, in one persistent ring kernel.
 //
 // daiwk.github.io write-up of SpecOPD, section "Equations": alpha = sum_v
 // min(q(v), p(v)); L = 1 - (1/(B W)) sum_b sum_j prod_{i<=j} alpha_{b,i};
@@ -13,8 +13,11 @@
 // and every copy goes through a ring of shared-memory slots fed by one
 // producer thread, so HBM reads run ahead of the arithmetic and through the
 // reductions between the passes.  Gradient: dL/dz = g q ([q < p] - q_less)
-// from the draft logits and the bits written by pass 2; every warp access is
-// contiguous.
+// from the draft logits and the bits written by pass 2.  The statistics are
+// bound by instruction issue and the gradient by HBM, so the same kernel runs
+// both side by side: gradient warps on every SM stream the gradient of the
+// rows whose branch is already finished while the consumer warps work on the
+// next rows.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -126,20 +129,33 @@ __device__ __forceinline__ uint32_t p2_group(const uint4& zw, const uint4& tw, f
 //             evict_last) into the online base-2 (max, sum) of both softmaxes;
 //   pass 2 -- the same bytes again, an L2 hit (one row per SM is a small part
 //             of the L2), for alpha, q_less and the [q < p] bits.
-// Warp 0 is the producer and warp 1 the row epilogue.  The producer walks the
-// chunk sequence P1(row), P2(row), P1(next row), ... and bulk-copies each
-// chunk of draft and teacher logits into the next free slot (no multicast);
-// the epilogue warp takes each row's results from a two-entry queue and runs
-// the E2E-TV row epilogue.  The other warps consume the slots in the same
-// order, so the copies run ahead through the reductions between the passes.  Per-row reductions use fixed shuffle trees
-// (reproducible results).  All waits are bounded; the consumer warps always
-// pass the same named barriers, whatever happened, so none can be left behind.
-constexpr int kRProd = 64;                       // producer warp, epilogue warp
-constexpr int kRCons = 512;                      // consumer threads (16 warps)
-constexpr int kRThreads = kRProd + kRCons;
+// Warp 0 is the producer, warp 1 the row epilogue and warp 2 the gradient
+// producer.  The producer walks the chunk sequence P1(row), P2(row), P1(next
+// row), ... and bulk-copies each chunk of draft and teacher logits into the
+// next free slot (no multicast); the epilogue warp takes each row's results
+// from a two-entry queue and runs the E2E-TV row epilogue, which publishes a
+// branch's dL/dalpha once its last row is in.  The 16 consumer warps consume
+// the slots in the same order, so the copies run ahead through the reductions
+// between the passes.  The 8 gradient warps stream the gradient of this CTA's
+// rows once published (grad_producer / grad_consumer below).  Per-row
+// reductions use fixed shuffle trees (reproducible results).  All waits are
+// bounded; the consumer warps always pass the same named barriers, whatever
+// happened, so none can be left behind.
+constexpr int kRHead = 128;                      // warpgroup 0: producer warp, epilogue warp, 2 idle
+constexpr int kRCons = 512;                      // consumer threads (16 warps, warpgroups 1-4)
+constexpr int kRGradWarps = 8;                   // gradient warps (warpgroups 5-6)
+constexpr int kGUnit = 8192;                     // logits per gradient stage
+constexpr int kGStages = 4;
+constexpr uint32_t kGStageBytes = kGUnit * 2 + kGUnit / 8;  // draft logits + bits
+constexpr int kRThreads = kRHead + kRCons + 32 * kRGradWarps;
 constexpr int kRWarps = kRCons / 32;
+// registers per thread: 72 at launch (896 threads), then warpgroup 0 drops to
+// 56, the gradient warpgroups to 48 and the consumers rise to 88
+constexpr int kRRegLaunch = 72, kRRegHead = 56, kRRegCons = 88, kRRegGrad = 48;
+static_assert(kRHead * kRRegHead + kRCons * kRRegCons + 32 * kRGradWarps * kRRegGrad <= kRThreads * kRRegLaunch,
+              "register split exceeds the launch's registers");
 constexpr int kRChunk = 12288;                   // logits per chunk and array (3 groups per consumer)
-constexpr int kRSlots = 4;                        // 4 x 48 KB ring
+constexpr int kRSlots = 3;                        // 3 x 48 KB ring
 constexpr int kRGroups = kRChunk / 8;            // 16-byte groups per chunk and array
 constexpr uint32_t kRSlotBytes = 2u * kRChunk * 2u;
 
@@ -161,13 +177,35 @@ __device__ __forceinline__ void bulk_g2s_policy(void* dst, const void* src, uint
       "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
       : "memory");
 }
+// 16-byte store that skips L1 and enters L2 with the given eviction policy
+// (evict_first for the gradient, so it does not push the statistics' pass-1
+// rows out of the L2 before pass 2 re-reads them)
+__device__ __forceinline__ void st_global_v4_policy(float* p, const float4& v, uint64_t pol) {
+  asm volatile("st.global.L1::no_allocate.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(v.x),
+               "f"(v.y), "f"(v.z), "f"(v.w), "l"(pol)
+               : "memory");
+}
 __device__ __forceinline__ void cons_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kRCons) : "memory"); }
+
+struct GradCtl {
+  uint64_t full[kGStages];
+  uint64_t empty[kGStages];
+  float info[kGStages][4];  // (lz2, q_less, dL/dalpha) of the stage's row
+};
 
 struct RingRed {
   float r1[kRWarps][4];  // pass-1 partials (mz, sz, mt, st) by consumer warp
   float r2[kRWarps][2];  // pass-2 partials (alpha, q_less)
   int bad[kRWarps];
 };
+
+// shared memory: ring slots | RingCtl | RingRed | GradCtl | gradient stages
+constexpr size_t kRCtlOff = (size_t)kRSlots * kRSlotBytes;
+constexpr size_t kRRedOff = kRCtlOff + sizeof(RingCtl);
+constexpr size_t kGCtlOff = kRRedOff + sizeof(RingRed);
+constexpr size_t kGBufOff = (kGCtlOff + sizeof(GradCtl) + 127) / 128 * 128;
+constexpr size_t kRSmem = kGBufOff + (size_t)kGStages * kGStageBytes;
+static_assert(kRSmem <= 232448, "ring kernel exceeds the shared memory of a CTA");
 
 __device__ __forceinline__ void ring_drain_wait(uint64_t* bar, uint32_t parity) {
   const long long t0 = clock64();
@@ -176,11 +214,17 @@ __device__ __forceinline__ void ring_drain_wait(uint64_t* bar, uint32_t parity) 
   }
 }
 
+__device__ void grad_producer(const OverlapArgs& a, GradCtl* gc, uint8_t* gbuf, volatile int* abort_flag);
+__device__ void grad_consumer(const OverlapArgs& a, GradCtl* gc, const uint8_t* gbuf, volatile int* abort_flag, int gw,
+                              int lane);
+
 __global__ void __launch_bounds__(kRThreads, 1) tv_stats_bf16_ring_kernel(const OverlapArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* ring = smem;
-  RingCtl* ctl = reinterpret_cast<RingCtl*>(ring + kRSlots * kRSlotBytes);
-  RingRed* rr = reinterpret_cast<RingRed*>(ctl + 1);
+  RingCtl* ctl = reinterpret_cast<RingCtl*>(smem + kRCtlOff);
+  RingRed* rr = reinterpret_cast<RingRed*>(smem + kRRedOff);
+  GradCtl* gc = reinterpret_cast<GradCtl*>(smem + kGCtlOff);
+  uint8_t* gbuf = smem + kGBufOff;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int len8 = (int)(a.V & ~7LL);
   const int tail = (int)(a.V - len8);
@@ -194,20 +238,25 @@ __global__ void __launch_bounds__(kRThreads, 1) tv_stats_bf16_ring_kernel(const 
       mbar_init(&ctl->epi_full[e], 1);
       mbar_init(&ctl->epi_empty[e], 1);
     }
+    for (int g = 0; g < kGStages; ++g) {
+      mbar_init(&gc->full[g], 1);
+      mbar_init(&gc->empty[g], kRGradWarps);
+    }
     ctl->abort_flag = 0;
     fence_barrier_init();
   }
   __syncthreads();
   volatile int* abort_flag = &ctl->abort_flag;
 
-  if (warp < kRProd / 32) {
+  if (warp < kRHead / 32) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRRegHead));
     // ================= producer: chunk sequence P1(row), P2(row), P1(next row), ...
     if (warp == 0 && lane == 0) {
       const uint64_t pol_keep = l2_policy_evict_last();
       const uint64_t pol_drop = l2_policy_evict_first();
       long long n = 0;  // chunks issued
       bool ok = true;
-      for (long long row = blockIdx.x; ok && row < a.rows; row += gridDim.x) {
+      for (long long row = a.row_begin + blockIdx.x; ok && row < a.row_end; row += gridDim.x) {
         const __nv_bfloat16* zrow = static_cast<const __nv_bfloat16*>(a.draft) + row * a.ld_draft;
         const __nv_bfloat16* trow = static_cast<const __nv_bfloat16*>(a.teacher) + row * a.ld_teacher;
         for (int pass = 0; ok && pass < 2; ++pass) {
@@ -235,7 +284,7 @@ __global__ void __launch_bounds__(kRThreads, 1) tv_stats_bf16_ring_kernel(const 
       // consumers' and the producer's paths (its atomics and the branch's
       // last-arriver loads are long round trips)
       int i = 0;
-      for (long long row = blockIdx.x; row < a.rows; row += gridDim.x, ++i) {
+      for (long long row = a.row_begin + blockIdx.x; row < a.row_end; row += gridDim.x, ++i) {
         const int e = i & 1;
         if (!mbar_wait(&ctl->epi_full[e], (uint32_t)(i >> 1) & 1u, abort_flag)) break;
         const float x = ctl->epi[e][0], y = ctl->epi[e][1], lz2 = ctl->epi[e][2], lt2 = ctl->epi[e][3];
@@ -244,17 +293,28 @@ __global__ void __launch_bounds__(kRThreads, 1) tv_stats_bf16_ring_kernel(const 
         if (bad) atomicOr(reinterpret_cast<unsigned*>(a.status), SPECOPD_FLAG_NONFINITE);
         row_epilogue(a, row, x, y, lz2, lt2);
       }
+    } else if (warp == 2 && lane == 0) {
+      // ================= gradient producer: stages of finished rows
+      grad_producer(a, gc, gbuf, abort_flag);
     }
     return;
   }
 
+  if (warp >= (kRHead + kRCons) / 32) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRRegGrad));
+    // ================= gradient of rows finished by an earlier launch
+    grad_consumer(a, gc, gbuf, abort_flag, warp - (kRHead + kRCons) / 32, lane);
+    return;
+  }
+
   // ================= consumers (16 warps, three 16-byte groups of each array per chunk each)
-  const int ct = tid - kRProd;
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRRegCons));
+  const int ct = tid - kRHead;
   const int cw = ct >> 5;
   long long n = 0;  // chunks consumed
   bool ok = true;   // uniform per warp; a failed wait only skips work, never a barrier
   long long irow = 0;  // rows of this CTA so far
-  for (long long row = blockIdx.x; row < a.rows; row += gridDim.x, ++irow) {
+  for (long long row = a.row_begin + blockIdx.x; row < a.row_end; row += gridDim.x, ++irow) {
     const __nv_bfloat16* zrow = static_cast<const __nv_bfloat16*>(a.draft) + row * a.ld_draft;
     const __nv_bfloat16* trow = static_cast<const __nv_bfloat16*>(a.teacher) + row * a.ld_teacher;
 
@@ -407,89 +467,166 @@ __global__ void __launch_bounds__(kRThreads, 1) tv_stats_bf16_ring_kernel(const 
 }
 
 // ---------------- gradient
-// A warp covers 512 consecutive logits per pass: lane l owns logits 4l..4l+3
-// of each 128-logit step, so every load (8 bytes of draft logits, one byte of
-// bits) and every store (16 bytes of gradient) is contiguous across the warp.
-// The four steps' loads are all issued before any arithmetic.
-constexpr int kGradThreads = 256;
-constexpr int kGradSteps = 4;
-constexpr int kGradElemsPerWarp = 128 * kGradSteps;
+// The ring kernel's gradient side.  CTA c takes rows grad_begin + c, + gridDim.x,
+// ... (the rows whose statistics it computed, when both ranges coincide).  A
+// row waits until its branch's dL/dalpha is published (count W + 1, set by
+// the branch's last row in this launch); then one producer thread streams
+// its draft logits and bits through kGStages stages of shared memory (bulk
+// copies, L2 evict_first, no multicast) and the gradient warps write
+// dL/dz = g q ([q < p] - q_less) with 16-byte streaming stores.  The launch
+// is cooperative: every CTA is resident and the statistics never wait for
+// the gradient, so every wait ends.  All waits are bounded.
+__device__ void grad_producer(const OverlapArgs& a, GradCtl* gc, uint8_t* gbuf, volatile int* abort_flag) {
+  const uint64_t pol = l2_policy_evict_first();
+  long long k = 0;  // stages issued
+  bool ok = true;
+  for (long long row = a.grad_begin + blockIdx.x; ok && row < a.grad_end; row += gridDim.x) {
+    const unsigned* cnt = a.branch_cnt + row / a.W;
+    const long long t0 = clock64();
+    while (ld_acquire(cnt) != (unsigned)(a.W + 1)) {
+      if (*abort_flag) {
+        ok = false;
+        break;
+      }
+      if (clock64() - t0 > kWaitLimitCycles) {
+        *abort_flag = 1;
+        atomicOr(reinterpret_cast<unsigned*>(a.status), SPECOPD_FLAG_TIMEOUT);
+        ok = false;
+        break;
+      }
+      __nanosleep(200);
+    }
+    if (!ok) break;
+    const float lz2 = __ldcg(a.lz2 + row), ql = __ldcg(a.ql + row), g = __ldcg(a.g + row);
+    // the bits were stored through the generic proxy; the copies read them
+    // through the async proxy
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    const __nv_bfloat16* zrow = static_cast<const __nv_bfloat16*>(a.draft) + row * a.ld_draft;
+    const uint8_t* mrow = a.mbits + row * a.mbits_ld;
+    for (long long e0 = 0; e0 < a.V; e0 += kGUnit, ++k) {
+      const int st = (int)(k % kGStages);
+      if (k >= kGStages && !mbar_wait(&gc->empty[st], (uint32_t)((k / kGStages) - 1) & 1u, abort_flag)) {
+        ok = false;
+        break;
+      }
+      gc->info[st][0] = lz2;
+      gc->info[st][1] = ql;
+      gc->info[st][2] = g;
+      const int n = (int)min((long long)kGUnit, a.V - e0);
+      const int nbk = n & ~127;  // bulk part: whole 128-logit steps
+      uint8_t* dz = gbuf + st * kGStageBytes;
+      if (nbk > 0) {
+        mbar_arrive_expect_tx(&gc->full[st], (uint32_t)(nbk * 2 + nbk / 8));
+        bulk_g2s_policy(dz, zrow + e0, (uint32_t)nbk * 2u, &gc->full[st], pol);
+        bulk_g2s_policy(dz + kGUnit * 2, mrow + e0 / 8, (uint32_t)nbk / 8u, &gc->full[st], pol);
+      } else {
+        mbar_arrive(&gc->full[st]);
+      }
+    }
+  }
+  // every issued copy must land before the CTA may exit
+  for (long long j = (k > kGStages ? k - kGStages : 0); j < k; ++j)
+    ring_drain_wait(&gc->full[j % kGStages], (uint32_t)(j / kGStages) & 1u);
+}
 
-__global__ void __launch_bounds__(kGradThreads) tv_grad_bf16_kernel(const OverlapArgs a, int bx) {
-  const long long row = blockIdx.x / bx;
-  const int bxi = blockIdx.x - (int)(row * bx);
-  const int lane = threadIdx.x & 31;
-  const long long wbase = ((long long)bxi * (kGradThreads / 32) + (threadIdx.x >> 5)) * kGradElemsPerWarp;
-  if (wbase >= a.V) return;
-  const float L2 = a.lz2[row];
-  const float Q = a.ql[row];
-  const float G = a.g[row];
-  const __nv_bfloat16* zrow = static_cast<const __nv_bfloat16*>(a.draft) + row * a.ld_draft;
-  const uint8_t* mrow = a.mbits + row * a.mbits_ld;
-  float* grow = a.grad + row * a.ld_grad;
-  const bool live = L2 != -INFINITY;
-  const float2 l2e = make_float2(kLog2e, kLog2e), nl = make_float2(live ? -L2 : 0.f, live ? -L2 : 0.f);
-  if (wbase + kGradElemsPerWarp <= a.V) {
-    uint2 zw[kGradSteps];
-    uint32_t nib[kGradSteps];
-#pragma unroll
-    for (int v = 0; v < kGradSteps; ++v) {
-      const long long e = wbase + v * 128 + 4 * lane;
-      zw[v] = __ldcs(reinterpret_cast<const uint2*>(zrow + e));
-      nib[v] = mrow[e >> 3];
-    }
-#pragma unroll
-    for (int v = 0; v < kGradSteps; ++v) {
-      const long long e = wbase + v * 128 + 4 * lane;
-      const uint32_t bits = nib[v] >> ((lane & 1) * 4);
-      const uint32_t z0 = bmax2(zw[v].x, kNegInf2), z1 = bmax2(zw[v].y, kNegInf2);  // inactive -> q = 0
-      const float2 x0 = __ffma2_rn(make_float2(bf_lo(z0), bf_hi(z0)), l2e, nl);
-      const float2 x1 = __ffma2_rn(make_float2(bf_lo(z1), bf_hi(z1)), l2e, nl);
+__device__ void grad_consumer(const OverlapArgs& a, GradCtl* gc, const uint8_t* gbuf, volatile int* abort_flag, int gw,
+                              int lane) {
+  const float2 l2e = make_float2(kLog2e, kLog2e);
+  const uint64_t spol = l2_policy_evict_first();
+  long long k = 0;
+  for (long long row = a.grad_begin + blockIdx.x; row < a.grad_end; row += gridDim.x) {
+    const __nv_bfloat16* zrow = static_cast<const __nv_bfloat16*>(a.draft) + row * a.ld_draft;
+    const uint8_t* mrow = a.mbits + row * a.mbits_ld;
+    float* grow = a.grad + row * a.ld_grad;
+    for (long long e0 = 0; e0 < a.V; e0 += kGUnit, ++k) {
+      const int st = (int)(k % kGStages);
+      if (!mbar_wait_warp(&gc->full[st], (uint32_t)(k / kGStages) & 1u, abort_flag)) return;
+      const float L2 = gc->info[st][0], Q = gc->info[st][1], G = gc->info[st][2];
+      const bool live = L2 != -INFINITY;
       const float gg = live ? G : 0.f;
-      float4 o;
-      o.x = gg * ex2(x0.x) * ((float)(bits & 1u) - Q);
-      o.y = gg * ex2(x0.y) * ((float)((bits >> 1) & 1u) - Q);
-      o.z = gg * ex2(x1.x) * ((float)((bits >> 2) & 1u) - Q);
-      o.w = gg * ex2(x1.y) * ((float)((bits >> 3) & 1u) - Q);
-      __stcs(reinterpret_cast<float4*>(grow + e), o);
-    }
-  } else {
-    for (long long e = wbase + lane; e < min((long long)a.V, wbase + kGradElemsPerWarp); e += 32) {
-      const float z = __bfloat162float(zrow[e]);
-      const bool active = live && z == z && fabsf(z) != INFINITY;
-      const float q = active ? ex2(fmaf(z, kLog2e, -L2)) : 0.f;
-      const uint32_t bit = (mrow[e >> 3] >> (e & 7)) & 1u;
-      grow[e] = G * q * ((float)bit - Q);
+      const float2 nl = make_float2(live ? -L2 : 0.f, live ? -L2 : 0.f);
+      const float omq = 1.f - Q, zmq = 0.f - Q;  // [q < p] - q_less for bit 1 and bit 0
+      const int n = (int)min((long long)kGUnit, a.V - e0);
+      const int nbk = n & ~127;
+      const uint8_t* sz = gbuf + st * kGStageBytes;
+      const uint8_t* sb = sz + kGUnit * 2;
+      for (int v = gw; v * 128 < nbk; v += kRGradWarps) {
+        const int e = v * 128 + 4 * lane;
+        const uint2 zw = *reinterpret_cast<const uint2*>(sz + 2 * e);
+        const uint32_t bits = (uint32_t)sb[e >> 3] >> ((lane & 1) * 4);
+        const uint32_t z0 = bmax2(zw.x, kNegInf2), z1 = bmax2(zw.y, kNegInf2);  // inactive -> q = 0
+        const float2 x0 = __ffma2_rn(make_float2(bf_lo(z0), bf_hi(z0)), l2e, nl);
+        const float2 x1 = __ffma2_rn(make_float2(bf_lo(z1), bf_hi(z1)), l2e, nl);
+        float4 o;
+        o.x = gg * ex2(x0.x) * ((bits & 1u) ? omq : zmq);
+        o.y = gg * ex2(x0.y) * ((bits & 2u) ? omq : zmq);
+        o.z = gg * ex2(x1.x) * ((bits & 4u) ? omq : zmq);
+        o.w = gg * ex2(x1.y) * ((bits & 8u) ? omq : zmq);
+        st_global_v4_policy(grow + e0 + e, o, spol);
+      }
+      if (gw == 0) {  // fewer than 128 logits at the end of the row: plain loads
+        for (long long e = e0 + nbk + lane; e < e0 + n; e += 32) {
+          const float z = __bfloat162float(zrow[e]);
+          const bool active = live && z == z && fabsf(z) != INFINITY;
+          const float q = active ? ex2(fmaf(z, kLog2e, -L2)) : 0.f;
+          const uint32_t bit = (__ldcg(mrow + (e >> 3)) >> (e & 7)) & 1u;
+          grow[e] = G * q * ((float)bit - Q);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&gc->empty[st]);
     }
   }
 }
 
 }  // namespace
 
-// Persistent ring statistics kernel: one CTA per SM (192 KB of ring),
-// at most one CTA per row.
+// Persistent ring kernel: one CTA per SM; statistics of rows [row_begin,
+// row_end), at most one CTA per row, and, when rows [grad_begin, grad_end)
+// are given, their gradient on every SM's gradient warps (a cooperative
+// launch: the gradient warps wait for branches finished by other CTAs).
 cudaError_t launch_tv_stats_bf16(const OverlapArgs& a, cudaStream_t stream) {
-  if (a.rows == 0) return cudaSuccess;
+  const long long nrows = a.row_end - a.row_begin;
+  const long long ngrad = a.grad_end - a.grad_begin;
+  if (nrows <= 0 && ngrad <= 0) return cudaSuccess;
   if (a.V > 0x7fffffffLL - kRChunk) return cudaErrorInvalidValue;
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  const size_t smem = (size_t)kRSlots * kRSlotBytes + sizeof(RingCtl) + sizeof(RingRed);
+  // setmaxnreg.inc waits until the warpgroups that gave registers back have
+  // done so: the split must fit in what the launch allocates
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, tv_stats_bf16_ring_kernel);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kRRegLaunch) return cudaErrorInvalidConfiguration;
+  const size_t smem = kRSmem;
   e = cudaFuncSetAttribute(tv_stats_bf16_ring_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const long long grid = a.rows < sms ? a.rows : sms;
-  tv_stats_bf16_ring_kernel<<<(unsigned)grid, kRThreads, smem, stream>>>(a);
-  return cudaGetLastError();
+  const long long grid = (ngrad > 0 || nrows > sms) ? sms : nrows;
+  if (ngrad <= 0) {
+    tv_stats_bf16_ring_kernel<<<(unsigned)grid, kRThreads, smem, stream>>>(a);
+    return cudaGetLastError();
+  }
+  // the gradient warps wait for branches finished by other CTAs: all CTAs
+  // must be resident at once
+  OverlapArgs arg = a;
+  void* params[] = {&arg};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(tv_stats_bf16_ring_kernel), dim3((unsigned)grid),
+                                     dim3(kRThreads), params, smem, stream);
 }
 
-cudaError_t launch_tv_grad_bf16(const OverlapArgs& a, cudaStream_t stream) {
-  if (a.rows == 0) return cudaSuccess;
-  const long long per_block = (long long)kGradElemsPerWarp * (kGradThreads / 32);
-  const long long bx = (a.V + per_block - 1) / per_block;
-  tv_grad_bf16_kernel<<<(unsigned)(bx * a.rows), kGradThreads, 0, stream>>>(a, (int)bx);
-  return cudaGetLastError();
+// Fused statistics + gradient in one cooperative launch: the consumer warps
+// run the statistics row by row while the gradient warps of every SM stream
+// the gradient of the rows whose branch is finished.
+cudaError_t launch_tv_fused_bf16(OverlapArgs a, cudaStream_t stream) {
+  if (a.rows <= 0) return cudaSuccess;
+  a.row_begin = 0;
+  a.row_end = a.rows;
+  a.grad_begin = 0;
+  a.grad_end = a.rows;
+  return launch_tv_stats_bf16(a, stream);
 }
 
 }  // namespace specopd

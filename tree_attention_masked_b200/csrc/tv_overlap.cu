@@ -433,9 +433,10 @@ cudaError_t launch_tv_stats(const OverlapArgs& a, specopd_dtype dtype, cudaStrea
   return dtype == SPECOPD_BF16 ? launch_tv_stats_bf16(a, stream) : launch_stats_t<float>(a, stream);
 }
 
+// fp32 gradient (the bf16 gradient runs inside launch_tv_fused_bf16)
 cudaError_t launch_tv_grad(const OverlapArgs& a, specopd_dtype dtype, cudaStream_t stream) {
   if (a.rows == 0) return cudaSuccess;
-  return dtype == SPECOPD_BF16 ? launch_tv_grad_bf16(a, stream) : launch_grad_t<float>(a, stream);
+  return dtype == SPECOPD_BF16 ? cudaErrorInvalidValue : launch_grad_t<float>(a, stream);
 }
 
 cudaError_t launch_e2e_loss(const float* alpha, int64_t num_branches, int W, double inv_count, float* loss,
