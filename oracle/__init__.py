@@ -19,8 +19,10 @@ Modules:
                 softmax attention, plus the independent per-branch causal form
   overlap    -- full-vocabulary overlap alpha, E2E-TV loss, and the gradient
                 with respect to draft logits
+  lm_head    -- prediction logits from hidden states and a head, and the
+                overlap statistics taken from them
 
 Every function is plain fp64 NumPy written from the definitions; nothing is
 blocked, fused or reordered.
 """
-from . import tree, attention, overlap  # noqa: F401
+from . import tree, attention, overlap, lm_head  # noqa: F401

@@ -150,3 +150,25 @@ def test_sibling_leak_breaks_causal_equivalence():
     finally:
         T.visible = orig
     assert np.max(np.abs(bad - ind)) > 1e-3
+
+
+def test_lm_head_slips_break_pins():
+    """A head used untransposed, or q_less counted with <= instead of <,
+    breaks the one-hot readout and the identical-model pins."""
+    import pytest
+    from oracle import lm_head as LM
+    rng = np.random.default_rng(11)
+    H, V = 6, 11
+    head = rng.normal(size=(V, H))
+    with pytest.raises(ValueError):  # h @ head cannot even be formed for H != V
+        np.eye(H) @ head
+    sq = rng.normal(size=(H, H))     # a square head: the untransposed product runs but is wrong
+    assert not np.array_equal(np.eye(H) @ sq, sq.T)
+    assert np.array_equal(LM.prediction_logits(np.eye(H), sq), sq.T)
+    h = rng.normal(size=(4, H))
+    z = h @ head.T
+    q, active, log_q = O.draft_probs(z)
+    _, log_p = O.teacher_probs(z)
+    bad_q_less = (q * ((log_q <= log_p) & active)).sum(axis=-1)
+    good = LM.row_statistics(z, z)["q_less"]
+    assert np.all(good == 0.0) and np.all(np.abs(bad_q_less - 1.0) < 1e-12)
