@@ -244,6 +244,41 @@ int specopd_tv_overlap_e2e(const void* draft, const void* teacher, specopd_dtype
                            double count, float* alpha, float* loss, float* grad_draft, int64_t ld_grad,
                            void* workspace, size_t workspace_bytes, int32_t* status, specopd_stream_t stream);
 
+/* Bytes of workspace specopd_lm_head_overlap needs (0 for invalid sizes). */
+size_t specopd_lm_head_workspace_bytes(int64_t rows, int64_t V);
+
+/*
+ * specopd_lm_head_overlap -- overlap, E2E-TV loss and dL/dalpha straight from
+ * hidden states and LM heads, without materialising the [rows, V] logits.
+ *
+ * The write-up's section "Inputs and code mapping": prediction_logits reads
+ * supplied hidden states and a supplied head, and e2e_tv_loss consumes the
+ * same-history aligned logits of draft and teacher.  Reading (the pages name
+ * nothing more): logits = h head^T, no bias, temperature 1, every vocabulary
+ * entry active.  alpha, L and dL/dalpha are those of specopd_tv_overlap_e2e
+ * (section "Equations").  The logits of a row are formed twice, tile by tile
+ * in TMEM (bf16 products, fp32 accumulation): once for the normalisers, once
+ * for alpha and q_less.
+ *
+ * h_draft [rows, Hd], head_draft [V, Hd], h_teacher [rows, Ht],
+ * head_teacher [V, Ht]: device bf16, row-major and contiguous, 16-byte
+ * aligned; Hd and Ht are multiples of 64.  Rows are predictions b-major (row
+ * b*W + i-1 holds y_{b,i}); rows must equal num_branches * W; count <= 0
+ * means rows.  Outputs (device fp32): alpha [rows] (nullable: then kept in the
+ * workspace), q_less [rows], lse_draft / lse_teacher [rows] (natural log),
+ * loss (scalar) and grad_alpha [rows], all but loss nullable.  workspace:
+ * device, >= specopd_lm_head_workspace_bytes(rows, V), 256-byte aligned;
+ * the caller owns every buffer.  A non-finite logit sets
+ * SPECOPD_FLAG_NONFINITE in *status; a timed-out in-kernel wait sets
+ * SPECOPD_FLAG_TIMEOUT.  Returns SPECOPD_ERR_SHAPE / _ARG / _ALIGN /
+ * _WORKSPACE before anything is enqueued, SPECOPD_ERR_CUDA if a launch fails.
+ */
+int specopd_lm_head_overlap(const void* h_draft, const void* head_draft, int Hd, const void* h_teacher,
+                            const void* head_teacher, int Ht, int64_t rows, int64_t V, int64_t num_branches, int W,
+                            double count, float* alpha, float* q_less, float* lse_draft, float* lse_teacher,
+                            float* loss, float* grad_alpha, void* workspace, size_t workspace_bytes,
+                            int32_t* status, specopd_stream_t stream);
+
 /*
  * specopd_tv_overlap_e2e_static -- specopd_tv_overlap_e2e without a workspace.
  *

@@ -258,3 +258,71 @@ def make_workload(i: int, seed: int = 0, workers: int = 0, with_logits: bool = T
                          vocab=248320, sig_t=4.0, sig_n=2.0, seed=seed, workers=workers,
                          with_logits=with_logits)
     raise ValueError(f"unknown workload {i}")
+
+
+# ---------------------------------------------------------------------------
+# Hidden states and LM heads (prediction logits formed from them, never stored)
+# ---------------------------------------------------------------------------
+
+_TID_H_TEACHER, _TID_W_TEACHER, _TID_H_DRAFT, _TID_W_DRAFT = range(100, 104)
+
+
+@dataclasses.dataclass
+class LmHeadCase:
+    name: str
+    num_branches: int
+    W: int
+    V: int
+    Hd: int
+    Ht: int
+    h_draft: np.ndarray   # [rows, Hd] bf16 bits (uint16)
+    w_draft: np.ndarray   # [V, Hd]
+    h_teacher: np.ndarray  # [rows, Ht]
+    w_teacher: np.ndarray  # [V, Ht]
+
+    @property
+    def rows(self) -> int:
+        return self.num_branches * self.W
+
+
+def _head_chunk(args) -> Tuple[int, np.ndarray, np.ndarray]:
+    """Rows [256 c, 256 c + 256) of both heads (the substreams of _normal_rows)."""
+    seed, c, rows, Hd, Ht, sig_t, sig_n = args
+    rt = np.random.default_rng([seed, _TID_W_TEACHER, 0, c])
+    wt = rt.standard_normal((rows, Ht), dtype=np.float32) * np.float32(sig_t / np.sqrt(Ht))
+    wt_b = bf16_round(wt)
+    rd = np.random.default_rng([seed, _TID_W_DRAFT, 0, c])
+    if Hd == Ht:
+        noise = rd.standard_normal((rows, Hd), dtype=np.float32) * np.float32(sig_n / np.sqrt(Hd))
+        wd_b = bf16_round(bf16_to_f32(wt_b) + noise)
+    else:
+        wd_b = bf16_round(rd.standard_normal((rows, Hd), dtype=np.float32) * np.float32(sig_t / np.sqrt(Hd)))
+    return c, wd_b, wt_b
+
+
+def make_lm_head_case(name: str, num_branches: int, W: int, V: int, Hd: int, Ht: int, sig_t: float,
+                      sig_n: float, seed: int = 0, workers: int = 0) -> LmHeadCase:
+    """Teacher hidden states h_t ~ N(0, 1) and head w_t ~ N(0, sig_t^2 / Ht), so
+    that teacher logits have standard deviation about sig_t.  With Hd == Ht the
+    draft reads the same hidden states through w_d = w_t + N(0, sig_n^2 / Hd)
+    (its logits are the teacher's plus noise of deviation about sig_n);
+    otherwise it has its own h_d ~ N(0, 1) and w_d ~ N(0, sig_t^2 / Hd).
+    Everything is drawn in fp32 and rounded to bf16 once; the heads are drawn
+    in 256-row chunks, each from its own substream, so `workers` processes
+    give the same bytes as one."""
+    rows = num_branches * W
+    ht = _normal_rows(seed, _TID_H_TEACHER, 0, rows, Ht, 1.0)
+    jobs = [(seed, c, min(_ROW_CHUNK, V - c * _ROW_CHUNK), Hd, Ht, sig_t, sig_n)
+            for c in range((V + _ROW_CHUNK - 1) // _ROW_CHUNK)]
+    if workers and len(jobs) > 1:
+        with mp.get_context("spawn").Pool(workers) as pool:
+            results = pool.map(_head_chunk, jobs, chunksize=4)
+    else:
+        results = [_head_chunk(j) for j in jobs]
+    wd_b = np.empty((V, Hd), dtype=np.uint16)
+    wt_b = np.empty((V, Ht), dtype=np.uint16)
+    for c, d, t in results:
+        wd_b[c * _ROW_CHUNK:c * _ROW_CHUNK + d.shape[0]] = d
+        wt_b[c * _ROW_CHUNK:c * _ROW_CHUNK + t.shape[0]] = t
+    hd_b = bf16_round(ht) if Hd == Ht else bf16_round(_normal_rows(seed, _TID_H_DRAFT, 0, rows, Hd, 1.0))
+    return LmHeadCase(name, num_branches, W, V, Hd, Ht, hd_b, wd_b, bf16_round(ht), wt_b)

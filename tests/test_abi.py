@@ -103,10 +103,24 @@ def test_argument_errors_before_launch(S):
                                          16, None) == -2
     assert lib["specopd_rope"](16, 16, 16, 16, 1, 4, 2, 2, 6, 16, 1e4, None) == -2
     assert lib["specopd_e2e_tv_loss"](16, 2, 0, 0.0, 16, None, None) == -2
+    # LM head: hidden sizes must be multiples of 64, rows = num_branches * W,
+    # 16-byte aligned operands, a large enough workspace
+    lm = lib["specopd_lm_head_overlap"]
+    need = S.specopd_lm_head_workspace_bytes(8, 1000)
+    assert lm(16, 16, 96, 16, 16, 128, 8, 1000, 2, 4, 0.0, 16, None, None, None, 16, None, 256, need, 16, None) == -2
+    assert lm(16, 16, 128, 16, 16, 128, 8, 1000, 3, 4, 0.0, 16, None, None, None, 16, None, 256, need, 16, None) == -2
+    assert lm(24, 16, 128, 16, 16, 128, 8, 1000, 2, 4, 0.0, 16, None, None, None, 16, None, 256, need, 16, None) == -6
+    assert lm(16, 16, 128, 16, 16, 128, 8, 1000, 2, 4, 0.0, 16, None, None, None, 16, None, 256, need - 1, 16,
+              None) == -5
+    assert lm(16, 16, 128, 16, 16, 128, 8, 1000, 2, 4, 0.0, 16, None, None, None, None, None, 256, need, 16,
+              None) == -1
     assert S._c["specopd_status_string"](-5) == b"workspace missing, too small or misaligned"
 
 
 def test_workspace_sizes(S):
+    n_tiles = (151936 + 255) // 256
+    assert S.specopd_lm_head_workspace_bytes(1024, 151936) >= n_tiles * 1024 * 24 + 3 * 1024 * 4
+    assert S.specopd_lm_head_workspace_bytes(-1, 10) == 0
     assert S.specopd_attention_workspace_bytes(S.BF16, 100, 4, 2, 128) == (
         (100 * 4 * 128 * 2 + 255) // 256 * 256 + (100 * 2 * 128 * 2 + 255) // 256 * 256)
     ws = S.specopd_overlap_workspace_bytes(1024, 151936, 64)

@@ -1,0 +1,112 @@
+"""Overlap statistics from hidden states and LM heads on the GPU against the
+oracle: alpha, q_less and L within 1e-4 absolute, the normalisers within 1e-4
+absolute, dL/dalpha within 1e-4 absolute.  The GPU forms the logits with bf16
+products and fp32 accumulation; the oracle in fp64 from the same bf16 values."""
+import numpy as np
+import pytest
+import torch
+
+import synthetic as SY
+from oracle import lm_head as LM
+from tree_attention_masked_b200 import specopd as S
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-4
+
+
+def run(case, count=0.0, with_optional=True):
+    dev = torch.device("cuda")
+    t = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    hd, wd, ht, wt = t(case.h_draft), t(case.w_draft), t(case.h_teacher), t(case.w_teacher)
+    R = case.rows
+    f = lambda: torch.full((R,), float("nan"), device=dev)
+    out = {"alpha": f(), "loss": torch.full((1,), float("nan"), device=dev)}
+    if with_optional:
+        out.update(q_less=f(), lse_draft=f(), lse_teacher=f(), grad_alpha=f())
+    ws = torch.empty(S.specopd_lm_head_workspace_bytes(R, case.V), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    S.specopd_lm_head_overlap(hd, wd, ht, wt, case.num_branches, case.W, count, out["alpha"], out["loss"], ws,
+                              status, q_less=out.get("q_less"), lse_draft=out.get("lse_draft"),
+                              lse_teacher=out.get("lse_teacher"), grad_alpha=out.get("grad_alpha"))
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    return {k: v.cpu().numpy().astype(np.float64) for k, v in out.items()}
+
+
+def oracle(case, rows=None, count=None):
+    f64 = lambda a: SY.to_f64(a, "bf16")
+    hd, ht = f64(case.h_draft), f64(case.h_teacher)
+    if rows is not None:
+        hd, ht = hd[rows], ht[rows]
+    W = case.W if rows is None else len(rows)
+    return LM.lm_head_overlap(hd, f64(case.w_draft), ht, f64(case.w_teacher), W, count)
+
+
+CASES = [
+    # name, branches, W, V, Hd, Ht
+    ("tiny", 2, 4, 1000, 128, 128),        # one row tile, a ragged vocabulary tile
+    ("ragged-rows", 5, 7, 777, 64, 64),    # 35 rows: a partial row tile; the smallest hidden size
+    ("exact-tiles", 32, 8, 512, 128, 128),  # 256 rows and 512 entries: whole tiles only
+    ("two-heads", 3, 16, 3000, 64, 192),   # different draft and teacher hidden sizes
+    ("multi-tile", 24, 16, 8191, 256, 256),  # 3 row tiles x 32 vocabulary tiles, more tiles than some SMs take
+    ("one-entry", 1, 1, 1, 64, 64),        # V = 1: q = p = 1, alpha = 1
+]
+
+
+@pytest.mark.parametrize("name,nb,W,V,Hd,Ht", CASES)
+def test_lm_head_overlap_matches_oracle(name, nb, W, V, Hd, Ht):
+    case = SY.make_lm_head_case(name, nb, W, V, Hd, Ht, sig_t=3.0, sig_n=1.5, seed=len(name))
+    got = run(case)
+    ref = oracle(case)
+    keys = ["alpha", "q_less", "lse_draft", "lse_teacher", "grad_alpha"]
+    if V == 1:
+        # q = p = 1 exactly: a tie that fp32 rounding may settle either way.
+        # Both q_less = 0 and 1 are valid subgradients of min there, and the
+        # gradient q (bit - q_less) is 0 for both, so only the set is checked.
+        keys.remove("q_less")
+        assert set(got["q_less"].tolist()) <= {0.0, 1.0}
+    for k in keys:
+        assert np.max(np.abs(got[k] - ref[k])) <= TOL, (k, np.max(np.abs(got[k] - ref[k])))
+    assert abs(got["loss"][0] - ref["loss"]) <= TOL
+
+
+def test_identical_models_give_full_overlap():
+    case = SY.make_lm_head_case("same", 4, 8, 5000, 128, 128, sig_t=3.0, sig_n=0.0, seed=3)
+    assert np.array_equal(case.w_draft, case.w_teacher) and np.array_equal(case.h_draft, case.h_teacher)
+    got = run(case)
+    assert np.max(np.abs(got["alpha"] - 1.0)) <= 1e-5
+    assert np.all(got["q_less"] == 0.0)   # identical logits: q < p nowhere
+    assert abs(got["loss"][0]) <= 1e-5
+
+
+def test_optional_outputs_and_count():
+    case = SY.make_lm_head_case("opt", 3, 4, 2048, 64, 64, sig_t=2.0, sig_n=1.0, seed=9)
+    a = run(case, with_optional=False)
+    b = run(case, count=100.0)
+    assert np.array_equal(a["alpha"], b["alpha"])   # the same launches: identical bits
+    ref = oracle(case, count=100)
+    assert abs(b["loss"][0] - ref["loss"]) <= TOL
+
+
+def test_repeatable_bits():
+    case = SY.make_lm_head_case("rep", 8, 16, 4096, 128, 128, sig_t=3.0, sig_n=1.5, seed=5)
+    a, b = run(case), run(case)
+    for k in a:
+        assert np.array_equal(a[k], b[k]), k
+
+
+def test_full_size_sampled_branches():
+    """The 8B-style shape: 1,024 prediction rows, hidden size 4,096, V = 151,936
+    (594 vocabulary tiles, 8 row tiles); the oracle on three whole branches."""
+    case = SY.make_lm_head_case("full", 64, 16, 151936, 4096, 4096, sig_t=3.0, sig_n=1.5, seed=0, workers=8)
+    got = run(case)
+    assert 0.0 <= got["loss"][0] <= 1.0
+    for b in (0, 37, 63):
+        rows = np.arange(b * 16, (b + 1) * 16)
+        ref = oracle(case, rows=rows)
+        for k in ("alpha", "q_less", "lse_draft", "lse_teacher"):
+            assert np.max(np.abs(got[k][rows] - ref[k])) <= TOL, (b, k)
+    # the loss from the GPU's own alpha, by the definition
+    from oracle import overlap as OO
+    assert abs(got["loss"][0] - OO.e2e_tv_loss(got["alpha"], 16)) <= 1e-6

@@ -294,6 +294,54 @@ int specopd_tv_overlap_e2e(const void* draft, const void* teacher, specopd_dtype
   return SPECOPD_OK;
 }
 
+size_t specopd_lm_head_workspace_bytes(int64_t rows, int64_t V) {
+  if (rows < 0 || V < 1) return 0;
+  return lm_head_layout(rows, V).total;
+}
+
+int specopd_lm_head_overlap(const void* h_draft, const void* head_draft, int Hd, const void* h_teacher,
+                            const void* head_teacher, int Ht, int64_t rows, int64_t V, int64_t num_branches, int W,
+                            double count, float* alpha, float* q_less, float* lse_draft, float* lse_teacher,
+                            float* loss, float* grad_alpha, void* workspace, size_t workspace_bytes,
+                            int32_t* status, specopd_stream_t stream) {
+  if (W < 1 || W > SPECOPD_MAX_W || num_branches < 0 || rows != num_branches * W) return SPECOPD_ERR_SHAPE;
+  if (V < 1 || V > (1LL << 31) - 256 || Hd < 64 || Ht < 64 || Hd % 64 || Ht % 64 || Hd > (1 << 20) ||
+      Ht > (1 << 20) || rows > (1LL << 31) - 128)
+    return SPECOPD_ERR_SHAPE;
+  if (!loss || !status) return SPECOPD_ERR_ARG;
+  if (!(count <= 0.0) && !std::isfinite(count)) return SPECOPD_ERR_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (rows == 0) return cuda_status(cudaMemsetAsync(loss, 0, sizeof(float), st));
+  if (!h_draft || !head_draft || !h_teacher || !head_teacher) return SPECOPD_ERR_ARG;
+  if (!aligned16(h_draft) || !aligned16(head_draft) || !aligned16(h_teacher) || !aligned16(head_teacher))
+    return SPECOPD_ERR_ALIGN;
+  const LmHeadLayout L = lm_head_layout(rows, V);
+  if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) % kAlign))
+    return SPECOPD_ERR_WORKSPACE;
+  const double n = count > 0.0 ? count : (double)rows;
+  LmHeadArgs a;
+  a.h_draft = h_draft;
+  a.w_draft = head_draft;
+  a.h_teacher = h_teacher;
+  a.w_teacher = head_teacher;
+  a.rows = rows;
+  a.V = V;
+  a.Hd = Hd;
+  a.Ht = Ht;
+  a.num_branches = num_branches;
+  a.W = W;
+  a.inv_count = 1.0 / n;
+  a.alpha = alpha;
+  a.q_less = q_less;
+  a.lse_draft = lse_draft;
+  a.lse_teacher = lse_teacher;
+  a.loss = loss;
+  a.grad_alpha = grad_alpha;
+  a.workspace = workspace;
+  a.status = status;
+  return cuda_status(launch_lm_head_overlap(a, st));
+}
+
 const char* specopd_status_string(int status) {
   switch (status) {
     case SPECOPD_OK: return "ok";

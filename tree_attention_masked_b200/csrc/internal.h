@@ -91,4 +91,31 @@ cudaError_t launch_tv_grad(const OverlapArgs& a, specopd_dtype dtype, cudaStream
 cudaError_t launch_e2e_loss(const float* alpha, int64_t num_branches, int W, double inv_count, float* loss,
                             float* grad_alpha, cudaStream_t stream);
 
+// Overlap statistics from hidden states and LM heads (lm_head_sm100.cu).
+struct LmHeadArgs {
+  const void* h_draft;    // [rows, Hd] bf16
+  const void* w_draft;    // [V, Hd] bf16
+  const void* h_teacher;  // [rows, Ht] bf16
+  const void* w_teacher;  // [V, Ht] bf16
+  int64_t rows, V;
+  int Hd, Ht;
+  int64_t num_branches;
+  int W;
+  double inv_count;
+  float* alpha;         // nullable: workspace then
+  float* q_less;        // nullable
+  float* lse_draft;     // nullable (natural log)
+  float* lse_teacher;   // nullable
+  float* loss;
+  float* grad_alpha;    // nullable
+  void* workspace;
+  int32_t* status;
+};
+struct LmHeadLayout {
+  int64_t n_tiles;
+  size_t part_a, part_b, lz2, lt2, alpha, total;
+};
+LmHeadLayout lm_head_layout(int64_t rows, int64_t V);
+cudaError_t launch_lm_head_overlap(const LmHeadArgs& a, cudaStream_t stream);
+
 }  // namespace specopd

@@ -1,0 +1,394 @@
+// Prediction logits from hidden states and a head, consumed tile by tile by
+// the overlap statistics: the [rows, V] logits never reach HBM.
+//
+// daiwk.github.io write-up of SpecOPD, section "Inputs and code mapping":
+// prediction_logits reads supplied hidden states and a supplied head (here
+// logits = h W^T: no bias, temperature 1), and e2e_tv_loss consumes the
+// same-history aligned logits of draft and teacher.  Section "Equations":
+// alpha = sum_v min(q, p), L from prefix products of alpha.
+//
+// alpha needs the normalisers of both softmaxes first, so the logits are
+// computed twice:
+//   pass A -- every (128-row, 256-entry) tile of draft and teacher logits
+//             into TMEM; the epilogue reduces each row's part of the tile to
+//             a base-2 (max, sum) pair per softmax;
+//   reduce  -- per row, the tile pairs merged in tile order: lz2, lt2;
+//   pass B -- the same tiles again; the epilogue forms the row's share of
+//             alpha = sum exp2(min(z2 - lz2, t2 - lt2)) and q_less;
+//   reduce  -- per row, the shares summed in tile order: alpha, q_less;
+// then the E2E-TV loss and dL/dalpha from alpha.
+//
+// Tile kernel: a persistent grid, one CTA per SM, tiles dealt round-robin in
+// vocabulary-major order (the row tiles of one head tile run together, so the
+// head tile comes from HBM once and from L2 for the others).  Warp 0 issues
+// TMA loads (2-D maps, 128-byte swizzle, no multicast) of [128 x 64] hidden
+// and [256 x 64] head boxes into a 4-stage ring; one thread of warp 1 issues
+// tcgen05.mma (kind::f16, M = 128, N = 256, K = 16) into TMEM columns
+// [0, 256) for the draft and [256, 512) for the teacher; warps 4-7 (one
+// TMEM lane quarter each, one row per thread) read the accumulators with
+// tcgen05.ld.  Each accumulator half has its own full / empty barriers, so
+// the epilogue of one half runs under the MMAs of the other.  All waits are
+// bounded; a timeout raises SPECOPD_FLAG_TIMEOUT and every role winds down.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "overlap_common.cuh"
+#include "ptx.cuh"
+#include "tmap.cuh"
+
+namespace specopd {
+namespace {
+
+constexpr int kLBM = 128;   // rows per tile
+constexpr int kLBN = 256;   // vocabulary entries per tile
+constexpr int kLBK = 64;    // hidden elements per stage (one 128-byte swizzle row)
+constexpr int kLStages = 4;
+constexpr int kLThreads = 256;
+constexpr uint32_t kLABytes = kLBM * kLBK * 2;  // 16 KB
+constexpr uint32_t kLBBytes = kLBN * kLBK * 2;  // 32 KB
+constexpr float kLLog2e = 1.4426950408889634f;
+
+struct alignas(1024) LmSmem {
+  uint8_t a[kLStages][kLABytes];
+  uint8_t b[kLStages][kLBBytes];
+  uint64_t full[kLStages];
+  uint64_t empty[kLStages];
+  uint64_t acc_full[2];   // MMAs of the draft / teacher half done
+  uint64_t acc_empty[2];  // the epilogue has read the half
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct LmParams {
+  int64_t rows, V;
+  int Hd, Ht;
+  int m_tiles, n_tiles;
+  float4* part_a;        // [n_tiles][rows]: (mz, sz, mt, st), base 2
+  float2* part_b;        // [n_tiles][rows]: (alpha share, q_less share)
+  const float* lz2;      // [rows] draft normaliser, base 2 (pass B)
+  const float* lt2;      // [rows] teacher normaliser, base 2 (pass B)
+  int32_t* status;
+};
+
+__device__ __forceinline__ void lm_drain_wait(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitLimitCycles) return;
+  }
+}
+
+template <int PASS>
+__global__ void __launch_bounds__(kLThreads, 1)
+    lm_head_tile_kernel(const __grid_constant__ CUtensorMap tm_hd, const __grid_constant__ CUtensorMap tm_wd,
+                        const __grid_constant__ CUtensorMap tm_ht, const __grid_constant__ CUtensorMap tm_wt,
+                        const LmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  LmSmem* sm = reinterpret_cast<LmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long total = (long long)p.m_tiles * p.n_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kLStages; ++s) {
+      mbar_init(&sm->full[s], 1);
+      mbar_init(&sm->empty[s], 1);
+    }
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&sm->acc_full[h], 1);
+      mbar_init(&sm->acc_empty[h], 4);
+    }
+    mbar_init(&sm->mma_done, 1);
+    sm->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(&sm->tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 32) {
+    prefetch_tmap(&tm_hd);
+    prefetch_tmap(&tm_wd);
+    prefetch_tmap(&tm_ht);
+    prefetch_tmap(&tm_wt);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm->tmem_base;
+  volatile int* abort_flag = &sm->abort_flag;
+
+  if (warp == 0) {
+    // ================= TMA producer
+    if (lane == 0) {
+      long long it = 0;
+      bool ok = true;
+      for (long long tau = blockIdx.x; ok && tau < total; tau += gridDim.x) {
+        const int m = (int)(tau % p.m_tiles), n = (int)(tau / p.m_tiles);
+        for (int h = 0; ok && h < 2; ++h) {
+          const CUtensorMap* ta = h ? &tm_ht : &tm_hd;
+          const CUtensorMap* tb = h ? &tm_wt : &tm_wd;
+          const int nk = (h ? p.Ht : p.Hd) / kLBK;
+          for (int kb = 0; kb < nk; ++kb, ++it) {
+            const int s = (int)(it % kLStages);
+            if (it >= kLStages && !mbar_wait(&sm->empty[s], (uint32_t)((it / kLStages) - 1) & 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&sm->full[s], kLABytes + kLBBytes);
+            tma_load_2d(sm->a[s], ta, kb * kLBK, m * kLBM, &sm->full[s]);
+            tma_load_2d(sm->b[s], tb, kb * kLBK, n * kLBN, &sm->full[s]);
+          }
+        }
+      }
+      // every issued copy must land before the CTA may exit
+      for (long long j = (it > kLStages ? it - kLStages : 0); j < it; ++j)
+        lm_drain_wait(&sm->full[j % kLStages], (uint32_t)(j / kLStages) & 1u);
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer (one thread)
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kLBM, kLBN, false);
+      long long it = 0;
+      int k = 0;  // tiles of this CTA so far
+      bool ok = true;
+      for (long long tau = blockIdx.x; ok && tau < total; tau += gridDim.x, ++k) {
+        for (int h = 0; ok && h < 2; ++h) {
+          if (k > 0 && !mbar_wait(&sm->acc_empty[h], (uint32_t)(k - 1) & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nk = (h ? p.Ht : p.Hd) / kLBK;
+          for (int kb = 0; kb < nk; ++kb, ++it) {
+            const int s = (int)(it % kLStages);
+            if (!mbar_wait(&sm->full[s], (uint32_t)(it / kLStages) & 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t ab = smem_u32(sm->a[s]), bb = smem_u32(sm->b[s]);
+#pragma unroll
+            for (int ks = 0; ks < kLBK / 16; ++ks)
+              mma_ss(tmem + h * kLBN, smem_desc_sw128(ab + ks * 32, 16, 1024),
+                     smem_desc_sw128(bb + ks * 32, 16, 1024), idesc, (kb > 0 || ks > 0) ? 1u : 0u);
+            mma_commit(&sm->empty[s]);
+          }
+          if (ok) mma_commit(&sm->acc_full[h]);
+        }
+      }
+      // all MMAs must finish before TMEM and shared memory are released
+      mma_commit(&sm->mma_done);
+      lm_drain_wait(&sm->mma_done, 0);
+    }
+  } else if (warp >= 4) {
+    // ================= epilogue: one row per thread, TMEM lanes 32 (warp % 4) + lane
+    const int q4 = warp & 3;
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    const int r_in = q4 * 32 + lane;
+    int k = 0;
+    bool ok = true;
+    for (long long tau = blockIdx.x; ok && tau < total; tau += gridDim.x, ++k) {
+      const int m = (int)(tau % p.m_tiles), n = (int)(tau / p.m_tiles);
+      const long long row = (long long)m * kLBM + r_in;
+      const long long col0 = (long long)n * kLBN;
+      const int ncols = (int)min((long long)kLBN, p.V - col0);
+      if (PASS == 0) {
+        float part[4];
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait_warp(&sm->acc_full[h], (uint32_t)k & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          float mx = -INFINITY, sum = 0.f;
+          for (int c = 0; c * 32 < ncols; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tmem + lane_base + h * kLBN + c * 32, r);
+            tmem_ld_wait();
+            const int nv = min(32, ncols - c * 32);
+            float cm = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (i < nv) cm = fmaxf(cm, __uint_as_float(r[i]) * kLLog2e);
+            float cs = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (i < nv) cs += ex2(fmaf(__uint_as_float(r[i]), kLLog2e, -cm));
+            lse_merge(mx, sum, cm, cs);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm->acc_empty[h]);
+          part[2 * h] = mx;
+          part[2 * h + 1] = sum;
+        }
+        if (ok && row < p.rows)
+          p.part_a[(long long)n * p.rows + row] = make_float4(part[0], part[1], part[2], part[3]);
+      } else {
+        if (!mbar_wait_warp(&sm->acc_full[0], (uint32_t)k & 1u, abort_flag) ||
+            !mbar_wait_warp(&sm->acc_full[1], (uint32_t)k & 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float lz = row < p.rows ? p.lz2[row] : 0.f;
+        const float lt = row < p.rows ? p.lt2[row] : 0.f;
+        float al = 0.f, ql = 0.f;
+        for (int c = 0; c * 32 < ncols; ++c) {
+          uint32_t rz[32], rt[32];
+          tmem_ld32(tmem + lane_base + c * 32, rz);
+          tmem_ld32(tmem + lane_base + kLBN + c * 32, rt);
+          tmem_ld_wait();
+          const int nv = min(32, ncols - c * 32);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (i < nv) {
+              const float da = fmaf(__uint_as_float(rz[i]), kLLog2e, -lz);
+              const float db = fmaf(__uint_as_float(rt[i]), kLLog2e, -lt);
+              const float e = ex2(fminf(da, db));
+              al += e;
+              if (da < db) ql += e;
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&sm->acc_empty[0]);
+          mbar_arrive(&sm->acc_empty[1]);
+        }
+        if (row < p.rows) p.part_b[(long long)n * p.rows + row] = make_float2(al, ql);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0 && sm->abort_flag) atomicOr(reinterpret_cast<unsigned*>(p.status), SPECOPD_FLAG_TIMEOUT);
+}
+
+// Per row, the tile pairs of pass A merged in tile order (one thread per row,
+// so the order is fixed): base-2 normalisers, natural ones for the caller, and
+// the non-finite check (a NaN or infinite logit leaves a non-finite pair).
+__global__ void lm_reduce_a_kernel(const float4* __restrict__ part, int n_tiles, int64_t rows, float* lz2,
+                                   float* lt2, float* lse_draft, float* lse_teacher, int32_t* status) {
+  const long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= rows) return;
+  float mz = -INFINITY, sz = 0.f, mt = -INFINITY, st = 0.f;
+  bool bad = false;
+  for (int n = 0; n < n_tiles; ++n) {
+    const float4 v = part[(long long)n * rows + row];
+    bad |= !(fabsf(v.x) < INFINITY) || !(fabsf(v.y) < INFINITY) || !(fabsf(v.z) < INFINITY) ||
+           !(fabsf(v.w) < INFINITY);
+    lse_merge(mz, sz, v.x, v.y);
+    lse_merge(mt, st, v.z, v.w);
+  }
+  const float a = mz + log2f(sz), b = mt + log2f(st);
+  lz2[row] = a;
+  lt2[row] = b;
+  if (lse_draft) lse_draft[row] = a * 0.6931471805599453f;
+  if (lse_teacher) lse_teacher[row] = b * 0.6931471805599453f;
+  if (bad) atomicOr(reinterpret_cast<unsigned*>(status), SPECOPD_FLAG_NONFINITE);
+}
+
+// Per row, pass B's shares summed in tile order.
+__global__ void lm_reduce_b_kernel(const float2* __restrict__ part, int n_tiles, int64_t rows, float* alpha,
+                                   float* q_less) {
+  const long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= rows) return;
+  float a = 0.f, q = 0.f;
+  for (int n = 0; n < n_tiles; ++n) {
+    const float2 v = part[(long long)n * rows + row];
+    a += v.x;
+    q += v.y;
+  }
+  alpha[row] = a;
+  if (q_less) q_less[row] = q;
+}
+
+// [rows, H] bf16, row-major -> 2-D map, box [64 elements][box_rows rows], 128-byte swizzle
+bool make_map_2d(CUtensorMap* tm, const void* ptr, int64_t rows, int H, int box_rows) {
+  TensorMapEncodeFn enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)H, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)H * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kLBK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+LmHeadLayout lm_head_layout(int64_t rows, int64_t V) {
+  LmHeadLayout L;
+  L.n_tiles = (V + kLBN - 1) / kLBN;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = (off + bytes + 255) / 256 * 256;
+    return at;
+  };
+  L.part_a = take((size_t)L.n_tiles * rows * sizeof(float4));
+  L.part_b = take((size_t)L.n_tiles * rows * sizeof(float2));
+  L.lz2 = take((size_t)rows * 4);
+  L.lt2 = take((size_t)rows * 4);
+  L.alpha = take((size_t)rows * 4);
+  L.total = off;
+  return L;
+}
+
+cudaError_t launch_lm_head_overlap(const LmHeadArgs& a, cudaStream_t stream) {
+  if (a.rows <= 0) return cudaSuccess;
+  CUtensorMap thd, twd, tht, twt;
+  if (!make_map_2d(&thd, a.h_draft, a.rows, a.Hd, kLBM) || !make_map_2d(&twd, a.w_draft, a.V, a.Hd, kLBN) ||
+      !make_map_2d(&tht, a.h_teacher, a.rows, a.Ht, kLBM) || !make_map_2d(&twt, a.w_teacher, a.V, a.Ht, kLBN))
+    return cudaErrorInvalidValue;
+  const LmHeadLayout L = lm_head_layout(a.rows, a.V);
+  uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+  LmParams p;
+  p.rows = a.rows;
+  p.V = a.V;
+  p.Hd = a.Hd;
+  p.Ht = a.Ht;
+  p.m_tiles = (int)((a.rows + kLBM - 1) / kLBM);
+  p.n_tiles = (int)L.n_tiles;
+  p.part_a = reinterpret_cast<float4*>(ws + L.part_a);
+  p.part_b = reinterpret_cast<float2*>(ws + L.part_b);
+  float* lz2 = reinterpret_cast<float*>(ws + L.lz2);
+  float* lt2 = reinterpret_cast<float*>(ws + L.lt2);
+  p.lz2 = lz2;
+  p.lt2 = lt2;
+  p.status = a.status;
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const size_t smem = sizeof(LmSmem) + 1024;
+  e = cudaFuncSetAttribute(lm_head_tile_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(lm_head_tile_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const long long total = (long long)p.m_tiles * p.n_tiles;
+  const unsigned grid = (unsigned)(total < sms ? total : sms);
+  const unsigned rb = (unsigned)((a.rows + 255) / 256);
+  lm_head_tile_kernel<0><<<grid, kLThreads, smem, stream>>>(thd, twd, tht, twt, p);
+  lm_reduce_a_kernel<<<rb, 256, 0, stream>>>(p.part_a, p.n_tiles, a.rows, lz2, lt2, a.lse_draft, a.lse_teacher,
+                                               a.status);
+  lm_head_tile_kernel<1><<<grid, kLThreads, smem, stream>>>(thd, twd, tht, twt, p);
+  float* alpha = a.alpha ? a.alpha : reinterpret_cast<float*>(ws + L.alpha);
+  lm_reduce_b_kernel<<<rb, 256, 0, stream>>>(p.part_b, p.n_tiles, a.rows, alpha, a.q_less);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_e2e_loss(alpha, a.num_branches, a.W, a.inv_count, a.loss, a.grad_alpha, stream);
+}
+
+}  // namespace specopd

@@ -30,6 +30,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "tmap.cuh"
 
 namespace specopd {
 namespace {
@@ -360,26 +361,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------ host side
-using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeFn get_encode() {
-  static EncodeFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeFn>(ptr);
-  }
-  return fn;
-}
-
 // [N, H, 128] bf16 -> 3-D map, box [64 elems][1 head][128 rows], 128-byte swizzle
 bool make_map(CUtensorMap* tm, const void* ptr, int64_t N, int H) {
-  EncodeFn enc = get_encode();
+  TensorMapEncodeFn enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)kHD, (cuuint64_t)H, (cuuint64_t)N};
   cuuint64_t strides[2] = {(cuuint64_t)kHD * 2, (cuuint64_t)H * kHD * 2};
