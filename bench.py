@@ -336,6 +336,10 @@ def run_gpu(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(case)
+    if world == 1 and not args.no_lm_head:
+        del st
+        torch.cuda.empty_cache()
+        out["kernels"]["lm_head_overlap"] = lm_head_measure(dev, peaks, args.seed)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -373,6 +377,51 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def lm_head_measure(dev, peaks, seed: int) -> dict:
+    """The LM-head path timed on its own (not part of the step): overlap
+    statistics, L and dL/dalpha straight from bf16 hidden states and heads at
+    the 8B-style shape (64 branches x W 16 = 1,024 rows, hidden 4,096 for both
+    models, V = 151,936).  The logits are formed twice (normalisers, then alpha)
+    and never stored: useful FLOPs count each logit once (2 GEMMs), executed
+    FLOPs both passes (4)."""
+    import torch
+    import synthetic as SY
+    from tree_attention_masked_b200 import specopd as S
+    nb, W, V, H = 64, 16, 151936, 4096
+    case = SY.make_lm_head_case("gqa8b-lm-head", nb, W, V, H, H, sig_t=3.0, sig_n=1.5, seed=seed,
+                                workers=min(8, os.cpu_count() or 1))
+    t = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    hd, wd, ht, wt = t(case.h_draft), t(case.w_draft), t(case.h_teacher), t(case.w_teacher)
+    R = case.rows
+    alpha = torch.empty(R, device=dev)
+    loss = torch.empty(1, device=dev)
+    ga = torch.empty(R, device=dev)
+    ws = torch.empty(S.specopd_lm_head_workspace_bytes(R, V), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    call = lambda: S.specopd_lm_head_overlap(hd, wd, ht, wt, nb, W, 0.0, alpha, loss, ws, status, grad_alpha=ga,
+                                             stream=stream)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    n = 10
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    gemm = 2.0 * R * H * V
+    useful = 2 * gemm / (ms * 1e-3) / 1e12
+    executed = 4 * gemm / (ms * 1e-3) / 1e12
+    return {"bound": "tensor", "ms": ms, "achieved": useful, "unit": "TFLOP/s", "peak": peaks["bf16"],
+            "frac": useful / peaks["bf16"], "useful_flops": 2 * gemm, "executed_flops": 4 * gemm,
+            "executed_tflops": executed, "executed_frac": executed / peaks["bf16"], "device_status": status.item(),
+            "shape": f"rows {R} (B {nb} x W {W}), hidden {H} (draft and teacher), V {V}, bf16",
+            "launches": 5}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -382,6 +431,7 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-lm-head", action="store_true", help="skip the separately timed LM-head path")
     args = ap.parse_args()
     # at least three untimed warm-up steps, whatever was asked for
     args.warmup = max(3, args.warmup)

@@ -273,22 +273,33 @@ __global__ void __launch_bounds__(kLThreads, 1)
   if (threadIdx.x == 0 && sm->abort_flag) atomicOr(reinterpret_cast<unsigned*>(p.status), SPECOPD_FLAG_TIMEOUT);
 }
 
-// Per row, the tile pairs of pass A merged in tile order (one thread per row,
-// so the order is fixed): base-2 normalisers, natural ones for the caller, and
-// the non-finite check (a NaN or infinite logit leaves a non-finite pair).
+// Per row (one warp), the tile pairs of pass A merged in a fixed order: lane
+// l takes tiles l, l + 32, ... in turn, then a fixed shuffle tree joins the
+// lanes.  Outputs: base-2 normalisers, natural ones for the caller, and the
+// non-finite check (a NaN or infinite logit leaves a non-finite pair).
 __global__ void lm_reduce_a_kernel(const float4* __restrict__ part, int n_tiles, int64_t rows, float* lz2,
                                    float* lt2, float* lse_draft, float* lse_teacher, int32_t* status) {
-  const long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long row = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
   if (row >= rows) return;
   float mz = -INFINITY, sz = 0.f, mt = -INFINITY, st = 0.f;
   bool bad = false;
-  for (int n = 0; n < n_tiles; ++n) {
+  for (int n = lane; n < n_tiles; n += 32) {
     const float4 v = part[(long long)n * rows + row];
     bad |= !(fabsf(v.x) < INFINITY) || !(fabsf(v.y) < INFINITY) || !(fabsf(v.z) < INFINITY) ||
            !(fabsf(v.w) < INFINITY);
     lse_merge(mz, sz, v.x, v.y);
     lse_merge(mt, st, v.z, v.w);
   }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float om = __shfl_xor_sync(0xffffffffu, mz, off), os = __shfl_xor_sync(0xffffffffu, sz, off);
+    const float pm = __shfl_xor_sync(0xffffffffu, mt, off), ps = __shfl_xor_sync(0xffffffffu, st, off);
+    lse_merge(mz, sz, om, os);
+    lse_merge(mt, st, pm, ps);
+  }
+  bad = __any_sync(0xffffffffu, bad);
+  if (lane != 0) return;
   const float a = mz + log2f(sz), b = mt + log2f(st);
   lz2[row] = a;
   lt2[row] = b;
@@ -297,17 +308,24 @@ __global__ void lm_reduce_a_kernel(const float4* __restrict__ part, int n_tiles,
   if (bad) atomicOr(reinterpret_cast<unsigned*>(status), SPECOPD_FLAG_NONFINITE);
 }
 
-// Per row, pass B's shares summed in tile order.
+// Per row (one warp), pass B's shares summed in the same fixed order.
 __global__ void lm_reduce_b_kernel(const float2* __restrict__ part, int n_tiles, int64_t rows, float* alpha,
                                    float* q_less) {
-  const long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long row = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
   if (row >= rows) return;
   float a = 0.f, q = 0.f;
-  for (int n = 0; n < n_tiles; ++n) {
+  for (int n = lane; n < n_tiles; n += 32) {
     const float2 v = part[(long long)n * rows + row];
     a += v.x;
     q += v.y;
   }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, off);
+    q += __shfl_xor_sync(0xffffffffu, q, off);
+  }
+  if (lane != 0) return;
   alpha[row] = a;
   if (q_less) q_less[row] = q;
 }
@@ -379,7 +397,7 @@ cudaError_t launch_lm_head_overlap(const LmHeadArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const long long total = (long long)p.m_tiles * p.n_tiles;
   const unsigned grid = (unsigned)(total < sms ? total : sms);
-  const unsigned rb = (unsigned)((a.rows + 255) / 256);
+  const unsigned rb = (unsigned)((a.rows + 7) / 8);  // one warp per row, 8 per block
   lm_head_tile_kernel<0><<<grid, kLThreads, smem, stream>>>(thd, twd, tht, twt, p);
   lm_reduce_a_kernel<<<rb, 256, 0, stream>>>(p.part_a, p.n_tiles, a.rows, lz2, lt2, a.lse_draft, a.lse_teacher,
                                                a.status);
