@@ -339,7 +339,7 @@ def run_gpu(args):
     if world == 1 and not args.no_lm_head:
         del st
         torch.cuda.empty_cache()
-        out["kernels"]["lm_head_overlap"] = lm_head_measure(dev, peaks, args.seed)
+        out["kernels"]["lm_head_overlap"] = lm_head_measure(dev, peaks, args.seed, args.lm_head_vocab)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -377,7 +377,7 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
-def lm_head_measure(dev, peaks, seed: int) -> dict:
+def lm_head_measure(dev, peaks, seed: int, V: int = 151936) -> dict:
     """The LM-head path timed on its own (not part of the step): overlap
     statistics, L and dL/dalpha straight from bf16 hidden states and heads at
     the 8B-style shape (64 branches x W 16 = 1,024 rows, hidden 4,096 for both
@@ -387,7 +387,7 @@ def lm_head_measure(dev, peaks, seed: int) -> dict:
     import torch
     import synthetic as SY
     from tree_attention_masked_b200 import specopd as S
-    nb, W, V, H = 64, 16, 151936, 4096
+    nb, W, H = 64, 16, 4096
     case = SY.make_lm_head_case("gqa8b-lm-head", nb, W, V, H, H, sig_t=3.0, sig_n=1.5, seed=seed,
                                 workers=min(8, os.cpu_count() or 1))
     t = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
@@ -432,11 +432,21 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-lm-head", action="store_true", help="skip the separately timed LM-head path")
+    ap.add_argument("--lm-head-only", action="store_true",
+                    help="time only the LM-head path (one JSON line; for profiling it alone)")
+    ap.add_argument("--lm-head-vocab", type=int, default=151936, help="vocabulary of the LM-head path")
     args = ap.parse_args()
     # at least three untimed warm-up steps, whatever was asked for
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
         run_reference(args)
+    elif args.lm_head_only:
+        import torch
+        from tree_attention_masked_b200.build import build
+        build()
+        d = lm_head_measure(torch.device("cuda", 0), load_peaks(), args.seed, args.lm_head_vocab)
+        print(json.dumps({"metric": "LM head + overlap statistics (logits never stored)", "value": d["achieved"],
+                          "unit": d["unit"], "higher_is_better": True, "kernel": d}), flush=True)
     else:
         run_gpu(args)
 
