@@ -383,7 +383,8 @@ def lm_head_measure(dev, peaks, seed: int, V: int = 151936) -> dict:
     the 8B-style shape (64 branches x W 16 = 1,024 rows, hidden 4,096 for both
     models, V = 151,936).  The logits are formed twice (normalisers, then alpha)
     and never stored: useful FLOPs count each logit once (2 GEMMs), executed
-    FLOPs both passes (4)."""
+    FLOPs both passes (4).  ms_with_grad_draft adds the third (draft-only) pass
+    that writes dL/dz."""
     import torch
     import synthetic as SY
     from tree_attention_masked_b200 import specopd as S
@@ -399,25 +400,31 @@ def lm_head_measure(dev, peaks, seed: int, V: int = 151936) -> dict:
     ws = torch.empty(S.specopd_lm_head_workspace_bytes(R, V), dtype=torch.uint8, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    call = lambda: S.specopd_lm_head_overlap(hd, wd, ht, wt, nb, W, 0.0, alpha, loss, ws, status, grad_alpha=ga,
-                                             stream=stream)
-    for _ in range(3):
-        call()
-    torch.cuda.synchronize()
-    n = 10
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(n):
-        call()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / n
+    grad = torch.empty(R, V, device=dev)
+    call = lambda g: S.specopd_lm_head_overlap(hd, wd, ht, wt, nb, W, 0.0, alpha, loss, ws, status, grad_alpha=ga,
+                                               grad=g, stream=stream)
+
+    def time_ms(g, n=10):
+        for _ in range(3):
+            call(g)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            call(g)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    ms = time_ms(None)
+    ms_grad = time_ms(grad)
     gemm = 2.0 * R * H * V
     useful = 2 * gemm / (ms * 1e-3) / 1e12
     executed = 4 * gemm / (ms * 1e-3) / 1e12
     return {"bound": "tensor", "ms": ms, "achieved": useful, "unit": "TFLOP/s", "peak": peaks["bf16"],
             "frac": useful / peaks["bf16"], "useful_flops": 2 * gemm, "executed_flops": 4 * gemm,
             "executed_tflops": executed, "executed_frac": executed / peaks["bf16"], "device_status": status.item(),
+            "ms_with_grad_draft": ms_grad, "launches_with_grad_draft": 6,
             "shape": f"rows {R} (B {nb} x W {W}), hidden {H} (draft and teacher), V {V}, bf16",
             "launches": 5}
 

@@ -255,10 +255,11 @@ size_t specopd_lm_head_workspace_bytes(int64_t rows, int64_t V);
  * supplied hidden states and a supplied head, and e2e_tv_loss consumes the
  * same-history aligned logits of draft and teacher.  Reading (the pages name
  * nothing more): logits = h head^T, no bias, temperature 1, every vocabulary
- * entry active.  alpha, L and dL/dalpha are those of specopd_tv_overlap_e2e
- * (section "Equations").  The logits of a row are formed twice, tile by tile
- * in TMEM (bf16 products, fp32 accumulation): once for the normalisers, once
- * for alpha and q_less.
+ * entry active.  alpha, L, dL/dalpha and dL/dz are those of
+ * specopd_tv_overlap_e2e (section "Equations").  The logits of a row are formed
+ * tile by tile in TMEM (bf16 products, fp32 accumulation) twice, once for the
+ * normalisers and once for alpha and q_less, and with grad_draft a third time
+ * (draft only) to write dL/dz = dL/dalpha * q (1[q < p] - q_less).
  *
  * h_draft [rows, Hd], head_draft [V, Hd], h_teacher [rows, Ht],
  * head_teacher [V, Ht]: device bf16, row-major and contiguous, 16-byte
@@ -266,7 +267,8 @@ size_t specopd_lm_head_workspace_bytes(int64_t rows, int64_t V);
  * b*W + i-1 holds y_{b,i}); rows must equal num_branches * W; count <= 0
  * means rows.  Outputs (device fp32): alpha [rows] (nullable: then kept in the
  * workspace), q_less [rows], lse_draft / lse_teacher [rows] (natural log),
- * loss (scalar) and grad_alpha [rows], all but loss nullable.  workspace:
+ * loss (scalar), grad_alpha [rows] and grad_draft [rows, ld_grad] (16-byte
+ * aligned rows, ld_grad >= V), all but loss nullable.  workspace:
  * device, >= specopd_lm_head_workspace_bytes(rows, V), 256-byte aligned;
  * the caller owns every buffer.  A non-finite logit sets
  * SPECOPD_FLAG_NONFINITE in *status; a timed-out in-kernel wait sets
@@ -276,8 +278,8 @@ size_t specopd_lm_head_workspace_bytes(int64_t rows, int64_t V);
 int specopd_lm_head_overlap(const void* h_draft, const void* head_draft, int Hd, const void* h_teacher,
                             const void* head_teacher, int Ht, int64_t rows, int64_t V, int64_t num_branches, int W,
                             double count, float* alpha, float* q_less, float* lse_draft, float* lse_teacher,
-                            float* loss, float* grad_alpha, void* workspace, size_t workspace_bytes,
-                            int32_t* status, specopd_stream_t stream);
+                            float* loss, float* grad_alpha, float* grad_draft, int64_t ld_grad, void* workspace,
+                            size_t workspace_bytes, int32_t* status, specopd_stream_t stream);
 
 /*
  * specopd_tv_overlap_e2e_static -- specopd_tv_overlap_e2e without a workspace.

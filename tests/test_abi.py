@@ -107,13 +107,18 @@ def test_argument_errors_before_launch(S):
     # 16-byte aligned operands, a large enough workspace
     lm = lib["specopd_lm_head_overlap"]
     need = S.specopd_lm_head_workspace_bytes(8, 1000)
-    assert lm(16, 16, 96, 16, 16, 128, 8, 1000, 2, 4, 0.0, 16, None, None, None, 16, None, 256, need, 16, None) == -2
-    assert lm(16, 16, 128, 16, 16, 128, 8, 1000, 3, 4, 0.0, 16, None, None, None, 16, None, 256, need, 16, None) == -2
-    assert lm(24, 16, 128, 16, 16, 128, 8, 1000, 2, 4, 0.0, 16, None, None, None, 16, None, 256, need, 16, None) == -6
-    assert lm(16, 16, 128, 16, 16, 128, 8, 1000, 2, 4, 0.0, 16, None, None, None, 16, None, 256, need - 1, 16,
-              None) == -5
-    assert lm(16, 16, 128, 16, 16, 128, 8, 1000, 2, 4, 0.0, 16, None, None, None, None, None, 256, need, 16,
-              None) == -1
+    assert lm(16, 16, 96, 16, 16, 128, 8, 1000, 2, 4, 0.0, 16, None, None, None, 16, None, None, 0, 256, need, 16, None) == -2
+    assert lm(16, 16, 128, 16, 16, 128, 8, 1000, 3, 4, 0.0, 16, None, None, None, 16, None, None, 0, 256, need, 16, None) == -2
+    assert lm(24, 16, 128, 16, 16, 128, 8, 1000, 2, 4, 0.0, 16, None, None, None, 16, None, None, 0, 256, need, 16, None) == -6
+    assert lm(16, 16, 128, 16, 16, 128, 8, 1000, 2, 4, 0.0, 16, None, None, None, 16, None, None, 0, 256, need - 1,
+              16, None) == -5
+    assert lm(16, 16, 128, 16, 16, 128, 8, 1000, 2, 4, 0.0, 16, None, None, None, None, None, None, 0, 256, need,
+              16, None) == -1
+    # a gradient buffer with a leading dimension below V or not a multiple of 4 floats
+    assert lm(16, 16, 128, 16, 16, 128, 8, 1000, 2, 4, 0.0, 16, None, None, None, 16, None, 16, 999, 256, need, 16,
+              None) == -6
+    assert lm(16, 16, 128, 16, 16, 128, 8, 1000, 2, 4, 0.0, 16, None, None, None, 16, None, 16, 1002, 256, need, 16,
+              None) == -6
     assert S._c["specopd_status_string"](-5) == b"workspace missing, too small or misaligned"
 
 

@@ -1,21 +1,28 @@
 """Overlap statistics from hidden states and LM heads on the GPU against the
 oracle: alpha, q_less and L within 1e-4 absolute, the normalisers within 1e-4
-absolute, dL/dalpha within 1e-4 absolute.  The GPU forms the logits with bf16
-products and fp32 accumulation; the oracle in fp64 from the same bf16 values."""
+absolute, dL/dalpha within 1e-4 absolute, dL/dz within 1e-3 relative L2.  The
+GPU forms the logits with bf16 products and fp32 accumulation; the oracle in
+fp64 from the same bf16 values."""
 import numpy as np
 import pytest
 import torch
 
 import synthetic as SY
 from oracle import lm_head as LM
+from oracle import overlap as OO
 from tree_attention_masked_b200 import specopd as S
 
 pytestmark = pytest.mark.gpu
 
 TOL = 1e-4
+GRAD_TOL = 1e-3
 
 
-def run(case, count=0.0, with_optional=True):
+def rel_l2(a, b):
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def run(case, count=0.0, with_optional=True, with_grad=True):
     dev = torch.device("cuda")
     t = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
     hd, wd, ht, wt = t(case.h_draft), t(case.w_draft), t(case.h_teacher), t(case.w_teacher)
@@ -26,21 +33,35 @@ def run(case, count=0.0, with_optional=True):
         out.update(q_less=f(), lse_draft=f(), lse_teacher=f(), grad_alpha=f())
     ws = torch.empty(S.specopd_lm_head_workspace_bytes(R, case.V), dtype=torch.uint8, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
+    grad = None
+    if with_grad:  # rows padded to a multiple of 4 floats; the pad must stay untouched
+        ld = (case.V + 3) // 4 * 4
+        gbuf = torch.full((R, ld), 7.0, device=dev)
+        grad = gbuf[:, :case.V]
     S.specopd_lm_head_overlap(hd, wd, ht, wt, case.num_branches, case.W, count, out["alpha"], out["loss"], ws,
                               status, q_less=out.get("q_less"), lse_draft=out.get("lse_draft"),
-                              lse_teacher=out.get("lse_teacher"), grad_alpha=out.get("grad_alpha"))
+                              lse_teacher=out.get("lse_teacher"), grad_alpha=out.get("grad_alpha"), grad=grad)
     torch.cuda.synchronize()
     assert status.item() == 0
-    return {k: v.cpu().numpy().astype(np.float64) for k, v in out.items()}
+    res = {k: v.cpu().numpy().astype(np.float64) for k, v in out.items()}
+    if with_grad:
+        assert torch.all(gbuf[:, case.V:] == 7.0)
+        res["grad"] = grad.cpu().numpy().astype(np.float64)
+    return res
 
 
 def oracle(case, rows=None, count=None):
+    """The oracle's statistics, plus dL/dz (the overlap module's gradient on the
+    oracle's logits).  rows: whole branches; count then defaults to all rows."""
     f64 = lambda a: SY.to_f64(a, "bf16")
     hd, ht = f64(case.h_draft), f64(case.h_teacher)
     if rows is not None:
         hd, ht = hd[rows], ht[rows]
-    W = case.W if rows is None else len(rows)
-    return LM.lm_head_overlap(hd, f64(case.w_draft), ht, f64(case.w_teacher), W, count)
+        count = case.rows if count is None else count
+    wd, wt = f64(case.w_draft), f64(case.w_teacher)
+    out = LM.lm_head_overlap(hd, wd, ht, wt, case.W, count)
+    out["grad"] = OO.e2e_tv_grad_draft(LM.prediction_logits(hd, wd), LM.prediction_logits(ht, wt), case.W, count)
+    return out
 
 
 CASES = [
@@ -69,6 +90,10 @@ def test_lm_head_overlap_matches_oracle(name, nb, W, V, Hd, Ht):
     for k in keys:
         assert np.max(np.abs(got[k] - ref[k])) <= TOL, (k, np.max(np.abs(got[k] - ref[k])))
     assert abs(got["loss"][0] - ref["loss"]) <= TOL
+    if V == 1:
+        assert np.max(np.abs(got["grad"])) <= 1e-6   # q (bit - q_less) = 0 for either tie decision
+    else:
+        assert rel_l2(got["grad"], ref["grad"]) <= GRAD_TOL, rel_l2(got["grad"], ref["grad"])
 
 
 def test_identical_models_give_full_overlap():
@@ -78,11 +103,13 @@ def test_identical_models_give_full_overlap():
     assert np.max(np.abs(got["alpha"] - 1.0)) <= 1e-5
     assert np.all(got["q_less"] == 0.0)   # identical logits: q < p nowhere
     assert abs(got["loss"][0]) <= 1e-5
+    # q < p nowhere and q_less = 0: dL/dz = g q (0 - 0) = 0 exactly
+    assert np.all(got["grad"] == 0.0)
 
 
 def test_optional_outputs_and_count():
     case = SY.make_lm_head_case("opt", 3, 4, 2048, 64, 64, sig_t=2.0, sig_n=1.0, seed=9)
-    a = run(case, with_optional=False)
+    a = run(case, with_optional=False, with_grad=False)
     b = run(case, count=100.0)
     assert np.array_equal(a["alpha"], b["alpha"])   # the same launches: identical bits
     ref = oracle(case, count=100)
@@ -105,8 +132,9 @@ def test_full_size_sampled_branches():
     for b in (0, 37, 63):
         rows = np.arange(b * 16, (b + 1) * 16)
         ref = oracle(case, rows=rows)
-        for k in ("alpha", "q_less", "lse_draft", "lse_teacher"):
+        for k in ("alpha", "q_less", "lse_draft", "lse_teacher", "grad_alpha"):
             assert np.max(np.abs(got[k][rows] - ref[k])) <= TOL, (b, k)
+        assert rel_l2(got["grad"][rows], ref["grad"]) <= GRAD_TOL, b
     # the loss from the GPU's own alpha, by the definition
     from oracle import overlap as OO
     assert abs(got["loss"][0] - OO.e2e_tv_loss(got["alpha"], 16)) <= 1e-6

@@ -302,8 +302,8 @@ size_t specopd_lm_head_workspace_bytes(int64_t rows, int64_t V) {
 int specopd_lm_head_overlap(const void* h_draft, const void* head_draft, int Hd, const void* h_teacher,
                             const void* head_teacher, int Ht, int64_t rows, int64_t V, int64_t num_branches, int W,
                             double count, float* alpha, float* q_less, float* lse_draft, float* lse_teacher,
-                            float* loss, float* grad_alpha, void* workspace, size_t workspace_bytes,
-                            int32_t* status, specopd_stream_t stream) {
+                            float* loss, float* grad_alpha, float* grad_draft, int64_t ld_grad, void* workspace,
+                            size_t workspace_bytes, int32_t* status, specopd_stream_t stream) {
   if (W < 1 || W > SPECOPD_MAX_W || num_branches < 0 || rows != num_branches * W) return SPECOPD_ERR_SHAPE;
   if (V < 1 || V > (1LL << 31) - 256 || Hd < 64 || Ht < 64 || Hd % 64 || Ht % 64 || Hd > (1 << 20) ||
       Ht > (1 << 20) || rows > (1LL << 31) - 128)
@@ -315,6 +315,7 @@ int specopd_lm_head_overlap(const void* h_draft, const void* head_draft, int Hd,
   if (!h_draft || !head_draft || !h_teacher || !head_teacher) return SPECOPD_ERR_ARG;
   if (!aligned16(h_draft) || !aligned16(head_draft) || !aligned16(h_teacher) || !aligned16(head_teacher))
     return SPECOPD_ERR_ALIGN;
+  if (grad_draft && (ld_grad < V || !aligned16(grad_draft) || (ld_grad * 4) % 16)) return SPECOPD_ERR_ALIGN;
   const LmHeadLayout L = lm_head_layout(rows, V);
   if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) % kAlign))
     return SPECOPD_ERR_WORKSPACE;
@@ -337,6 +338,8 @@ int specopd_lm_head_overlap(const void* h_draft, const void* head_draft, int Hd,
   a.lse_teacher = lse_teacher;
   a.loss = loss;
   a.grad_alpha = grad_alpha;
+  a.grad_draft = grad_draft;
+  a.ld_grad = ld_grad;
   a.workspace = workspace;
   a.status = status;
   return cuda_status(launch_lm_head_overlap(a, st));

@@ -108,12 +108,14 @@ struct LmHeadArgs {
   float* lse_teacher;   // nullable
   float* loss;
   float* grad_alpha;    // nullable
+  float* grad_draft;    // nullable: [rows, ld_grad] dL/dz
+  int64_t ld_grad;
   void* workspace;
   int32_t* status;
 };
 struct LmHeadLayout {
   int64_t n_tiles;
-  size_t part_a, part_b, lz2, lt2, alpha, total;
+  size_t part_a, part_b, lz2, lt2, alpha, q_less, g, bits, total;
 };
 LmHeadLayout lm_head_layout(int64_t rows, int64_t V);
 cudaError_t launch_lm_head_overlap(const LmHeadArgs& a, cudaStream_t stream);

@@ -16,7 +16,10 @@
 //   pass B -- the same tiles again; the epilogue forms the row's share of
 //             alpha = sum exp2(min(z2 - lz2, t2 - lt2)) and q_less;
 //   reduce  -- per row, the shares summed in tile order: alpha, q_less;
-// then the E2E-TV loss and dL/dalpha from alpha.
+// then the E2E-TV loss and dL/dalpha from alpha, and, when the caller asks for
+// the gradient with respect to the draft logits,
+//   pass C -- the draft tiles a third time; the epilogue writes
+//             dL/dz = g q ([q < p] - q_less) from pass B's comparison bits.
 //
 // Tile kernel: a persistent grid, one CTA per SM, tiles dealt round-robin in
 // vocabulary-major order (the row tiles of one head tile run together, so the
@@ -67,8 +70,15 @@ struct LmParams {
   int m_tiles, n_tiles;
   float4* part_a;        // [n_tiles][rows]: (mz, sz, mt, st), base 2
   float2* part_b;        // [n_tiles][rows]: (alpha share, q_less share)
-  const float* lz2;      // [rows] draft normaliser, base 2 (pass B)
+  const float* lz2;      // [rows] draft normaliser, base 2 (passes B, C)
   const float* lt2;      // [rows] teacher normaliser, base 2 (pass B)
+  uint32_t* bits;        // [n_words][rows]: bit i of word w = [q < p] at entry 32 w + i (pass B
+                         // writes it when non-null; pass C reads it)
+  int64_t n_words;       // ceil(V / 32)
+  const float* ql;       // [rows] q_less (pass C)
+  const float* g;        // [rows] dL/dalpha (pass C)
+  float* grad;           // [rows, ld_grad] dL/dz (pass C)
+  int64_t ld_grad;
   int32_t* status;
 };
 
@@ -89,6 +99,7 @@ __global__ void __launch_bounds__(kLThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const long long total = (long long)p.m_tiles * p.n_tiles;
+  constexpr int kHalves = PASS == 2 ? 1 : 2;  // pass C forms the draft logits only
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kLStages; ++s) {
@@ -126,7 +137,7 @@ __global__ void __launch_bounds__(kLThreads, 1)
       bool ok = true;
       for (long long tau = blockIdx.x; ok && tau < total; tau += gridDim.x) {
         const int m = (int)(tau % p.m_tiles), n = (int)(tau / p.m_tiles);
-        for (int h = 0; ok && h < 2; ++h) {
+        for (int h = 0; ok && h < kHalves; ++h) {
           const CUtensorMap* ta = h ? &tm_ht : &tm_hd;
           const CUtensorMap* tb = h ? &tm_wt : &tm_wd;
           const int nk = (h ? p.Ht : p.Hd) / kLBK;
@@ -154,7 +165,7 @@ __global__ void __launch_bounds__(kLThreads, 1)
       int k = 0;  // tiles of this CTA so far
       bool ok = true;
       for (long long tau = blockIdx.x; ok && tau < total; tau += gridDim.x, ++k) {
-        for (int h = 0; ok && h < 2; ++h) {
+        for (int h = 0; ok && h < kHalves; ++h) {
           if (k > 0 && !mbar_wait(&sm->acc_empty[h], (uint32_t)(k - 1) & 1u, abort_flag)) {
             ok = false;
             break;
@@ -226,6 +237,42 @@ __global__ void __launch_bounds__(kLThreads, 1)
         }
         if (ok && row < p.rows)
           p.part_a[(long long)n * p.rows + row] = make_float4(part[0], part[1], part[2], part[3]);
+      } else if (PASS == 2) {
+        // dL/dz = g q ([q < p] - q_less) from the draft logits and pass B's bits
+        if (!mbar_wait_warp(&sm->acc_full[0], (uint32_t)k & 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const bool live_row = row < p.rows;
+        const float lz = live_row ? p.lz2[row] : 0.f;
+        const float G = live_row ? p.g[row] : 0.f;
+        const float Q = live_row ? p.ql[row] : 0.f;
+        const float omq = 1.f - Q, zmq = 0.f - Q;
+        float* grow = p.grad + row * p.ld_grad + col0;
+        for (int c = 0; c * 32 < ncols; ++c) {
+          uint32_t rz[32];
+          tmem_ld32(tmem + lane_base + c * 32, rz);
+          const uint32_t word = live_row ? p.bits[((long long)n * (kLBN / 32) + c) * p.rows + row] : 0u;
+          tmem_ld_wait();
+          const int nv = min(32, ncols - c * 32);
+          float o[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            o[i] = G * ex2(fmaf(__uint_as_float(rz[i]), kLLog2e, -lz)) * (((word >> i) & 1u) ? omq : zmq);
+          if (live_row) {
+            if (nv == 32) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 4)
+                __stcs(reinterpret_cast<float4*>(grow + c * 32 + i), make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]));
+            } else {
+              for (int i = 0; i < nv; ++i) grow[c * 32 + i] = o[i];
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm->acc_empty[0]);
       } else {
         if (!mbar_wait_warp(&sm->acc_full[0], (uint32_t)k & 1u, abort_flag) ||
             !mbar_wait_warp(&sm->acc_full[1], (uint32_t)k & 1u, abort_flag)) {
@@ -242,6 +289,7 @@ __global__ void __launch_bounds__(kLThreads, 1)
           tmem_ld32(tmem + lane_base + kLBN + c * 32, rt);
           tmem_ld_wait();
           const int nv = min(32, ncols - c * 32);
+          uint32_t word = 0;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             if (i < nv) {
@@ -249,9 +297,13 @@ __global__ void __launch_bounds__(kLThreads, 1)
               const float db = fmaf(__uint_as_float(rt[i]), kLLog2e, -lt);
               const float e = ex2(fminf(da, db));
               al += e;
-              if (da < db) ql += e;
+              if (da < db) {
+                ql += e;
+                word |= 1u << i;
+              }
             }
           }
+          if (p.bits && row < p.rows) p.bits[((long long)n * (kLBN / 32) + c) * p.rows + row] = word;
         }
         tc_fence_before();
         __syncwarp();
@@ -359,6 +411,9 @@ LmHeadLayout lm_head_layout(int64_t rows, int64_t V) {
   L.lz2 = take((size_t)rows * 4);
   L.lt2 = take((size_t)rows * 4);
   L.alpha = take((size_t)rows * 4);
+  L.q_less = take((size_t)rows * 4);
+  L.g = take((size_t)rows * 4);
+  L.bits = take((size_t)L.n_tiles * (kLBN / 32) * rows * 4);
   L.total = off;
   return L;
 }
@@ -384,6 +439,14 @@ cudaError_t launch_lm_head_overlap(const LmHeadArgs& a, cudaStream_t stream) {
   float* lt2 = reinterpret_cast<float*>(ws + L.lt2);
   p.lz2 = lz2;
   p.lt2 = lt2;
+  p.n_words = L.n_tiles * (kLBN / 32);
+  p.bits = a.grad_draft ? reinterpret_cast<uint32_t*>(ws + L.bits) : nullptr;
+  float* q_less = a.q_less ? a.q_less : reinterpret_cast<float*>(ws + L.q_less);
+  float* g = a.grad_alpha ? a.grad_alpha : reinterpret_cast<float*>(ws + L.g);
+  p.ql = q_less;
+  p.g = g;
+  p.grad = a.grad_draft;
+  p.ld_grad = a.ld_grad;
   p.status = a.status;
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -395,6 +458,8 @@ cudaError_t launch_lm_head_overlap(const LmHeadArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(lm_head_tile_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(lm_head_tile_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   const long long total = (long long)p.m_tiles * p.n_tiles;
   const unsigned grid = (unsigned)(total < sms ? total : sms);
   const unsigned rb = (unsigned)((a.rows + 7) / 8);  // one warp per row, 8 per block
@@ -403,10 +468,14 @@ cudaError_t launch_lm_head_overlap(const LmHeadArgs& a, cudaStream_t stream) {
                                                a.status);
   lm_head_tile_kernel<1><<<grid, kLThreads, smem, stream>>>(thd, twd, tht, twt, p);
   float* alpha = a.alpha ? a.alpha : reinterpret_cast<float*>(ws + L.alpha);
-  lm_reduce_b_kernel<<<rb, 256, 0, stream>>>(p.part_b, p.n_tiles, a.rows, alpha, a.q_less);
+  lm_reduce_b_kernel<<<rb, 256, 0, stream>>>(p.part_b, p.n_tiles, a.rows, alpha, q_less);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_e2e_loss(alpha, a.num_branches, a.W, a.inv_count, a.loss, a.grad_alpha, stream);
+  e = launch_e2e_loss(alpha, a.num_branches, a.W, a.inv_count, a.loss, g, stream);
+  if (e != cudaSuccess || !a.grad_draft) return e;
+  // pass C: the draft logits once more, now with dL/dalpha known, into dL/dz
+  lm_head_tile_kernel<2><<<grid, kLThreads, smem, stream>>>(thd, twd, tht, twt, p);
+  return cudaGetLastError();
 }
 
 }  // namespace specopd

@@ -73,7 +73,7 @@ _c = {
                                           _i64, _i64, _i64, _int, _f64, _vp, _vp, _vp, _i64, _vp, _vp),
     "specopd_lm_head_workspace_bytes": _sig("specopd_lm_head_workspace_bytes", _sz, _i64, _i64),
     "specopd_lm_head_overlap": _sig("specopd_lm_head_overlap", _int, _vp, _vp, _int, _vp, _vp, _int, _i64, _i64,
-                                    _i64, _int, _f64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp),
+                                    _i64, _int, _f64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp, _vp),
     "specopd_status_string": _sig("specopd_status_string", ctypes.c_char_p, _int),
 }
 
@@ -226,9 +226,9 @@ def specopd_lm_head_workspace_bytes(rows: int, V: int) -> int:
 
 def specopd_lm_head_overlap(h_draft, head_draft, h_teacher, head_teacher, num_branches: int, W: int,
                             count: float, alpha, loss, workspace, status, q_less=None, lse_draft=None,
-                            lse_teacher=None, grad_alpha=None, stream=None) -> None:
-    """Overlap, E2E-TV loss and dL/dalpha from bf16 hidden states [rows, H]
-    and heads [V, H] (contiguous); the logits are never stored."""
+                            lse_teacher=None, grad_alpha=None, grad=None, stream=None) -> None:
+    """Overlap, E2E-TV loss, dL/dalpha and (with grad) dL/dz from bf16 hidden
+    states [rows, H] and heads [V, H] (contiguous); the logits are never stored."""
     _contig(h_draft, head_draft, h_teacher, head_teacher)
     for t in (h_draft, head_draft, h_teacher, head_teacher):
         if t.dtype != torch.bfloat16:
@@ -237,4 +237,5 @@ def specopd_lm_head_overlap(h_draft, head_draft, h_teacher, head_teacher, num_br
     _check("specopd_lm_head_overlap", _c["specopd_lm_head_overlap"](
         _ptr(h_draft), _ptr(head_draft), h_draft.shape[1], _ptr(h_teacher), _ptr(head_teacher), h_teacher.shape[1],
         h_draft.shape[0], head_draft.shape[0], num_branches, W, count, _ptr(alpha), _ptr(q_less), _ptr(lse_draft),
-        _ptr(lse_teacher), _ptr(loss), _ptr(grad_alpha), _ptr(workspace), wb, _ptr(status), _stream(stream)))
+        _ptr(lse_teacher), _ptr(loss), _ptr(grad_alpha), _ptr(grad), grad.stride(0) if grad is not None else 0,
+        _ptr(workspace), wb, _ptr(status), _stream(stream)))
