@@ -55,6 +55,7 @@ constexpr float kLLog2e = 1.4426950408889634f;
 struct alignas(1024) LmSmem {
   uint8_t a[kLStages][kLABytes];
   uint8_t b[kLStages][kLBBytes];
+  float out[4][32][33];   // pass C: a warp's 32 x 32 gradient block, transposed for coalesced stores
   uint64_t full[kLStages];
   uint64_t empty[kLStages];
   uint64_t acc_full[2];   // MMAs of the draft / teacher half done
@@ -165,13 +166,18 @@ __global__ void __launch_bounds__(kLThreads, 1)
       int k = 0;  // tiles of this CTA so far
       bool ok = true;
       for (long long tau = blockIdx.x; ok && tau < total; tau += gridDim.x, ++k) {
-        for (int h = 0; ok && h < kHalves; ++h) {
-          if (k > 0 && !mbar_wait(&sm->acc_empty[h], (uint32_t)(k - 1) & 1u, abort_flag)) {
+        for (int mdl = 0; ok && mdl < kHalves; ++mdl) {
+          // TMEM half: the model's own in passes A and B; in pass C (draft
+          // only) the halves alternate between tiles, so the epilogue of one
+          // tile runs under the MMAs of the next
+          const int h = PASS == 2 ? (k & 1) : mdl;
+          const int use = PASS == 2 ? (k >> 1) : k;  // earlier uses of half h
+          if (use > 0 && !mbar_wait(&sm->acc_empty[h], (uint32_t)(use - 1) & 1u, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const int nk = (h ? p.Ht : p.Hd) / kLBK;
+          const int nk = (mdl ? p.Ht : p.Hd) / kLBK;
           for (int kb = 0; kb < nk; ++kb, ++it) {
             const int s = (int)(it % kLStages);
             if (!mbar_wait(&sm->full[s], (uint32_t)(it / kLStages) & 1u, abort_flag)) {
@@ -239,7 +245,8 @@ __global__ void __launch_bounds__(kLThreads, 1)
           p.part_a[(long long)n * p.rows + row] = make_float4(part[0], part[1], part[2], part[3]);
       } else if (PASS == 2) {
         // dL/dz = g q ([q < p] - q_less) from the draft logits and pass B's bits
-        if (!mbar_wait_warp(&sm->acc_full[0], (uint32_t)k & 1u, abort_flag)) {
+        const int hb = k & 1;  // the TMEM half this tile went to
+        if (!mbar_wait_warp(&sm->acc_full[hb], (uint32_t)(k >> 1) & 1u, abort_flag)) {
           ok = false;
           break;
         }
@@ -249,30 +256,28 @@ __global__ void __launch_bounds__(kLThreads, 1)
         const float G = live_row ? p.g[row] : 0.f;
         const float Q = live_row ? p.ql[row] : 0.f;
         const float omq = 1.f - Q, zmq = 0.f - Q;
-        float* grow = p.grad + row * p.ld_grad + col0;
+        float(*blk)[33] = sm->out[q4];
+        const long long row0 = (long long)m * kLBM + q4 * 32;  // the warp's first row
         for (int c = 0; c * 32 < ncols; ++c) {
           uint32_t rz[32];
-          tmem_ld32(tmem + lane_base + c * 32, rz);
+          tmem_ld32(tmem + lane_base + hb * kLBN + c * 32, rz);
           const uint32_t word = live_row ? p.bits[((long long)n * (kLBN / 32) + c) * p.rows + row] : 0u;
           tmem_ld_wait();
           const int nv = min(32, ncols - c * 32);
-          float o[32];
+          // lane = row: each lane fills its row of the block ...
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            o[i] = G * ex2(fmaf(__uint_as_float(rz[i]), kLLog2e, -lz)) * (((word >> i) & 1u) ? omq : zmq);
-          if (live_row) {
-            if (nv == 32) {
-#pragma unroll
-              for (int i = 0; i < 32; i += 4)
-                __stcs(reinterpret_cast<float4*>(grow + c * 32 + i), make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]));
-            } else {
-              for (int i = 0; i < nv; ++i) grow[c * 32 + i] = o[i];
-            }
-          }
+            blk[lane][i] = G * ex2(fmaf(__uint_as_float(rz[i]), kLLog2e, -lz)) * (((word >> i) & 1u) ? omq : zmq);
+          __syncwarp();
+          // ... then the warp stores it row by row: 32 consecutive floats per store
+          float* gcol = p.grad + col0 + c * 32 + lane;
+          for (int r = 0; r < 32; ++r)
+            if (row0 + r < p.rows && lane < nv) __stcs(gcol + (row0 + r) * p.ld_grad, blk[r][lane]);
+          __syncwarp();
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm->acc_empty[0]);
+        if (lane == 0) mbar_arrive(&sm->acc_empty[hb]);
       } else {
         if (!mbar_wait_warp(&sm->acc_full[0], (uint32_t)k & 1u, abort_flag) ||
             !mbar_wait_warp(&sm->acc_full[1], (uint32_t)k & 1u, abort_flag)) {
