@@ -59,7 +59,7 @@ struct OverlapLayout {
 // Workspace of the fused overlap pass (all regions 256-byte aligned):
 //   mbits     [rows][mbits_ld]  one bit per logit, [q < p]
 //   lz2, ql, g [rows]           draft normaliser (base 2), q_less, dL/dalpha
-//   counters  branch arrivals [nb] + branches done [1]
+//   counters  branch arrivals [nb] + branches done [1] + gradient units claimed [1]
 //   bsum      [nb] doubles      each branch's share of L
 OverlapLayout overlap_layout(int64_t rows, int64_t V, int64_t nb) {
   OverlapLayout L;
@@ -74,7 +74,7 @@ OverlapLayout overlap_layout(int64_t rows, int64_t V, int64_t nb) {
   L.g = off;
   off = align_up(off + (size_t)rows * 4);
   L.counters = off;
-  L.counters_bytes = (size_t)(nb + 1) * 4;
+  L.counters_bytes = (size_t)(nb + 2) * 4;
   off = align_up(off + L.counters_bytes);
   L.bsum = off;
   off = align_up(off + (size_t)nb * 8);
@@ -268,7 +268,7 @@ int specopd_tv_overlap_e2e(const void* draft, const void* teacher, specopd_dtype
   a.ql = reinterpret_cast<float*>(ws + L.ql);
   a.g = reinterpret_cast<float*>(ws + L.g);
   uint32_t* counters = reinterpret_cast<uint32_t*>(ws + L.counters);
-  a.branch_cnt = counters;  // [nb] arrivals per branch, then [1] branches done
+  a.branch_cnt = counters;  // [nb] arrivals per branch, [1] branches done, [1] gradient units claimed
   a.branch_sum = reinterpret_cast<double*>(ws + L.bsum);
   a.loss = loss;
   a.W = W;

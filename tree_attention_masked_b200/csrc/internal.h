@@ -70,7 +70,8 @@ struct OverlapArgs {
   float* lz2;        // [rows] draft normaliser, log2 units
   float* ql;         // [rows] q_less
   float* g;          // [rows] dL/dalpha
-  uint32_t* branch_cnt;  // [num_branches + 1], zero on entry
+  uint32_t* branch_cnt;  // [num_branches + 2], zero on entry: arrivals per branch, branches done,
+                         // gradient units claimed
   double* branch_sum;    // [num_branches]
   float* loss;
   int W;

@@ -146,6 +146,7 @@ constexpr int kRCons = 512;                      // consumer threads (16 warps, 
 constexpr int kRGradWarps = 8;                   // gradient warps (warpgroups 5-6)
 constexpr int kGUnit = 8192;                     // logits per gradient stage
 constexpr int kGStages = 4;
+constexpr int kGParts = 4;                       // gradient units per row (claimed one at a time)
 constexpr uint32_t kGStageBytes = kGUnit * 2 + kGUnit / 8;  // draft logits + bits
 constexpr int kRThreads = kRHead + kRCons + 32 * kRGradWarps;
 constexpr int kRWarps = kRCons / 32;
@@ -191,6 +192,8 @@ struct GradCtl {
   uint64_t full[kGStages];
   uint64_t empty[kGStages];
   float info[kGStages][4];  // (lz2, q_less, dL/dalpha) of the stage's row
+  long long row[kGStages];  // the stage's row; -1: no more work
+  int e0[kGStages];         // the stage's first logit
 };
 
 struct RingRed {
@@ -467,43 +470,67 @@ __global__ void __launch_bounds__(kRThreads, 1) tv_stats_bf16_ring_kernel(const 
 }
 
 // ---------------- gradient
-// The ring kernel's gradient side.  CTA c takes rows grad_begin + c, + gridDim.x,
-// ... (the rows whose statistics it computed, when both ranges coincide).  A
-// row waits until its branch's dL/dalpha is published (count W + 1, set by
-// the branch's last row in this launch); then one producer thread streams
-// its draft logits and bits through kGStages stages of shared memory (bulk
-// copies, L2 evict_first, no multicast) and the gradient warps write
-// dL/dz = g q ([q < p] - q_less) with 16-byte streaming stores.  The launch
-// is cooperative: every CTA is resident and the statistics never wait for
-// the gradient, so every wait ends.  All waits are bounded.
+// The ring kernel's gradient side.  The gradient of rows [grad_begin,
+// grad_end) is cut into units of a quarter row (in row order) that the CTAs'
+// gradient producers claim from a global counter, so whichever SM is free
+// takes the next unit and the last branches' gradient spreads over the whole
+// GPU.  A unit waits until its branch's dL/dalpha is published (count W + 1,
+// set by the branch's last row in this launch); then one producer thread
+// streams its draft logits and bits through kGStages stages of shared memory
+// (bulk copies, L2 evict_first, no multicast), each tagged with its row and
+// first logit, and the gradient warps write dL/dz = g q ([q < p] - q_less)
+// with 16-byte stores hinted L2 evict_first.  The launch is cooperative: every
+// CTA is resident and the statistics never wait for the gradient, so every
+// wait ends.  All waits are bounded.
 __device__ void grad_producer(const OverlapArgs& a, GradCtl* gc, uint8_t* gbuf, volatile int* abort_flag) {
   const uint64_t pol = l2_policy_evict_first();
+  const long long nrows = a.grad_end - a.grad_begin;
+  const long long per_row = (a.V + kGUnit - 1) / kGUnit;  // stages per row
+  const long long per_unit = (per_row + kGParts - 1) / kGParts;
+  const long long units = kGParts * nrows;
+  unsigned* claim = a.branch_cnt + a.num_branches + 1;
   long long k = 0;  // stages issued
-  bool ok = true;
-  for (long long row = a.grad_begin + blockIdx.x; ok && row < a.grad_end; row += gridDim.x) {
-    const unsigned* cnt = a.branch_cnt + row / a.W;
-    const long long t0 = clock64();
-    while (ld_acquire(cnt) != (unsigned)(a.W + 1)) {
-      if (*abort_flag) {
-        ok = false;
-        break;
+  bool ok = nrows > 0;
+  long long u = ok ? (long long)atomicAdd(claim, 1u) : units;
+  long long pub_b = -1, sc_row = -1;  // the last branch seen published, the row whose scalars are held
+  float lz2 = 0.f, ql = 0.f, g = 0.f;
+  while (ok && u < units) {
+    const long long un = (long long)atomicAdd(claim, 1u);  // the next unit, claimed early
+    const long long row = a.grad_begin + u / kGParts;
+    const long long b = row / a.W;
+    if (b != pub_b) {
+      const unsigned* cnt = a.branch_cnt + b;
+      const long long t0 = clock64();
+      while (ld_acquire(cnt) != (unsigned)(a.W + 1)) {
+        if (*abort_flag) {
+          ok = false;
+          break;
+        }
+        if (clock64() - t0 > kWaitLimitCycles) {
+          *abort_flag = 1;
+          atomicOr(reinterpret_cast<unsigned*>(a.status), SPECOPD_FLAG_TIMEOUT);
+          ok = false;
+          break;
+        }
+        __nanosleep(200);
       }
-      if (clock64() - t0 > kWaitLimitCycles) {
-        *abort_flag = 1;
-        atomicOr(reinterpret_cast<unsigned*>(a.status), SPECOPD_FLAG_TIMEOUT);
-        ok = false;
-        break;
-      }
-      __nanosleep(200);
+      if (!ok) break;
+      pub_b = b;
+      // the bits were stored through the generic proxy; the copies read them
+      // through the async proxy
+      asm volatile("fence.proxy.async.global;" ::: "memory");
     }
-    if (!ok) break;
-    const float lz2 = __ldcg(a.lz2 + row), ql = __ldcg(a.ql + row), g = __ldcg(a.g + row);
-    // the bits were stored through the generic proxy; the copies read them
-    // through the async proxy
-    asm volatile("fence.proxy.async.global;" ::: "memory");
+    if (row != sc_row) {
+      lz2 = __ldcg(a.lz2 + row);
+      ql = __ldcg(a.ql + row);
+      g = __ldcg(a.g + row);
+      sc_row = row;
+    }
     const __nv_bfloat16* zrow = static_cast<const __nv_bfloat16*>(a.draft) + row * a.ld_draft;
     const uint8_t* mrow = a.mbits + row * a.mbits_ld;
-    for (long long e0 = 0; e0 < a.V; e0 += kGUnit, ++k) {
+    const long long s0 = (u % kGParts) * per_unit, s1 = min(per_row, s0 + per_unit);
+    for (long long sidx = s0; sidx < s1; ++sidx, ++k) {
+      const long long e0 = sidx * kGUnit;
       const int st = (int)(k % kGStages);
       if (k >= kGStages && !mbar_wait(&gc->empty[st], (uint32_t)((k / kGStages) - 1) & 1u, abort_flag)) {
         ok = false;
@@ -512,6 +539,8 @@ __device__ void grad_producer(const OverlapArgs& a, GradCtl* gc, uint8_t* gbuf, 
       gc->info[st][0] = lz2;
       gc->info[st][1] = ql;
       gc->info[st][2] = g;
+      gc->row[st] = row;
+      gc->e0[st] = (int)e0;
       const int n = (int)min((long long)kGUnit, a.V - e0);
       const int nbk = n & ~127;  // bulk part: whole 128-logit steps
       uint8_t* dz = gbuf + st * kGStageBytes;
@@ -523,6 +552,16 @@ __device__ void grad_producer(const OverlapArgs& a, GradCtl* gc, uint8_t* gbuf, 
         mbar_arrive(&gc->full[st]);
       }
     }
+    u = un;
+  }
+  // tell the gradient warps there is no more work: a stage tagged row -1
+  if (ok) {
+    const int st = (int)(k % kGStages);
+    if (k < kGStages || mbar_wait(&gc->empty[st], (uint32_t)((k / kGStages) - 1) & 1u, abort_flag)) {
+      gc->row[st] = -1;
+      mbar_arrive(&gc->full[st]);
+      ++k;
+    }
   }
   // every issued copy must land before the CTA may exit
   for (long long j = (k > kGStages ? k - kGStages : 0); j < k; ++j)
@@ -531,51 +570,52 @@ __device__ void grad_producer(const OverlapArgs& a, GradCtl* gc, uint8_t* gbuf, 
 
 __device__ void grad_consumer(const OverlapArgs& a, GradCtl* gc, const uint8_t* gbuf, volatile int* abort_flag, int gw,
                               int lane) {
+  if (a.grad_end <= a.grad_begin) return;
   const float2 l2e = make_float2(kLog2e, kLog2e);
   const uint64_t spol = l2_policy_evict_first();
-  long long k = 0;
-  for (long long row = a.grad_begin + blockIdx.x; row < a.grad_end; row += gridDim.x) {
+  for (long long k = 0;; ++k) {
+    const int st = (int)(k % kGStages);
+    if (!mbar_wait_warp(&gc->full[st], (uint32_t)(k / kGStages) & 1u, abort_flag)) return;
+    const long long row = gc->row[st];
+    if (row < 0) return;
+    const long long e0 = gc->e0[st];
+    const float L2 = gc->info[st][0], Q = gc->info[st][1], G = gc->info[st][2];
     const __nv_bfloat16* zrow = static_cast<const __nv_bfloat16*>(a.draft) + row * a.ld_draft;
     const uint8_t* mrow = a.mbits + row * a.mbits_ld;
     float* grow = a.grad + row * a.ld_grad;
-    for (long long e0 = 0; e0 < a.V; e0 += kGUnit, ++k) {
-      const int st = (int)(k % kGStages);
-      if (!mbar_wait_warp(&gc->full[st], (uint32_t)(k / kGStages) & 1u, abort_flag)) return;
-      const float L2 = gc->info[st][0], Q = gc->info[st][1], G = gc->info[st][2];
-      const bool live = L2 != -INFINITY;
-      const float gg = live ? G : 0.f;
-      const float2 nl = make_float2(live ? -L2 : 0.f, live ? -L2 : 0.f);
-      const float omq = 1.f - Q, zmq = 0.f - Q;  // [q < p] - q_less for bit 1 and bit 0
-      const int n = (int)min((long long)kGUnit, a.V - e0);
-      const int nbk = n & ~127;
-      const uint8_t* sz = gbuf + st * kGStageBytes;
-      const uint8_t* sb = sz + kGUnit * 2;
-      for (int v = gw; v * 128 < nbk; v += kRGradWarps) {
-        const int e = v * 128 + 4 * lane;
-        const uint2 zw = *reinterpret_cast<const uint2*>(sz + 2 * e);
-        const uint32_t bits = (uint32_t)sb[e >> 3] >> ((lane & 1) * 4);
-        const uint32_t z0 = bmax2(zw.x, kNegInf2), z1 = bmax2(zw.y, kNegInf2);  // inactive -> q = 0
-        const float2 x0 = __ffma2_rn(make_float2(bf_lo(z0), bf_hi(z0)), l2e, nl);
-        const float2 x1 = __ffma2_rn(make_float2(bf_lo(z1), bf_hi(z1)), l2e, nl);
-        float4 o;
-        o.x = gg * ex2(x0.x) * ((bits & 1u) ? omq : zmq);
-        o.y = gg * ex2(x0.y) * ((bits & 2u) ? omq : zmq);
-        o.z = gg * ex2(x1.x) * ((bits & 4u) ? omq : zmq);
-        o.w = gg * ex2(x1.y) * ((bits & 8u) ? omq : zmq);
-        st_global_v4_policy(grow + e0 + e, o, spol);
-      }
-      if (gw == 0) {  // fewer than 128 logits at the end of the row: plain loads
-        for (long long e = e0 + nbk + lane; e < e0 + n; e += 32) {
-          const float z = __bfloat162float(zrow[e]);
-          const bool active = live && z == z && fabsf(z) != INFINITY;
-          const float q = active ? ex2(fmaf(z, kLog2e, -L2)) : 0.f;
-          const uint32_t bit = (__ldcg(mrow + (e >> 3)) >> (e & 7)) & 1u;
-          grow[e] = G * q * ((float)bit - Q);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&gc->empty[st]);
+    const bool live = L2 != -INFINITY;
+    const float gg = live ? G : 0.f;
+    const float2 nl = make_float2(live ? -L2 : 0.f, live ? -L2 : 0.f);
+    const float omq = 1.f - Q, zmq = 0.f - Q;  // [q < p] - q_less for bit 1 and bit 0
+    const int n = (int)min((long long)kGUnit, a.V - e0);
+    const int nbk = n & ~127;
+    const uint8_t* sz = gbuf + st * kGStageBytes;
+    const uint8_t* sb = sz + kGUnit * 2;
+    for (int v = gw; v * 128 < nbk; v += kRGradWarps) {
+      const int e = v * 128 + 4 * lane;
+      const uint2 zw = *reinterpret_cast<const uint2*>(sz + 2 * e);
+      const uint32_t bits = (uint32_t)sb[e >> 3] >> ((lane & 1) * 4);
+      const uint32_t z0 = bmax2(zw.x, kNegInf2), z1 = bmax2(zw.y, kNegInf2);  // inactive -> q = 0
+      const float2 x0 = __ffma2_rn(make_float2(bf_lo(z0), bf_hi(z0)), l2e, nl);
+      const float2 x1 = __ffma2_rn(make_float2(bf_lo(z1), bf_hi(z1)), l2e, nl);
+      float4 o;
+      o.x = gg * ex2(x0.x) * ((bits & 1u) ? omq : zmq);
+      o.y = gg * ex2(x0.y) * ((bits & 2u) ? omq : zmq);
+      o.z = gg * ex2(x1.x) * ((bits & 4u) ? omq : zmq);
+      o.w = gg * ex2(x1.y) * ((bits & 8u) ? omq : zmq);
+      st_global_v4_policy(grow + e0 + e, o, spol);
     }
+    if (gw == 0) {  // fewer than 128 logits at the end of the row: plain loads
+      for (long long e = e0 + nbk + lane; e < e0 + n; e += 32) {
+        const float z = __bfloat162float(zrow[e]);
+        const bool active = live && z == z && fabsf(z) != INFINITY;
+        const float q = active ? ex2(fmaf(z, kLog2e, -L2)) : 0.f;
+        const uint32_t bit = (__ldcg(mrow + (e >> 3)) >> (e & 7)) & 1u;
+        grow[e] = G * q * ((float)bit - Q);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&gc->empty[st]);
   }
 }
 
