@@ -52,20 +52,6 @@ struct Elem<float> {
   }
   __device__ static float one(const float* p) { return *p; }
 };
-template <>
-struct Elem<__nv_bfloat16> {
-  __device__ static void load8(const __nv_bfloat16* p, float (&x)[8]) {
-    const uint4 u = *reinterpret_cast<const uint4*>(p);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      x[2 * i] = __uint_as_float(w[i] << 16);
-      x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-  }
-  __device__ static float one(const __nv_bfloat16* p) { return __bfloat162float(*p); }
-};
-
 struct StatSmem {
   float part[8];      // this CTA's partials, read by the cluster
   float bcast[4];
