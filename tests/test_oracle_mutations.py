@@ -172,3 +172,24 @@ def test_lm_head_slips_break_pins():
     bad_q_less = (q * ((log_q <= log_p) & active)).sum(axis=-1)
     good = LM.row_statistics(z, z)["q_less"]
     assert np.all(good == 0.0) and np.all(np.abs(bad_q_less - 1.0) < 1e-12)
+
+
+def test_gdn_decay_outside_the_correction_breaks_the_erase_pin():
+    """S_t = alpha S - beta (S k) k^T + beta v k^T (decay not applied to the
+    correction term) leaves -0.5 v1 k1^T where the true rule erases the key."""
+    from oracle import gdn as G
+    rng = np.random.default_rng(12)
+    k1 = np.linalg.qr(rng.normal(size=(6, 6)))[0][:, 0]
+    v1 = rng.normal(size=4)
+
+    def slipped(k, v, alpha, beta):
+        S = np.zeros((v.shape[1], k.shape[1]))
+        for t in range(k.shape[0]):
+            S = alpha[t] * S - beta[t] * np.outer(S @ k[t], k[t]) + beta[t] * np.outer(v[t], k[t])
+        return S
+    k = np.vstack([k1, k1])
+    v = np.vstack([v1, np.zeros(4)])
+    a, b = np.array([1.0, 0.5]), np.array([1.0, 1.0])
+    _, S = G.gdn_sequence(k, k, v, a, b)
+    assert np.max(np.abs(S)) < 1e-13
+    assert np.max(np.abs(slipped(k, v, a, b))) > 0.1
