@@ -244,6 +244,41 @@ int specopd_tv_overlap_e2e(const void* draft, const void* teacher, specopd_dtype
                            double count, float* alpha, float* loss, float* grad_draft, int64_t ld_grad,
                            void* workspace, size_t workspace_bytes, int32_t* status, specopd_stream_t stream);
 
+/* Bytes of workspace specopd_gdn_tree needs: the fp32 trunk checkpoints,
+ * (sum over trees of T / 64) * H * 128 * 128 * 4 rounded up to 256 (0 for an
+ * invalid description). */
+size_t specopd_gdn_workspace_bytes(const specopd_tree_desc* desc, int H);
+
+/*
+ * specopd_gdn_tree -- Gated DeltaNet linear attention over a proposal tree,
+ * every packed row reading the recurrent state of its own history, with
+ * indexed state replay.
+ *
+ * SpecOPD (thelatestinai.com listing), Fig 5: a shared trunk pass caches an
+ * fp32 GDN state at every C = 64 boundary; each branch copies the checkpoint
+ * at or before its anchor, replays the trunk features up to the anchor, then
+ * updates the state over its own tokens and reads it with each token's query;
+ * checkpoints stay immutable.  Reading (the pages print no formula): the
+ * gated delta rule per head, state S in R^{dv x dk} starting at zero,
+ *   S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *   o_t = S_t q_t.
+ * A branch's history is the trunk through its anchor, then its own earlier
+ * tokens (the packing of specopd_build_tree_mask for the same description).
+ *
+ * q, k, v [N, H, 128] bf16 (dk = dv = 128; k normalised upstream), alpha,
+ * beta [N, H] fp32, out [N, H, 128] fp32: device, row-major, 16-byte aligned.
+ * The features are consumed as given (projections, short convolution and
+ * normalisation happen upstream).  workspace: device, >=
+ * specopd_gdn_workspace_bytes, 256-byte aligned; it holds the checkpoints
+ * after the call.  Anchors outside [P, T-1] set SPECOPD_FLAG_ANCHOR and are
+ * clamped.  Returns SPECOPD_ERR_SHAPE for dk or dv other than 128 or N not
+ * the packed row count, SPECOPD_ERR_ARG / _ALIGN / _WORKSPACE before anything
+ * is enqueued, SPECOPD_ERR_CUDA if a launch fails.
+ */
+int specopd_gdn_tree(const specopd_tree_desc* desc, const void* q, const void* k, const void* v,
+                     const float* alpha, const float* beta, float* out, int64_t N, int H, int dk, int dv,
+                     void* workspace, size_t workspace_bytes, int32_t* status, specopd_stream_t stream);
+
 /* Bytes of workspace specopd_lm_head_overlap needs (0 for invalid sizes). */
 size_t specopd_lm_head_workspace_bytes(int64_t rows, int64_t V);
 

@@ -326,3 +326,57 @@ def make_lm_head_case(name: str, num_branches: int, W: int, V: int, Hd: int, Ht:
         wt_b[c * _ROW_CHUNK:c * _ROW_CHUNK + t.shape[0]] = t
     hd_b = bf16_round(ht) if Hd == Ht else bf16_round(_normal_rows(seed, _TID_H_DRAFT, 0, rows, Hd, 1.0))
     return LmHeadCase(name, num_branches, W, V, Hd, Ht, hd_b, wd_b, bf16_round(ht), wt_b)
+
+
+# ---------------------------------------------------------------------------
+# Gated DeltaNet features per packed row (consumed as given by the GDN path)
+# ---------------------------------------------------------------------------
+
+_TID_GDN_Q, _TID_GDN_K, _TID_GDN_V, _TID_GDN_A, _TID_GDN_B = range(110, 115)
+
+
+@dataclasses.dataclass
+class GdnCase:
+    name: str
+    trunk_len: List[int]
+    prompt_len: List[int]
+    num_branches: List[int]
+    W: int
+    H: int
+    pack_terminal: bool
+    anchors: np.ndarray   # int32 [sum B], zero-based within each tree
+    q: np.ndarray         # [N, H, 128] bf16 bits
+    k: np.ndarray         # [N, H, 128] bf16 bits, rows of unit norm before rounding
+    v: np.ndarray         # [N, H, 128] bf16 bits
+    alpha: np.ndarray     # [N, H] fp32 in [0.9, 1)
+    beta: np.ndarray      # [N, H] fp32 in [0.1, 0.9)
+
+    @property
+    def num_rows(self) -> int:
+        return self.q.shape[0]
+
+
+def make_gdn_case(name: str, trees: Sequence[Tuple[int, int, int]], W: int, H: int, seed: int = 0,
+                  pack_terminal: bool = True, anchors: Sequence[Sequence[int]] = None) -> GdnCase:
+    """Per packed row and head: q ~ N(0, 1/128), k = a N(0, I) draw scaled to
+    unit norm, v ~ N(0, 1) (all rounded to bf16 once), decay alpha ~ U[0.9, 1)
+    and write strength beta ~ U[0.1, 0.9) in fp32.  Anchors as for the
+    attention workloads unless given per tree."""
+    d = 128
+    rpb = W if pack_terminal else W - 1
+    N = int(sum(T + B * rpb for T, _, B in trees))
+    anc = []
+    for t, (T, P, B) in enumerate(trees):
+        anc.append(np.asarray(anchors[t], dtype=np.int32) if anchors is not None
+                   else _draw_anchors(seed, t, P, T, B, True, False))
+    q = _normal_rows(seed, _TID_GDN_Q, 0, N, H * d, 1.0 / np.sqrt(d)).reshape(N, H, d)
+    k = _normal_rows(seed, _TID_GDN_K, 0, N, H * d, 1.0).reshape(N, H, d)
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = _normal_rows(seed, _TID_GDN_V, 0, N, H * d, 1.0).reshape(N, H, d)
+    rng_a = np.random.default_rng([seed, _TID_GDN_A, 0, 0])
+    rng_b = np.random.default_rng([seed, _TID_GDN_B, 0, 0])
+    alpha = rng_a.uniform(0.9, 1.0, size=(N, H)).astype(np.float32)
+    beta = rng_b.uniform(0.1, 0.9, size=(N, H)).astype(np.float32)
+    return GdnCase(name, [t[0] for t in trees], [t[1] for t in trees], [t[2] for t in trees], W, H, pack_terminal,
+                   np.concatenate(anc) if anc else np.zeros(0, np.int32), bf16_round(q), bf16_round(k),
+                   bf16_round(v), alpha, beta)

@@ -294,6 +294,39 @@ int specopd_tv_overlap_e2e(const void* draft, const void* teacher, specopd_dtype
   return SPECOPD_OK;
 }
 
+size_t specopd_gdn_workspace_bytes(const specopd_tree_desc* desc, int H) {
+  TreeParams p;
+  if (tree_params(desc, &p) != SPECOPD_OK || H < 1) return 0;
+  return align_up(gdn_checkpoint_floats(p, H) * sizeof(float));
+}
+
+int specopd_gdn_tree(const specopd_tree_desc* desc, const void* q, const void* k, const void* v,
+                     const float* alpha, const float* beta, float* out, int64_t N, int H, int dk, int dv,
+                     void* workspace, size_t workspace_bytes, int32_t* status, specopd_stream_t stream) {
+  GdnArgs g;
+  const int s = tree_params(desc, &g.tp);
+  if (s != SPECOPD_OK) return s;
+  if (dk != 128 || dv != 128 || H < 1 || H > 1024) return SPECOPD_ERR_SHAPE;
+  if (N != (int64_t)g.tp.row_base[g.tp.num_trees]) return SPECOPD_ERR_SHAPE;
+  if (!q || !k || !v || !alpha || !beta || !out || !status) return SPECOPD_ERR_ARG;
+  if (g.tp.total_branches > 0 && !desc->anchors) return SPECOPD_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(out)) return SPECOPD_ERR_ALIGN;
+  const size_t need = align_up(gdn_checkpoint_floats(g.tp, H) * sizeof(float));
+  if (need > 0 && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) % kAlign)))
+    return SPECOPD_ERR_WORKSPACE;
+  g.q = q;
+  g.k = k;
+  g.v = v;
+  g.alpha = alpha;
+  g.beta = beta;
+  g.out = out;
+  g.H = H;
+  g.anchors = desc->anchors;
+  g.ckpt = static_cast<float*>(workspace);
+  g.status = status;
+  return cuda_status(launch_gdn_tree(g, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t specopd_lm_head_workspace_bytes(int64_t rows, int64_t V) {
   if (rows < 0 || V < 1) return 0;
   return lm_head_layout(rows, V).total;

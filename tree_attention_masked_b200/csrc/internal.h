@@ -92,6 +92,24 @@ cudaError_t launch_tv_grad(const OverlapArgs& a, specopd_dtype dtype, cudaStream
 cudaError_t launch_e2e_loss(const float* alpha, int64_t num_branches, int W, double inv_count, float* loss,
                             float* grad_alpha, cudaStream_t stream);
 
+// Gated DeltaNet over a proposal tree with indexed state replay (gdn.cu).
+struct GdnArgs {
+  const void* q;        // [N, H, 128] bf16
+  const void* k;        // [N, H, 128] bf16
+  const void* v;        // [N, H, 128] bf16
+  const float* alpha;   // [N, H]
+  const float* beta;    // [N, H]
+  float* out;           // [N, H, 128] fp32
+  int H;
+  const int32_t* anchors;  // device [total branches], zero-based within the tree
+  float* ckpt;             // [sum_t T_t / 64][H][128][128] fp32 checkpoints
+  int32_t* status;
+  TreeParams tp;
+  int32_t ck_off[SPECOPD_MAX_TREES];  // first checkpoint of each tree (set by the launcher)
+};
+size_t gdn_checkpoint_floats(const TreeParams& tp, int H);
+cudaError_t launch_gdn_tree(GdnArgs g, cudaStream_t stream);
+
 // Overlap statistics from hidden states and LM heads (lm_head_sm100.cu).
 struct LmHeadArgs {
   const void* h_draft;    // [rows, Hd] bf16

@@ -71,6 +71,9 @@ _c = {
                                    _int, _f64, _vp, _vp, _vp, _i64, _vp, _sz, _vp, _vp),
     "specopd_tv_overlap_e2e_static": _sig("specopd_tv_overlap_e2e_static", _int, _vp, _vp, _int, _i64, _i64,
                                           _i64, _i64, _i64, _int, _f64, _vp, _vp, _vp, _i64, _vp, _vp),
+    "specopd_gdn_workspace_bytes": _sig("specopd_gdn_workspace_bytes", _sz, _desc_p, _int),
+    "specopd_gdn_tree": _sig("specopd_gdn_tree", _int, _desc_p, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _int, _int,
+                             _int, _vp, _sz, _vp, _vp),
     "specopd_lm_head_workspace_bytes": _sig("specopd_lm_head_workspace_bytes", _sz, _i64, _i64),
     "specopd_lm_head_overlap": _sig("specopd_lm_head_overlap", _int, _vp, _vp, _int, _vp, _vp, _int, _i64, _i64,
                                     _i64, _int, _f64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp, _vp),
@@ -239,3 +242,17 @@ def specopd_lm_head_overlap(h_draft, head_draft, h_teacher, head_teacher, num_br
         h_draft.shape[0], head_draft.shape[0], num_branches, W, count, _ptr(alpha), _ptr(q_less), _ptr(lse_draft),
         _ptr(lse_teacher), _ptr(loss), _ptr(grad_alpha), _ptr(grad), grad.stride(0) if grad is not None else 0,
         _ptr(workspace), wb, _ptr(status), _stream(stream)))
+
+
+def specopd_gdn_workspace_bytes(trees: Trees, H: int) -> int:
+    return _c["specopd_gdn_workspace_bytes"](trees.ref(), H)
+
+
+def specopd_gdn_tree(trees: Trees, q, k, v, alpha, beta, out, workspace, status, stream=None) -> None:
+    """Gated DeltaNet over the packed tree: q, k, v [N, H, 128] bf16, alpha,
+    beta [N, H] fp32, out [N, H, 128] fp32 (all contiguous)."""
+    _contig(q, k, v, alpha, beta, out)
+    wb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("specopd_gdn_tree", _c["specopd_gdn_tree"](
+        trees.ref(), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(out), q.shape[0], q.shape[1],
+        q.shape[2], v.shape[2], _ptr(workspace), wb, _ptr(status), _stream(stream)))
