@@ -340,6 +340,7 @@ def run_gpu(args):
         del st
         torch.cuda.empty_cache()
         out["kernels"]["lm_head_overlap"] = lm_head_measure(dev, peaks, args.seed, args.lm_head_vocab)
+        out["kernels"]["gdn_tree"] = gdn_measure(dev, peaks, args.seed)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -429,6 +430,50 @@ def lm_head_measure(dev, peaks, seed: int, V: int = 151936) -> dict:
             "launches": 5}
 
 
+def gdn_measure(dev, peaks, seed: int, H: int = 32) -> dict:
+    """The GDN linear-attention path timed on its own (not part of the step):
+    gated delta rule over the 8B-style tree (T 4,096, 64 branches x W 16,
+    5,120 packed rows) with H heads of d_k = d_v = 128.  Work counts the
+    recurrence's multiply-adds (3 d_k d_v per token and head) over the trunk
+    pass, the replays from the C = 64 checkpoints and the branch tokens.  The
+    recurrence is sequential along the trunk, so the bound is the latency of one
+    step times the trunk length, not a throughput peak."""
+    import torch
+    import synthetic as SY
+    from tree_attention_masked_b200 import specopd as S
+    T, P, B, W = 4096, 1024, 64, 16
+    case = SY.make_gdn_case("gqa8b-gdn", [(T, P, B)], W=W, H=H, seed=seed)
+    bf = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    anchors = torch.from_numpy(case.anchors).to(dev)
+    trees = S.Trees(case.trunk_len, case.prompt_len, case.num_branches, W, anchors, True)
+    q, k, v = bf(case.q), bf(case.k), bf(case.v)
+    alpha, beta = torch.from_numpy(case.alpha).to(dev), torch.from_numpy(case.beta).to(dev)
+    out = torch.empty(case.num_rows, H, 128, device=dev)
+    ws = torch.empty(S.specopd_gdn_workspace_bytes(trees, H), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    call = lambda: S.specopd_gdn_tree(trees, q, k, v, alpha, beta, out, ws, status, stream=stream)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    n = 10
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    replay = int(sum((int(a) + 1) % 64 for a in case.anchors))
+    tokens = T + replay + B * W
+    flops = 2.0 * 3 * 128 * 128 * H * tokens
+    return {"bound": "latency (sequential along the trunk)", "ms": ms, "achieved": flops / (ms * 1e-3) / 1e12,
+            "unit": "TFLOP/s", "flops": flops, "trunk_tokens": T, "replayed_tokens": replay,
+            "branch_tokens": B * W, "us_per_trunk_step": ms * 1e3 / T, "device_status": status.item(),
+            "shape": f"T {T}, B {B} x W {W}, {H} heads, d_k = d_v = 128, bf16 features, fp32 state",
+            "launches": 2}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -442,11 +487,19 @@ def main():
     ap.add_argument("--lm-head-only", action="store_true",
                     help="time only the LM-head path (one JSON line; for profiling it alone)")
     ap.add_argument("--lm-head-vocab", type=int, default=151936, help="vocabulary of the LM-head path")
+    ap.add_argument("--gdn-only", action="store_true", help="time only the GDN path (one JSON line)")
     args = ap.parse_args()
     # at least three untimed warm-up steps, whatever was asked for
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
         run_reference(args)
+    elif args.gdn_only:
+        import torch
+        from tree_attention_masked_b200.build import build
+        build()
+        d = gdn_measure(torch.device("cuda", 0), load_peaks(), args.seed)
+        print(json.dumps({"metric": "GDN over the proposal tree (indexed state replay)", "value": d["ms"],
+                          "unit": "ms", "higher_is_better": False, "kernel": d}), flush=True)
     elif args.lm_head_only:
         import torch
         from tree_attention_masked_b200.build import build

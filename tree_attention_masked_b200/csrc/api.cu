@@ -310,7 +310,9 @@ int specopd_gdn_tree(const specopd_tree_desc* desc, const void* q, const void* k
   if (N != (int64_t)g.tp.row_base[g.tp.num_trees]) return SPECOPD_ERR_SHAPE;
   if (!q || !k || !v || !alpha || !beta || !out || !status) return SPECOPD_ERR_ARG;
   if (g.tp.total_branches > 0 && !desc->anchors) return SPECOPD_ERR_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(out)) return SPECOPD_ERR_ALIGN;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (reinterpret_cast<uintptr_t>(alpha) & 3) ||
+      (reinterpret_cast<uintptr_t>(beta) & 3))
+    return SPECOPD_ERR_ALIGN;
   const size_t need = align_up(gdn_checkpoint_floats(g.tp, H) * sizeof(float));
   if (need > 0 && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) % kAlign)))
     return SPECOPD_ERR_WORKSPACE;
