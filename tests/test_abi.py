@@ -122,6 +122,23 @@ def test_argument_errors_before_launch(S):
     assert S._c["specopd_status_string"](-5) == b"workspace missing, too small or misaligned"
 
 
+def test_gdn_argument_errors_before_launch(S):
+    import torch
+    trees = S.Trees([200], [10], [4], 4, torch.zeros(4, dtype=torch.int32))
+    N = S.specopd_tree_packed_rows(trees)
+    need = S.specopd_gdn_workspace_bytes(trees, 2)
+    assert need == 3 * 2 * 128 * 128 * 4    # checkpoints after tokens 63, 127, 191
+    g = S._c["specopd_gdn_tree"]
+    args = lambda **kw: [trees.ref(), kw.get("q", 16), 16, 16, 16, 16, 16, kw.get("N", N), 2, kw.get("dk", 128),
+                         kw.get("dv", 128), 256, kw.get("ws", need), 16, None]
+    assert g(*args(dk=64)) == -2            # only d_k = d_v = 128
+    assert g(*args(dv=96)) == -2
+    assert g(*args(N=N - 1)) == -2          # N must be the packed row count
+    assert g(*args(q=24)) == -6             # 16-byte alignment
+    assert g(*args(ws=need - 1)) == -5      # the checkpoints must fit
+    assert g(*args(q=0)) == -1              # null input
+
+
 def test_workspace_sizes(S):
     n_tiles = (151936 + 255) // 256
     assert S.specopd_lm_head_workspace_bytes(1024, 151936) >= n_tiles * 1024 * 24 + 3 * 1024 * 4
