@@ -8,7 +8,7 @@ common module is ``synthetic``, which draws inputs and holds none of the
 method's arithmetic.
 
 Source: "SpecOPD: Branch-Parallel On-Policy Distillation for Speculative
-Decoding" as listed on thelatestinai.com (Fig 2, Fig 3, Fig 5, Algorithm 1) and the
+Decoding" as listed on thelatestinai.com (Fig 2, Fig 3, Fig 4, Fig 5, Algorithm 1) and the
 daiwk.github.io write-up of it (section "Equations", section "Inputs and code
 mapping", section "Checks, negative controls, and limits").
 
@@ -23,8 +23,10 @@ Modules:
                 overlap statistics taken from them
   gdn        -- gated delta rule (GDN linear attention) over a proposal tree,
                 every row reading the state of its own history
+  sparse     -- sparse attention with branch-consistent indexer groups: top-k
+                complete groups per row plus the causal tail
 
 Every function is plain fp64 NumPy written from the definitions; nothing is
 blocked, fused or reordered.
 """
-from . import tree, attention, overlap, lm_head, gdn  # noqa: F401
+from . import tree, attention, overlap, lm_head, gdn, sparse  # noqa: F401

@@ -193,3 +193,32 @@ def test_gdn_decay_outside_the_correction_breaks_the_erase_pin():
     _, S = G.gdn_sequence(k, k, v, a, b)
     assert np.max(np.abs(S)) < 1e-13
     assert np.max(np.abs(slipped(k, v, a, b))) > 0.1
+
+
+def test_sparse_boundary_group_keyed_by_trunk_only_breaks_the_branch_pin():
+    """Keying the group that a branch token completes by its trunk members only
+    (not branch-specific) makes both branches pick the same group, which the
+    branch-specific pin rules out."""
+    from oracle import sparse as SP
+    from oracle import tree as T
+
+    def slipped(pt, r, qi, ki, g, topk, kvh):
+        hist = SP.history(pt, r)
+        n = (len(hist)) // g
+        keys = []
+        for m in range(n):
+            members = [c for c in hist[m * g:(m + 1) * g] if pt.parent is not None and c < 12]  # trunk rows only
+            keys.append(np.mean(ki[members, kvh], axis=0))
+        scores = np.stack(keys) @ qi[r, kvh]
+        best = sorted(range(n), key=lambda m: (-scores[m], m))[:topk]
+        return [c for m in sorted(best) for c in hist[m * g:(m + 1) * g]]
+    pt = T.pack([12], [0], [2], [6, 6], 2, True)
+    qi = np.zeros((pt.num_rows, 1, 2))
+    ki = np.zeros((pt.num_rows, 1, 2))
+    qi[12, 0] = qi[14, 0] = [1.0, 0.0]
+    ki[12, 0], ki[14, 0] = [10.0, 0.0], [-10.0, 0.0]
+    ki[0:4, 0] = [0.5, 0.0]
+    good = (SP.selected_columns(pt, 12, qi, ki, 4, 1, 0), SP.selected_columns(pt, 14, qi, ki, 4, 1, 0))
+    bad = (slipped(pt, 12, qi, ki, 4, 1, 0), slipped(pt, 14, qi, ki, 4, 1, 0))
+    assert good[0] != good[1]
+    assert bad[0][:4] == bad[1][:4] == [0, 1, 2, 3]   # both branches fall back to the trunk group
