@@ -341,6 +341,10 @@ def run_gpu(args):
         torch.cuda.empty_cache()
         out["kernels"]["lm_head_overlap"] = lm_head_measure(dev, peaks, args.seed, args.lm_head_vocab)
         out["kernels"]["gdn_tree"] = gdn_measure(dev, peaks, args.seed)
+        try:  # a secondary measurement: an error is recorded, not raised
+            out["kernels"]["sparse_tree_attention"] = sparse_measure(dev, peaks, args.seed)
+        except Exception as exc:  # noqa: BLE001
+            out["kernels"]["sparse_tree_attention"] = {"error": f"{type(exc).__name__}: {exc}"}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -474,6 +478,62 @@ def gdn_measure(dev, peaks, seed: int, H: int = 32) -> dict:
             "launches": 2}
 
 
+def sparse_measure(dev, peaks, seed: int) -> dict:
+    """Sparse attention with branch-consistent indexer groups timed on its own
+    (not part of the step), on the shape of the GPU parity test's full-size
+    case: the 8B-style tree (T 4,096, 64 branches x W 16), 32/8 heads, d 128,
+    64-token groups, top-8, 64-wide indexer features.  Useful FLOPs count the
+    attended (row, column) pairs, 4 d per pair and query head."""
+    import torch
+    import synthetic as SY
+    from tree_attention_masked_b200 import specopd as S
+    g, topk, W = 64, 8, 16
+    case = SY.make_sparse_case("gqa8b-sparse", [(4096, 1024, 64)], W, 32, 8, 64, seed=seed)
+    bf = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    anchors = torch.from_numpy(case.anchors).to(dev)
+    trees = S.Trees(case.trunk_len, case.prompt_len, case.num_branches, W, anchors, True)
+    N = case.num_rows
+    i32 = dict(dtype=torch.int32, device=dev)
+    pos, trunk_limit, branch_of = (torch.empty(N, **i32) for _ in range(3))
+    anc_bits = torch.empty(N, dtype=torch.int64, device=dev)
+    pred_rows = torch.empty(max(int(sum(case.num_branches)) * W, 1), **i32)
+    cu_rows = torch.empty(2, **i32)
+    tile_meta = torch.empty(max(S.specopd_tree_num_tiles(trees), 1), 8, **i32)
+    status = torch.zeros(1, **i32)
+    S.specopd_build_tree_mask(trees, pos, trunk_limit, branch_of, anc_bits, pred_rows, cu_rows, tile_meta, status)
+    q, k, v, qi, ki = bf(case.q), bf(case.k), bf(case.v), bf(case.qi), bf(case.ki)
+    out = torch.empty(N, 32, 128, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(S.specopd_sparse_workspace_bytes(trees, 32, 8, 64, g), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    call = lambda: S.specopd_sparse_tree_attention(trees, q, k, v, qi, ki, out, pos, g, topk, 1e4, ws, status,
+                                                   stream=stream)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    n = 10
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    # attended pairs: per row, its chosen groups' members and its tail
+    T0, P0, B0 = 4096, 1024, 64
+    pairs = 0
+    for r in range(N):
+        p = r if r < T0 else int(case.anchors[(r - T0) // W]) + 1 + (r - T0) % W
+        nc = (p + 1) // g
+        pairs += min(nc, topk) * g + (p + 1 - nc * g)
+    flops = 4.0 * 128 * 32 * pairs
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"bound": "latency (SIMT: one warp per row and KV head)", "ms": ms, "achieved": achieved,
+            "unit": "TFLOP/s", "peak": peaks["bf16"], "frac": achieved / peaks["bf16"], "useful_flops": flops,
+            "attended_pairs": pairs, "device_status": status.item(),
+            "shape": "T 4096, B 64 x W 16, 32/8 heads, d 128, groups of 64, top-8, indexer width 64, bf16",
+            "launches": 3}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -488,11 +548,19 @@ def main():
                     help="time only the LM-head path (one JSON line; for profiling it alone)")
     ap.add_argument("--lm-head-vocab", type=int, default=151936, help="vocabulary of the LM-head path")
     ap.add_argument("--gdn-only", action="store_true", help="time only the GDN path (one JSON line)")
+    ap.add_argument("--sparse-only", action="store_true", help="time only the sparse indexer-group attention")
     args = ap.parse_args()
     # at least three untimed warm-up steps, whatever was asked for
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
         run_reference(args)
+    elif args.sparse_only:
+        import torch
+        from tree_attention_masked_b200.build import build
+        build()
+        d = sparse_measure(torch.device("cuda", 0), load_peaks(), args.seed)
+        print(json.dumps({"metric": "sparse attention with indexer groups over the proposal tree", "value": d["ms"],
+                          "unit": "ms", "higher_is_better": False, "kernel": d}), flush=True)
     elif args.gdn_only:
         import torch
         from tree_attention_masked_b200.build import build

@@ -279,6 +279,42 @@ int specopd_gdn_tree(const specopd_tree_desc* desc, const void* q, const void* k
                      const float* alpha, const float* beta, float* out, int64_t N, int H, int dk, int dv,
                      void* workspace, size_t workspace_bytes, int32_t* status, specopd_stream_t stream);
 
+/* Bytes of workspace specopd_sparse_tree_attention needs: rotated Q and K
+ * (bf16) and the trunk group keys (fp32), each rounded up to 256 bytes. */
+size_t specopd_sparse_workspace_bytes(const specopd_tree_desc* desc, int Hq, int Hkv, int di, int g);
+
+/*
+ * specopd_sparse_tree_attention -- sparse attention with branch-consistent
+ * indexer groups over a proposal tree.
+ *
+ * SpecOPD (thelatestinai.com listing), Fig 4: rows reuse complete trunk group
+ * keys; an incomplete boundary group stays in the causal tail; a group
+ * completed by branch tokens gets a branch-specific indexer key; indexer
+ * queries select complete groups with top-k; attention reads the selected
+ * groups plus the causal tail, which bypasses top-k.  Readings (the figure
+ * prints no formula): groups are g consecutive semantic positions of the
+ * row's own history (trunk through the anchor, then its branch); a complete
+ * group's key is the mean of its members' indexer keys; the score is the
+ * indexer query dotted with it, taken in fp32 in a fixed order (sequential
+ * sums, fused multiply-adds); the k best per KV head, ties to the earlier
+ * group; attention as specopd_tree_attention (rotate-half RoPE at `pos`,
+ * scale softmax_scale or 1/sqrt(d) when <= 0) over the chosen members and the
+ * tail, fp32 online softmax.
+ *
+ * q [N, Hq, 128], k, v [N, Hkv, 128], qi, ki [N, Hkv, di] (di <= 256), out
+ * [N, Hq, 128]: device bf16, row-major, 16-byte aligned; pos [N] from
+ * specopd_build_tree_mask for the same description.  1 <= topk <= 64; a
+ * tree's trunk plus one branch must hold at most 1,024 complete groups.
+ * workspace >= specopd_sparse_workspace_bytes, 256-byte aligned.  Returns
+ * SPECOPD_ERR_SHAPE / _ARG / _ALIGN / _WORKSPACE before anything is
+ * enqueued, SPECOPD_ERR_CUDA if a launch fails.
+ */
+int specopd_sparse_tree_attention(const specopd_tree_desc* desc, const void* q, const void* k, const void* v,
+                                  const void* qi, const void* ki, void* out, int64_t N, int Hq, int Hkv, int d,
+                                  int di, int g, int topk, float rope_theta, float softmax_scale, const int32_t* pos,
+                                  void* workspace, size_t workspace_bytes, int32_t* status,
+                                  specopd_stream_t stream);
+
 /* Bytes of workspace specopd_lm_head_overlap needs (0 for invalid sizes). */
 size_t specopd_lm_head_workspace_bytes(int64_t rows, int64_t V);
 

@@ -380,3 +380,48 @@ def make_gdn_case(name: str, trees: Sequence[Tuple[int, int, int]], W: int, H: i
     return GdnCase(name, [t[0] for t in trees], [t[1] for t in trees], [t[2] for t in trees], W, H, pack_terminal,
                    np.concatenate(anc) if anc else np.zeros(0, np.int32), bf16_round(q), bf16_round(k),
                    bf16_round(v), alpha, beta)
+
+
+# ---------------------------------------------------------------------------
+# Sparse attention with indexer groups: attention and indexer features per row
+# ---------------------------------------------------------------------------
+
+_TID_SP_Q, _TID_SP_K, _TID_SP_V, _TID_SP_QI, _TID_SP_KI = range(120, 125)
+
+
+@dataclasses.dataclass
+class SparseCase:
+    name: str
+    trunk_len: List[int]
+    prompt_len: List[int]
+    num_branches: List[int]
+    W: int
+    Hq: int
+    Hkv: int
+    di: int
+    pack_terminal: bool
+    anchors: np.ndarray   # int32 [sum B]
+    q: np.ndarray         # [N, Hq, 128] bf16 bits
+    k: np.ndarray         # [N, Hkv, 128]
+    v: np.ndarray         # [N, Hkv, 128]
+    qi: np.ndarray        # [N, Hkv, di] indexer queries
+    ki: np.ndarray        # [N, Hkv, di] indexer keys
+
+    @property
+    def num_rows(self) -> int:
+        return self.q.shape[0]
+
+
+def make_sparse_case(name: str, trees: Sequence[Tuple[int, int, int]], W: int, Hq: int, Hkv: int, di: int,
+                     seed: int = 0, pack_terminal: bool = True) -> SparseCase:
+    """Attention features q, k, v ~ N(0, 1) and indexer features qi, ki ~ N(0, 1),
+    drawn in fp32 and rounded to bf16 once; anchors as for the attention workloads."""
+    d = 128
+    rpb = W if pack_terminal else W - 1
+    N = int(sum(T + B * rpb for T, _, B in trees))
+    anc = [_draw_anchors(seed, t, P, T, B, True, False) for t, (T, P, B) in enumerate(trees)]
+    f = lambda tid, heads, width: bf16_round(_normal_rows(seed, tid, 0, N, heads * width, 1.0)).reshape(N, heads, width)
+    return SparseCase(name, [t[0] for t in trees], [t[1] for t in trees], [t[2] for t in trees], W, Hq, Hkv, di,
+                      pack_terminal, np.concatenate(anc) if anc else np.zeros(0, np.int32),
+                      f(_TID_SP_Q, Hq, d), f(_TID_SP_K, Hkv, d), f(_TID_SP_V, Hkv, d), f(_TID_SP_QI, Hkv, di),
+                      f(_TID_SP_KI, Hkv, di))

@@ -101,3 +101,12 @@ def test_tail_bypasses_top_k():
         tail = list(range((r + 1) // 3 * 3, r + 1))
         assert cols[len(cols) - len(tail):] == tail
         assert r in cols or (r + 1) % 3 == 0
+
+
+def test_fp32_decision_agrees_with_fp64_away_from_ties():
+    """Taking the scores in fp32 changes no selection unless two scores are
+    within fp32 rounding of each other (random features: none here)."""
+    pt = T.pack([40], [5], [3], [10, 25, 39], 4, True)
+    q, k, v, qi, ki = _inputs(pt.num_rows, 2, 1, 8, 16, 7)
+    for r in range(pt.num_rows):
+        assert SP.selected_columns(pt, r, qi, ki, 4, 2, 0) == SP.selected_columns(pt, r, qi, ki, 4, 2, 0, True)

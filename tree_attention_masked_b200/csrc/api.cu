@@ -329,6 +329,65 @@ int specopd_gdn_tree(const specopd_tree_desc* desc, const void* q, const void* k
   return cuda_status(launch_gdn_tree(g, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+static size_t sparse_ws(const TreeParams& p, int Hq, int Hkv, int di, int g, size_t* off_rk, size_t* off_gk) {
+  const int64_t N = p.row_base[p.num_trees];
+  *off_rk = align_up((size_t)N * Hq * 128 * 2);
+  *off_gk = *off_rk + align_up((size_t)N * Hkv * 128 * 2);
+  return *off_gk + align_up(sparse_group_keys(p, g) * Hkv * di * sizeof(float));
+}
+
+size_t specopd_sparse_workspace_bytes(const specopd_tree_desc* desc, int Hq, int Hkv, int di, int g) {
+  TreeParams p;
+  if (tree_params(desc, &p) != SPECOPD_OK || Hq < 1 || Hkv < 1 || di < 1 || g < 1) return 0;
+  size_t a, b;
+  return sparse_ws(p, Hq, Hkv, di, g, &a, &b);
+}
+
+int specopd_sparse_tree_attention(const specopd_tree_desc* desc, const void* q, const void* k, const void* v,
+                                  const void* qi, const void* ki, void* out, int64_t N, int Hq, int Hkv, int d,
+                                  int di, int g, int topk, float rope_theta, float softmax_scale, const int32_t* pos,
+                                  void* workspace, size_t workspace_bytes, int32_t* status,
+                                  specopd_stream_t stream) {
+  SparseArgs a;
+  const int st = tree_params(desc, &a.tp);
+  if (st != SPECOPD_OK) return st;
+  if (d != 128 || Hq < 1 || Hkv < 1 || Hq % Hkv || di < 1 || di > 256 || g < 1 || topk < 1 ||
+      topk > kSpMaxTopk)
+    return SPECOPD_ERR_SHAPE;
+  if (N != (int64_t)a.tp.row_base[a.tp.num_trees]) return SPECOPD_ERR_SHAPE;
+  for (int t = 0; t < a.tp.num_trees; ++t)  // every row's complete groups must fit the score buffer
+    if ((a.tp.trunk_len[t] + a.tp.rows_per_branch) / g > kSpMaxGroups) return SPECOPD_ERR_SHAPE;
+  if (!q || !k || !v || !qi || !ki || !out || !pos || !status) return SPECOPD_ERR_ARG;
+  if (a.tp.total_branches > 0 && !desc->anchors) return SPECOPD_ERR_ARG;
+  if (!(rope_theta > 0.f) || !std::isfinite(rope_theta)) return SPECOPD_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SPECOPD_ERR_ALIGN;
+  size_t off_rk, off_gk;
+  const size_t need = sparse_ws(a.tp, Hq, Hkv, di, g, &off_rk, &off_gk);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) % kAlign))
+    return SPECOPD_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.qi = qi;
+  a.ki = ki;
+  a.out = out;
+  a.rq = ws;
+  a.rk = ws + off_rk;
+  a.gkey = reinterpret_cast<float*>(ws + off_gk);
+  a.N = N;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.di = di;
+  a.g = g;
+  a.topk = topk;
+  a.theta = rope_theta;
+  a.scale_log2 = (softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(128.f)) * 1.4426950408889634f;
+  a.pos = pos;
+  a.anchors = desc->anchors;
+  return cuda_status(launch_sparse_attention(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t specopd_lm_head_workspace_bytes(int64_t rows, int64_t V) {
   if (rows < 0 || V < 1) return 0;
   return lm_head_layout(rows, V).total;

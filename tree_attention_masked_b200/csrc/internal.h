@@ -110,6 +110,30 @@ struct GdnArgs {
 size_t gdn_checkpoint_floats(const TreeParams& tp, int H);
 cudaError_t launch_gdn_tree(GdnArgs g, cudaStream_t stream);
 
+// Sparse attention with branch-consistent indexer groups (sparse_attn.cu).
+constexpr int kSpMaxGroups = 1024;  // complete groups a row may score
+constexpr int kSpMaxTopk = 64;
+struct SparseArgs {
+  const void* q;        // [N, Hq, 128] bf16
+  const void* k;        // [N, Hkv, 128] bf16
+  const void* v;        // [N, Hkv, 128] bf16
+  const void* qi;       // [N, Hkv, di] bf16 indexer queries
+  const void* ki;       // [N, Hkv, di] bf16 indexer keys
+  void* out;            // [N, Hq, 128] bf16
+  void* rq;             // workspace: rotated q
+  void* rk;             // workspace: rotated k
+  float* gkey;          // workspace: [trunk groups][Hkv][di] fp32
+  int64_t N;
+  int Hq, Hkv, di, g, topk;
+  float theta, scale_log2;
+  const int32_t* pos;      // [N] semantic positions (specopd_build_tree_mask)
+  const int32_t* anchors;  // [total branches]
+  TreeParams tp;
+  int32_t gk_off[SPECOPD_MAX_TREES + 1];  // first trunk group of each tree (set by the launcher)
+};
+size_t sparse_group_keys(const TreeParams& tp, int g);
+cudaError_t launch_sparse_attention(SparseArgs s, cudaStream_t stream);
+
 // Overlap statistics from hidden states and LM heads (lm_head_sm100.cu).
 struct LmHeadArgs {
   const void* h_draft;    // [rows, Hd] bf16

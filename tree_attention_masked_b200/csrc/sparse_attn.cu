@@ -1,0 +1,228 @@
+// Sparse attention with branch-consistent indexer groups over a proposal tree.
+//
+// SpecOPD (thelatestinai.com listing), Fig 4: every row reuses the complete
+// trunk group keys; an incomplete boundary group stays in the row's causal
+// tail; a group completed by branch tokens needs a branch-specific indexer
+// group key; indexer queries select eligible complete groups with top-k, and
+// attention reads the selected groups' keys and values plus the causal tail,
+// which bypasses top-k.  Readings (the figure prints no formula): groups are
+// g consecutive semantic positions of the row's own history (trunk through
+// the anchor, then its branch); a complete group's key is the mean of its
+// members' indexer keys; the score is the indexer query dotted with it; the
+// k best per KV head are taken, ties to the earlier group.
+//
+//   sparse_gkey_kernel -- the keys of every complete trunk group (shared by
+//                         all rows of the tree): fp32 mean in position order;
+//   sparse_attn_kernel -- one warp per (row, KV head): scores of the row's
+//                         complete groups (trunk keys from the table, keys of
+//                         groups holding branch tokens formed on the spot, in
+//                         the same order), top-k by repeated warp argmax,
+//                         then an fp32 online softmax over the chosen groups'
+//                         members and the tail for each query head of the KV
+//                         group (RoPE applied beforehand by the RoPE kernel).
+// Scores are sequential fp32 sums and fused multiply-adds in a fixed order,
+// so the selection is reproducible.
+#include <cuda_bf16.h>
+
+#include "internal.h"
+
+namespace specopd {
+namespace {
+
+constexpr int kSpD = 128;             // head dim
+constexpr int kSpWarps = 4;           // (row, KV head) items per CTA
+
+struct RowPlace {
+  int t;            // tree
+  long long base;   // first packed row of the tree
+  long long bfirst; // first packed row of the branch (branch rows)
+  int a;            // last trunk position of the history (the anchor; p itself for trunk rows)
+  int p;            // the row's semantic position
+};
+
+__device__ __forceinline__ RowPlace place_row(const SparseArgs& s, long long r) {
+  int lo = 0, hi = s.tp.num_trees - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) / 2;
+    if (s.tp.row_base[mid] <= r) lo = mid; else hi = mid - 1;
+  }
+  const int t = lo;
+  RowPlace x;
+  x.t = t;
+  x.base = s.tp.row_base[t];
+  const int T = s.tp.trunk_len[t], P = s.tp.prompt_len[t], rpb = s.tp.rows_per_branch;
+  const long long local = r - x.base;
+  if (local < T) {
+    x.p = (int)local;
+    x.a = x.p;
+    x.bfirst = 0;
+  } else {
+    const long long bl = (local - T) / rpb;
+    const int i = (int)((local - T) % rpb);
+    int a = s.anchors[s.tp.branch_base[t] + bl];
+    a = a < P ? P : (a > T - 1 ? T - 1 : a);
+    x.a = a;
+    x.p = a + 1 + i;
+    x.bfirst = x.base + T + bl * rpb;
+  }
+  return x;
+}
+
+__device__ __forceinline__ long long hist_row(const RowPlace& x, int q) {
+  return q <= x.a ? x.base + q : x.bfirst + (q - x.a - 1);
+}
+
+__device__ __forceinline__ float ldbf(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+__global__ void sparse_gkey_kernel(const SparseArgs s) {
+  const int gidx = blockIdx.x, kvh = blockIdx.y, e = threadIdx.x;
+  if (e >= s.di) return;
+  int t = 0;
+  while (t + 1 < s.tp.num_trees && s.gk_off[t + 1] <= gidx) ++t;
+  const int m = gidx - s.gk_off[t];
+  const long long base = s.tp.row_base[t];
+  const __nv_bfloat16* ki = static_cast<const __nv_bfloat16*>(s.ki);
+  float sum = 0.f;
+  for (int j = 0; j < s.g; ++j) sum += ldbf(ki + ((base + (long long)m * s.g + j) * s.Hkv + kvh) * s.di + e);
+  s.gkey[((long long)gidx * s.Hkv + kvh) * s.di + e] = sum / (float)s.g;
+}
+
+__global__ void __launch_bounds__(32 * kSpWarps) sparse_attn_kernel(const SparseArgs s) {
+  __shared__ float score[kSpWarps][kSpMaxGroups];
+  __shared__ int sel[kSpWarps][kSpMaxTopk];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long item = (long long)blockIdx.x * kSpWarps + w;
+  if (item >= s.N * s.Hkv) return;
+  const long long r = item / s.Hkv;
+  const int kvh = (int)(item % s.Hkv);
+  const RowPlace x = place_row(s, r);
+  const int t = x.t;
+  const int nc = (x.p + 1) / s.g;  // complete groups
+  const int tail0 = nc * s.g;
+  const __nv_bfloat16* qi = static_cast<const __nv_bfloat16*>(s.qi) + (r * s.Hkv + kvh) * s.di;
+  const __nv_bfloat16* ki = static_cast<const __nv_bfloat16*>(s.ki);
+
+  // ---- indexer scores of the complete groups
+  for (int m = lane; m < nc; m += 32) {
+    float acc = 0.f;
+    if (m * s.g + s.g - 1 <= x.a) {  // trunk group: the shared key
+      const float* key = s.gkey + ((long long)(s.gk_off[t] + m) * s.Hkv + kvh) * s.di;
+      for (int e = 0; e < s.di; ++e) acc = fmaf(ldbf(qi + e), key[e], acc);
+    } else {                          // holds branch tokens: this branch's key
+      for (int e = 0; e < s.di; ++e) {
+        float sum = 0.f;
+        for (int j = 0; j < s.g; ++j) sum += ldbf(ki + (hist_row(x, m * s.g + j) * s.Hkv + kvh) * s.di + e);
+        acc = fmaf(ldbf(qi + e), sum / (float)s.g, acc);
+      }
+    }
+    score[w][m] = acc;
+  }
+  __syncwarp();
+
+  // ---- top-k: repeated warp argmax (higher score, then lower index)
+  const int K = nc < s.topk ? nc : s.topk;
+  if (nc > s.topk) {
+    for (int it = 0; it < K; ++it) {
+      float bs = -INFINITY;
+      int bm = 0x7fffffff;
+      for (int m = lane; m < nc; m += 32) {
+        const float v = score[w][m];
+        if (v > bs || (v == bs && m < bm)) {
+          bs = v;
+          bm = m;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+        const int om = __shfl_xor_sync(0xffffffffu, bm, off);
+        if (os > bs || (os == bs && om < bm)) {
+          bs = os;
+          bm = om;
+        }
+      }
+      if (lane == 0) {
+        sel[w][it] = bm;
+        score[w][bm] = -INFINITY;
+      }
+      __syncwarp();
+    }
+    if (lane == 0) {  // groups in ascending order
+      for (int i = 1; i < K; ++i) {
+        const int v = sel[w][i];
+        int j = i - 1;
+        while (j >= 0 && sel[w][j] > v) {
+          sel[w][j + 1] = sel[w][j];
+          --j;
+        }
+        sel[w][j + 1] = v;
+      }
+    }
+  } else if (lane == 0) {
+    for (int i = 0; i < K; ++i) sel[w][i] = i;
+  }
+  __syncwarp();
+
+  // ---- attention over the chosen groups' members and the tail
+  const int ncols = K * s.g + (x.p + 1 - tail0);
+  const __nv_bfloat16* rq = static_cast<const __nv_bfloat16*>(s.rq);
+  const __nv_bfloat16* rk = static_cast<const __nv_bfloat16*>(s.rk);
+  const __nv_bfloat16* vv = static_cast<const __nv_bfloat16*>(s.v);
+  const int G = s.Hq / s.Hkv;
+  for (int hh = 0; hh < G; ++hh) {
+    const int h = kvh * G + hh;
+    float qv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) qv[i] = ldbf(rq + (r * s.Hq + h) * kSpD + lane * 4 + i) * s.scale_log2;
+    float mx = -INFINITY, l = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int c = 0; c < ncols; ++c) {
+      const int q = c < K * s.g ? sel[w][c / s.g] * s.g + c % s.g : tail0 + (c - K * s.g);
+      const long long col = hist_row(x, q);
+      const __nv_bfloat16* kp = rk + (col * s.Hkv + kvh) * kSpD + lane * 4;
+      float d = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) d = fmaf(qv[i], ldbf(kp + i), d);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+      const float mn = fmaxf(mx, d);
+      const float corr = exp2f(mx - mn), pw = exp2f(d - mn);
+      l = l * corr + pw;
+      const __nv_bfloat16* vp = vv + (col * s.Hkv + kvh) * kSpD + lane * 4;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[i] = fmaf(pw, ldbf(vp + i), o[i] * corr);
+      mx = mn;
+    }
+    __nv_bfloat16* op = static_cast<__nv_bfloat16*>(s.out) + (r * s.Hq + h) * kSpD + lane * 4;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) op[i] = __float2bfloat16(o[i] / l);
+  }
+}
+
+}  // namespace
+
+size_t sparse_group_keys(const TreeParams& tp, int g) {
+  size_t n = 0;
+  for (int t = 0; t < tp.num_trees; ++t) n += (size_t)(tp.trunk_len[t] / g);
+  return n;
+}
+
+cudaError_t launch_sparse_attention(SparseArgs s, cudaStream_t stream) {
+  int off = 0;
+  for (int t = 0; t < s.tp.num_trees; ++t) {
+    s.gk_off[t] = off;
+    off += s.tp.trunk_len[t] / s.g;
+  }
+  s.gk_off[s.tp.num_trees] = off;
+  cudaError_t e = launch_rope(s.q, s.k, s.rq, s.rk, SPECOPD_BF16, s.N, s.Hq, s.Hkv, kSpD, s.pos, s.theta, stream);
+  if (e != cudaSuccess) return e;
+  if (off > 0) {
+    sparse_gkey_kernel<<<dim3(off, s.Hkv), (s.di + 31) / 32 * 32, 0, stream>>>(s);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const long long items = s.N * s.Hkv;
+  sparse_attn_kernel<<<(unsigned)((items + kSpWarps - 1) / kSpWarps), 32 * kSpWarps, 0, stream>>>(s);
+  return cudaGetLastError();
+}
+
+}  // namespace specopd

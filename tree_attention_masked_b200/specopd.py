@@ -74,6 +74,10 @@ _c = {
     "specopd_gdn_workspace_bytes": _sig("specopd_gdn_workspace_bytes", _sz, _desc_p, _int),
     "specopd_gdn_tree": _sig("specopd_gdn_tree", _int, _desc_p, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _int, _int,
                              _int, _vp, _sz, _vp, _vp),
+    "specopd_sparse_workspace_bytes": _sig("specopd_sparse_workspace_bytes", _sz, _desc_p, _int, _int, _int, _int),
+    "specopd_sparse_tree_attention": _sig("specopd_sparse_tree_attention", _int, _desc_p, _vp, _vp, _vp, _vp, _vp,
+                                          _vp, _i64, _int, _int, _int, _int, _int, _int, _f32, _f32, _vp, _vp, _sz,
+                                          _vp, _vp),
     "specopd_lm_head_workspace_bytes": _sig("specopd_lm_head_workspace_bytes", _sz, _i64, _i64),
     "specopd_lm_head_overlap": _sig("specopd_lm_head_overlap", _int, _vp, _vp, _int, _vp, _vp, _int, _i64, _i64,
                                     _i64, _int, _f64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp, _vp),
@@ -256,3 +260,19 @@ def specopd_gdn_tree(trees: Trees, q, k, v, alpha, beta, out, workspace, status,
     _check("specopd_gdn_tree", _c["specopd_gdn_tree"](
         trees.ref(), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(out), q.shape[0], q.shape[1],
         q.shape[2], v.shape[2], _ptr(workspace), wb, _ptr(status), _stream(stream)))
+
+
+def specopd_sparse_workspace_bytes(trees: Trees, Hq: int, Hkv: int, di: int, g: int) -> int:
+    return _c["specopd_sparse_workspace_bytes"](trees.ref(), Hq, Hkv, di, g)
+
+
+def specopd_sparse_tree_attention(trees: Trees, q, k, v, qi, ki, out, pos, g: int, topk: int, rope_theta: float,
+                                  workspace, status, softmax_scale: float = 0.0, stream=None) -> None:
+    """Sparse attention with branch-consistent indexer groups: q [N, Hq, 128],
+    k, v [N, Hkv, 128], qi, ki [N, Hkv, di], out [N, Hq, 128] (bf16, contiguous)."""
+    _contig(q, k, v, qi, ki, out)
+    wb = workspace.numel() * workspace.element_size()
+    _check("specopd_sparse_tree_attention", _c["specopd_sparse_tree_attention"](
+        trees.ref(), _ptr(q), _ptr(k), _ptr(v), _ptr(qi), _ptr(ki), _ptr(out), q.shape[0], q.shape[1], k.shape[1],
+        q.shape[2], qi.shape[2], g, topk, rope_theta, softmax_scale, _ptr(pos), _ptr(workspace), wb, _ptr(status),
+        _stream(stream)))
