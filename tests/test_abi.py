@@ -139,6 +139,34 @@ def test_gdn_argument_errors_before_launch(S):
     assert g(*args(q=0)) == -1              # null input
 
 
+def test_sparse_argument_errors_before_launch(S):
+    import torch
+    trees = S.Trees([200], [10], [4], 4, torch.zeros(4, dtype=torch.int32))
+    N = S.specopd_tree_packed_rows(trees)
+    need = S.specopd_sparse_workspace_bytes(trees, 4, 2, 32, 8)
+    rq, rk, gk = N * 4 * 128 * 2, N * 2 * 128 * 2, (200 // 8) * 2 * 32 * 4
+    up = lambda x: (x + 255) // 256 * 256
+    assert need == up(rq) + up(rk) + up(gk)
+    f = S._c["specopd_sparse_tree_attention"]
+    args = lambda **kw: [trees.ref(), kw.get("q", 16), 16, 16, 16, 16, 16, kw.get("N", N), 4, kw.get("Hkv", 2),
+                         kw.get("d", 128), 32, kw.get("g", 8), kw.get("topk", 4), 1e4, 0.0, 16, 256,
+                         kw.get("ws", need), 16, None]
+    assert f(*args(d=64)) == -2             # d = 128 only
+    assert f(*args(Hkv=3)) == -2            # Hq a multiple of Hkv
+    assert f(*args(topk=65)) == -2          # top-k at most 64
+    assert f(*args(topk=0)) == -2
+    assert f(*args(g=0)) == -2
+    assert f(*args(N=N + 1)) == -2
+    assert f(*args(q=24)) == -6
+    assert f(*args(ws=need - 1)) == -5
+    assert f(*args(q=0)) == -1
+    # more than 1,024 complete groups in one history
+    big = S.Trees([3000], [10], [1], 4, torch.zeros(1, dtype=torch.int32))
+    nb = S.specopd_tree_packed_rows(big)
+    assert f(big.ref(), 16, 16, 16, 16, 16, 16, nb, 4, 2, 128, 32, 2, 4, 1e4, 0.0, 16, 256, 1 << 30, 16,
+             None) == -2
+
+
 def test_workspace_sizes(S):
     n_tiles = (151936 + 255) // 256
     assert S.specopd_lm_head_workspace_bytes(1024, 151936) >= n_tiles * 1024 * 24 + 3 * 1024 * 4
