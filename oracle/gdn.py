@@ -80,3 +80,44 @@ def checkpoint_states(q: np.ndarray, k: np.ndarray, v: np.ndarray, alpha: np.nda
             _, S = gdn_sequence(q[sl, h], k[sl, h], v[sl, h], alpha[sl, h], beta[sl, h], S)
             out[j, h] = S
     return out
+
+
+def gdn_sequence_chunked(q: np.ndarray, k: np.ndarray, v: np.ndarray, alpha: np.ndarray, beta: np.ndarray,
+                         C: int, state: np.ndarray = None):
+    """The same recurrence as gdn_sequence, C tokens at a time (a second
+    formulation, checked against the sequential one; it is the chunked form a
+    tensor-core trunk pass follows).
+
+    Within a chunk with start state S0, cumulative decays g_t = prod_{i<=t}
+    alpha_i and update vectors u_t (S_t = alpha_t S_{t-1} + u_t k_t^T), the
+    delta rule gives
+        u_t + beta_t sum_{i<t} (g_t / g_i) (k_t . k_i) u_i = beta_t (v_t - g_t S0 k_t),
+    a unit lower-triangular system (I + A) U = diag(beta) (V - diag(g) K S0^T);
+    then
+        O   = diag(g) Q S0^T + (L o (Q K^T)) U,   L_ti = g_t / g_i for i <= t,
+        S_C = g_C S0 + (diag(g_C / g) U)^T K.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    alpha = np.asarray(alpha, dtype=np.float64)
+    beta = np.asarray(beta, dtype=np.float64)
+    L, dk = k.shape
+    dv = v.shape[1]
+    S = np.zeros((dv, dk)) if state is None else np.array(state, dtype=np.float64)
+    o = np.zeros((L, dv))
+    for c0 in range(0, L, C):
+        sl = slice(c0, min(L, c0 + C))
+        qc, kc, vc, bc = q[sl], k[sl], v[sl], beta[sl]
+        lg = np.cumsum(np.log(alpha[sl]))              # log g_t
+        n = kc.shape[0]
+        ratio = np.exp(lg[:, None] - lg[None, :])      # g_t / g_i
+        A = np.tril(bc[:, None] * ratio * (kc @ kc.T), -1)
+        rhs = bc[:, None] * (vc - np.exp(lg)[:, None] * (kc @ S.T))
+        U = np.zeros((n, dv))
+        for t in range(n):                             # forward substitution, unit diagonal
+            U[t] = rhs[t] - A[t, :t] @ U[:t]
+        Lmask = np.tril(ratio)
+        o[sl] = np.exp(lg)[:, None] * (qc @ S.T) + (Lmask * (qc @ kc.T)) @ U
+        S = np.exp(lg[-1]) * S + (np.exp(lg[-1] - lg)[:, None] * U).T @ kc
+    return o, S

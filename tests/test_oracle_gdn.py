@@ -10,7 +10,9 @@ What fixes the answers:
     of the alphas;
   * tree structure: a branch anchored at the last trunk token continues the
     trunk sequence; a branch never sees other branches or trunk tokens after
-    its anchor; the C-token checkpoints equal the states of prefix runs.
+    its anchor; the C-token checkpoints equal the states of prefix runs;
+  * the chunked (triangular-solve) formulation equals the sequential one for
+    whole, ragged and single-token chunks and a non-zero start state.
 """
 import numpy as np
 
@@ -119,3 +121,17 @@ def test_checkpoints_are_prefix_states():
         for h in range(H):
             _, S = G.gdn_sequence(q[:C * j, h], k[:C * j, h], v[:C * j, h], a[:C * j, h], b[:C * j, h])
             assert np.max(np.abs(cp[j - 1, h] - S)) < 1e-12
+
+
+def test_chunked_form_equals_the_sequential_recurrence():
+    rng = np.random.default_rng(8)
+    L, dk, dv = 70, 8, 5
+    q, k, v = rng.normal(size=(L, dk)), rng.normal(size=(L, dk)), rng.normal(size=(L, dv))
+    k /= np.linalg.norm(k, axis=1, keepdims=True)
+    alpha, beta = rng.uniform(0.7, 1.0, size=L), rng.uniform(0.0, 1.0, size=L)
+    S0 = rng.normal(size=(dv, dk))
+    o_ref, S_ref = G.gdn_sequence(q, k, v, alpha, beta, S0)
+    for C in (1, 3, 16, 64, 100):                    # whole, ragged and single chunks
+        o, S = G.gdn_sequence_chunked(q, k, v, alpha, beta, C, S0)
+        assert np.max(np.abs(o - o_ref)) < 1e-10, C
+        assert np.max(np.abs(S - S_ref)) < 1e-10, C
