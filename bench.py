@@ -543,7 +543,8 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-lm-head", action="store_true", help="skip the separately timed LM-head path")
+    ap.add_argument("--no-lm-head", action="store_true",
+                    help="skip the separately timed next-row paths (LM head, GDN, sparse attention)")
     ap.add_argument("--lm-head-only", action="store_true",
                     help="time only the LM-head path (one JSON line; for profiling it alone)")
     ap.add_argument("--lm-head-vocab", type=int, default=151936, help="vocabulary of the LM-head path")
