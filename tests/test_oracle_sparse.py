@@ -110,3 +110,17 @@ def test_fp32_decision_agrees_with_fp64_away_from_ties():
     q, k, v, qi, ki = _inputs(pt.num_rows, 2, 1, 8, 16, 7)
     for r in range(pt.num_rows):
         assert SP.selected_columns(pt, r, qi, ki, 4, 2, 0) == SP.selected_columns(pt, r, qi, ki, 4, 2, 0, True)
+
+
+def test_exact_ties_pick_the_earliest_groups_in_both_precisions():
+    pt = T.pack([33], [0], [1], [20], 4, True)
+    N = pt.num_rows
+    zeros = np.zeros((N, 1, 8))
+    for r in (10, 32, 33, 36):
+        for fp32 in (False, True):
+            cols = SP.selected_columns(pt, r, zeros, zeros, 4, 2, 0, fp32)
+            hist = SP.history(pt, r)
+            p = len(hist) - 1
+            nc = (p + 1) // 4
+            expect = hist[:min(nc, 2) * 4] + hist[nc * 4:]
+            assert cols == expect, (r, fp32)
