@@ -6,7 +6,10 @@ mask build -> RoPE + tree-masked GQA attention -> fused overlap / E2E-TV loss /
 gradient.  The metric is supervised tokens (predictions contributing to the
 loss, sum_b W) scored per second.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2] [--impl reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 5] [--impl reference]
+
+The default workload is the largest single-GPU one ("scale27b": trunk 32,768,
+512 branches x 16 samples, 40/8 heads of 128, vocabulary 248,320).
 
 N > 1 runs under torchrun: each rank scores its own batch (weak scaling; the
 trees are independent problems, so the data path has no collective), the
@@ -16,6 +19,7 @@ timed region is bracketed by barriers and the slowest rank's time is used.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -30,14 +34,34 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "supervised tokens/s scored (tree attn + E2E-TV) on 1 B200; % of roofline"
-WORKLOAD_DEFAULT = 2
+WORKLOAD_DEFAULT = 5
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per step of a
-# step's kernels, from one ncu capture of each kernel on the gqa8b workload.
-# They hold only for the kernels they were taken on; a workload without a
-# capture reports null.  Overlap pass (statistics + gradient in one launch):
-# 1201.974 + 585.504512 MB.  Attention: 63.078144 + 6.784256 MB.
-MEASURED_TRAFFIC = {2: {"tv_overlap_e2e": 1787.478512e6, "tree_attention": 69.8624e6}}
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of a
+# step's kernels, each from one ncu capture (the profiles/ summary named in
+# "profile" gives the command).  Each entry records a digest of the kernel's
+# source files at capture time; when the sources differ from it the bench
+# reports null, so a figure never outlives the kernel it was taken on.
+KERNEL_SOURCES = {
+    "tree_attention": ["tree_attention_masked_b200/csrc/tree_attn_sm100.cu", "tree_attention_masked_b200/csrc/ptx.cuh"],
+    "tv_overlap_e2e": ["tree_attention_masked_b200/csrc/tv_bf16.cu", "tree_attention_masked_b200/csrc/overlap_common.cuh",
+                       "tree_attention_masked_b200/csrc/ptx.cuh"],
+}
+MEASURED_TRAFFIC = {}  # {(workload, kernel): {"bytes": B, "sha": digest, "profile": file}}
+
+
+def source_digest(kernel: str) -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: int, kernel: str):
+    e = MEASURED_TRAFFIC.get((workload, kernel))
+    if e is None or e["sha"] != source_digest(kernel):
+        return None
+    return e["bytes"]
 
 
 def load_peaks():
@@ -127,9 +151,20 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- CPU oracle timing
-def oracle_sample(case, rng, attn_rows: int, branches: int, mask_rows: int):
+# One sample of the oracle per call: the same plan for the native arm's
+# cpu_baseline (three samples) and for each step of the reference arm, so the
+# two estimate the same quantity.
+ORACLE_PLAN = dict(attn_rows=8, branches=2, mask_rows=256)
+
+
+def oracle_sample(case, rng, attn_rows: int, branches: int, mask_rows: int, f64=None):
     """Time the oracle on a bounded sample of one step; returns the estimated
-    seconds of a whole step and a description of the sample."""
+    seconds of a whole step and a description of the sample.
+
+    Per-unit work (a packed row's mask fields, a packed row's attention over
+    all heads, a branch's overlap + loss + gradient) is scaled by the number of
+    units in the step; work done once per step whatever the sample (tree
+    structure, RoPE of every key row) is counted once."""
     from oracle import attention as OA
     from oracle import overlap as OO
     from oracle import tree as OT
@@ -137,7 +172,7 @@ def oracle_sample(case, rng, attn_rows: int, branches: int, mask_rows: int):
 
     t0 = time.perf_counter()
     pt = OT.pack(case.trunk_len, case.prompt_len, case.num_branches, case.anchors, case.W, case.pack_terminal)
-    OT.positions(pt)
+    pos = OT.positions(pt)
     OT.prediction_rows(pt)
     t_struct = time.perf_counter() - t0
     N = pt.num_rows
@@ -145,11 +180,15 @@ def oracle_sample(case, rng, attn_rows: int, branches: int, mask_rows: int):
     t0 = time.perf_counter()
     OT.compact_fields(pt, rows)
     t_mask = (time.perf_counter() - t0) / len(rows) * N
+    q, k, v = f64 if f64 is not None else (to_f64(x, case.dtype) for x in (case.q, case.k, case.v))
+    t0 = time.perf_counter()
+    OA.rope(k, pos, case.theta)  # the once-per-step part of tree_attention below
+    t_rope_k = time.perf_counter() - t0
     rows = rng.choice(N, size=min(attn_rows, N), replace=False)
-    q, k, v = (to_f64(x, case.dtype) for x in (case.q, case.k, case.v))
     t0 = time.perf_counter()
     OA.tree_attention(pt, q, k, v, theta=case.theta, rows=rows)
-    t_attn = (time.perf_counter() - t0) / len(rows) * N
+    t_rows = max(time.perf_counter() - t0 - t_rope_k, 0.0)
+    t_attn = t_rope_k + t_rows / len(rows) * N
     nb = int(sum(case.num_branches))
     bs = rng.choice(nb, size=min(branches, nb), replace=False)
     t0 = time.perf_counter()
@@ -162,9 +201,9 @@ def oracle_sample(case, rng, attn_rows: int, branches: int, mask_rows: int):
         OO.e2e_tv_grad_draft(z, t, case.W, count=nb * case.W)
     t_ov = (time.perf_counter() - t0) / len(bs) * nb
     total = t_struct + t_mask + t_attn + t_ov
-    desc = (f"oracle on {len(rows)} of {N} packed rows (attention, all {case.Hq} heads), {mask_rows} rows of "
-            f"mask fields, {len(bs)} of {nb} branches (overlap + loss + gradient over all {case.W} rows), "
-            f"scaled linearly to the full step")
+    desc = (f"oracle on {len(rows)} of {N} packed rows (attention, all {case.Hq} heads; RoPE of all key rows "
+            f"counted once), {len(bs)} of {nb} branches (overlap + loss + gradient over all {case.W} rows), "
+            f"mask fields of {mask_rows} rows; per-row and per-branch times scaled to the full step")
     return total, desc
 
 
@@ -177,21 +216,35 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
-def cpu_baseline(case, seconds_target: float = 15.0):
+def oracle_inputs(case):
+    from synthetic import to_f64
+    return tuple(to_f64(x, case.dtype) for x in (case.q, case.k, case.v))
+
+
+def cpu_baseline(case, samples: int = 3):
     rng = np.random.default_rng(123)
-    # a first small sample fixes the cost per unit, then the sample is sized
-    # to about `seconds_target` of CPU work
-    t_step, _ = oracle_sample(case, rng, attn_rows=2, branches=1, mask_rows=8)
+    f64 = oracle_inputs(case)
+    ests = []
     t0 = time.perf_counter()
-    est, desc = oracle_sample(case, rng, attn_rows=8, branches=1, mask_rows=32)
-    spent = time.perf_counter() - t0
-    if spent < seconds_target / 3:
-        scale = max(1, int(seconds_target / max(spent, 1e-3)))
-        est, desc = oracle_sample(case, rng, attn_rows=min(8 * scale, 256), branches=min(scale, 8),
-                                  mask_rows=min(32 * scale, 512))
-    value = case.num_predictions / est
-    return {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle", "sample": desc,
-            "est_step_s": est}
+    for _ in range(samples):
+        est, desc = oracle_sample(case, rng, f64=f64, **ORACLE_PLAN)
+        ests.append(est)
+    wall = time.perf_counter() - t0
+    est = statistics.mean(ests)
+    return {"value": case.num_predictions / est, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": desc + f"; mean of {samples} samples, {wall:.1f} s wall", "est_step_s": est}
+
+
+def config_dict(case, figs, workload: int, seed: int, world: int) -> dict:
+    """The workload description printed by both arms."""
+    import synthetic as SY
+    in_bytes = case.q.nbytes + case.k.nbytes + case.v.nbytes
+    if case.draft is not None:
+        in_bytes += case.draft.nbytes + case.teacher.nbytes
+    return {"workload": SY.WORKLOADS[workload], "supervised_tokens_per_step": figs["R"],
+            "packed_rows": case.num_rows, "visible_pairs": figs["pairs"], "seed": seed,
+            "l2": "inputs larger than L2 (%.2f GB per step > 126 MB); each step streams them from HBM" % (in_bytes / 1e9),
+            "parallelism": f"dp{world} (independent tree batches per rank)"}
 
 
 # ----------------------------------------------------------------- GPU run
@@ -283,7 +336,7 @@ def run_gpu(args):
         h_loss.copy_(st.loss, non_blocking=True)
         h_alpha.copy_(st.alpha[:st.R], non_blocking=True)
 
-    Ke = min(K, 50)  # the host copies dominate; 50 steps are plenty
+    Ke = min(K, 50 if h2d < 2e9 else 10)  # the host copies dominate; a few steps are plenty
     for _ in range(max(1, Wm // 2)):
         e2e_step()
     torch.cuda.synchronize()
@@ -310,22 +363,34 @@ def run_gpu(args):
                            "frac": ov_gbs / peaks["hbm"], "algorithmic_bytes": figs["ov_bytes"]},
         "build_tree_mask": {"ms": t_mask},
     }
+    # A kernel timed inside a step run back to back for a second or more works
+    # under the power cap: its tensor peak is the sustained GEMM figure; the
+    # burst figure is reported beside it.
+    long_region = elapsed_ms >= 1000.0 and peaks.get("bf16_sustained")
+    tpeak = peaks["bf16_sustained"] if long_region else peaks["bf16"]
+    kt = kernels["tree_attention"]
+    kt["frac_burst"] = kt["frac"]
+    kt["peak_burst"] = kt["peak"]
+    kt["peak"] = tpeak
+    kt["frac"] = kt["achieved"] / tpeak
+    kt["traffic"] = measured_traffic(args.workload, "tree_attention")
+    kernels["tv_overlap_e2e"]["traffic"] = measured_traffic(args.workload, "tv_overlap_e2e")
     dom = "tree_attention" if t_attn >= t_ov else "tv_overlap_e2e"
     kd = kernels[dom]
+    peak_src = ("bf16_tflops_sustained: timed region %.1f s" % (elapsed_ms / 1e3) if long_region else "bf16_tflops burst"
+                ) if dom == "tree_attention" else "hbm_gbs"
     roofline = {"bound": kd["bound"], "achieved": kd["achieved"], "peak": kd["peak"], "unit": kd["unit"],
-                "frac": kd["frac"], "traffic": MEASURED_TRAFFIC.get(args.workload, {}).get(dom), "kernel": dom,
-                "peak_source": f"{peaks['source']} ({'bf16_tflops burst' if dom == 'tree_attention' else 'hbm_gbs'})"}
+                "frac": kd["frac"], "traffic": kd["traffic"], "kernel": dom,
+                "peak_source": f"{peaks['source']} ({peak_src})"}
+    if dom == "tree_attention":
+        roofline["frac_burst"] = kd["frac_burst"]
     tokens = figs["R"] * world
     value = tokens * K / (elapsed_ms * 1e-3)
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": Wm,
         "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": case.dtype, "data": "synthetic (seeded; no datasets or weights)",
-        "config": {"workload": SY.WORKLOADS[args.workload], "supervised_tokens_per_step": figs["R"],
-                   "packed_rows": case.num_rows, "visible_pairs": figs["pairs"], "seed": args.seed,
-                   "l2": "inputs larger than L2 (%.2f GB per step > 126 MB); each step streams them from HBM" %
-                         ((case.q.nbytes + case.k.nbytes + case.v.nbytes + case.draft.nbytes + case.teacher.nbytes) / 1e9),
-                   "parallelism": f"dp{world} (independent tree batches per rank)"},
+        "config": config_dict(case, figs, args.workload, args.seed, world),
         "roofline": roofline,
         "kernels": kernels,
         "clocks": clk,
@@ -353,33 +418,73 @@ def run_gpu(args):
 
 
 def run_reference(args):
+    """The reference arm: the fp64 oracle as it stands on the host cores, each
+    step one bounded sample of the workload (ORACLE_PLAN, the plan the native
+    arm's cpu_baseline uses) scaled to the full step."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     import synthetic as SY
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     case = SY.make_workload(args.workload, seed=args.seed, workers=min(8, os.cpu_count() or 1))
     figs = case_figures(case)
+    f64 = oracle_inputs(case)
     rng = np.random.default_rng(7)
     for _ in range(args.warmup):
-        oracle_sample(case, rng, attn_rows=1, branches=1, mask_rows=4)
+        oracle_sample(case, rng, f64=f64, **ORACLE_PLAN)
     ests = []
     t0 = time.perf_counter()
     desc = ""
     for _ in range(args.steps):
-        est, desc = oracle_sample(case, rng, attn_rows=2, branches=1, mask_rows=8)
+        est, desc = oracle_sample(case, rng, f64=f64, **ORACLE_PLAN)
         ests.append(est)
     wall = time.perf_counter() - t0
     est = statistics.mean(ests)
     value = figs["R"] / est
-    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3, "higher_is_better": True,
-           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; no datasets or weights)",
            "impl": "reference",
-           "config": {"workload": SY.WORKLOADS[args.workload], "supervised_tokens_per_step": figs["R"]},
+           "config": config_dict(case, figs, args.workload, args.seed, world),
            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                            "sample": desc + f"; {args.steps} samples, {wall:.1f} s wall"},
+                            "sample": desc + f"; mean of {args.steps} samples, {wall:.1f} s wall"},
            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
+
+
+def attention_only(args):
+    """Mask + RoPE + tree attention of one workload, no logits (a small
+    device footprint, for profiling the attention kernel alone)."""
+    import torch
+    import synthetic as SY
+    from tree_attention_masked_b200.build import build
+    build()
+    from tree_attention_masked_b200.scoring import ScoringStep
+    dev = torch.device("cuda", 0)
+    case = SY.make_workload(args.workload, seed=args.seed, workers=min(8, os.cpu_count() or 1), with_logits=False)
+    figs = case_figures(case)
+    st = ScoringStep(case.trunk_len, case.prompt_len, case.num_branches, case.W, case.Hq, case.Hkv, case.d,
+                     torch.bfloat16 if case.dtype == "bf16" else torch.float32, 1, device=dev,
+                     pack_terminal=case.pack_terminal, theta=case.theta, with_grad=False)
+    st.load(case)
+    stream = torch.cuda.current_stream(dev)
+    st.build_mask(stream)
+    for _ in range(args.warmup):
+        st.attention(stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        st.attention(stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    peaks = load_peaks()
+    tf = figs["flops"] / (ms * 1e-3) / 1e12
+    print(json.dumps({"metric": "RoPE + tree attention", "value": ms, "unit": "ms", "higher_is_better": False,
+                      "workload": SY.WORKLOADS[args.workload], "achieved_tflops": tf,
+                      "frac_burst": tf / peaks["bf16"], "useful_flops": figs["flops"],
+                      "device_status": st.check_status()}), flush=True)
 
 
 def lm_head_measure(dev, peaks, seed: int, V: int = 151936) -> dict:
@@ -537,7 +642,7 @@ def sparse_measure(dev, peaks, seed: int) -> dict:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", type=int, default=WORKLOAD_DEFAULT)
     ap.add_argument("--seed", type=int, default=0)
@@ -550,11 +655,15 @@ def main():
     ap.add_argument("--lm-head-vocab", type=int, default=151936, help="vocabulary of the LM-head path")
     ap.add_argument("--gdn-only", action="store_true", help="time only the GDN path (one JSON line)")
     ap.add_argument("--sparse-only", action="store_true", help="time only the sparse indexer-group attention")
+    ap.add_argument("--attention-only", action="store_true",
+                    help="time only RoPE + tree attention of the workload (no logits; for profiling)")
     args = ap.parse_args()
     # at least three untimed warm-up steps, whatever was asked for
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
         run_reference(args)
+    elif args.attention_only:
+        attention_only(args)
     elif args.sparse_only:
         import torch
         from tree_attention_masked_b200.build import build

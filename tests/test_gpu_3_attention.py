@@ -72,6 +72,11 @@ TC = [
     dict(trees=[(250, 30, 7)], W=6, Hq=4, Hkv=2, sort_anchors=False),
     dict(trees=[(90, 5, 3)], W=64, Hq=2, Hkv=1, anchors=[60, 5, 89]),  # full-width branches
     dict(trees=[(1100, 200, 40)], W=16, Hq=4, Hkv=1),                  # 9 trunk tiles, 5 branch tiles
+    # odd G: the last head of a KV group runs on two neighbouring tiles of one
+    # tree; 7 tiles over 3 trees, so one tile pair straddles a tree boundary
+    # (two single-slot CTAs) and the last tile has no partner
+    dict(trees=[(129, 0, 5), (77, 70, 3), (400, 100, 17)], W=3, Hq=10, Hkv=2),
+    dict(trees=[(300, 40, 9)], W=4, Hq=6, Hkv=2),                      # G = 3, three tiles
 ]
 
 

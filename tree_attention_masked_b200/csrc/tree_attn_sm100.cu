@@ -4,12 +4,17 @@
 // packed queries share the trunk's keys and values while each row attends only
 // to itself and its ancestors.  The pages give no kernel; this design is new:
 //
-//  * a CTA owns one 128-row query tile of one tree and two query heads that
-//    read the same KV head (GQA), so every K/V tile it loads feeds two heads;
-//  * the columns it visits are the tile's trunk span [tree_base, trunk_hi)
-//    followed by its branch span [br_lo, br_hi) (both from the mask builder);
-//    column blocks outside them are never loaded.  Trunk blocks below
-//    `trunk_full` are seen by every row and skip masking entirely;
+//  * a CTA owns two (query tile, query head) slots that read the same KV
+//    head (GQA), so every K/V tile it loads feeds both: two heads of one
+//    128-row tile, or -- for the last head of an odd group size G -- that
+//    head on two neighbouring tiles of one tree, so that no CTA runs with a
+//    single head (its second softmax warpgroup would idle and each K/V load
+//    would feed half the MMA work);
+//  * the columns it visits are the trunk span [tree_base, trunk_hi)
+//    followed by the branch span [br_lo, br_hi) of its tile(s) (from the mask
+//    builder; for two tiles their union, masked per row); column blocks
+//    outside them are never loaded.  Trunk blocks below `trunk_full` are seen
+//    by every row and skip masking entirely;
 //  * warp 0 issues TMA tile loads (no multicast) into a 4-slot K/V ring,
 //    one thread of warp 1 issues tcgen05.mma: S = Q K^T into TMEM, then
 //    O += P V with P read straight from TMEM;
@@ -65,7 +70,8 @@ struct Params {
   const uint64_t* anc_bits;
   const specopd_tile_meta* meta;
   int num_tiles;
-  int Hq, Hkv, G, pairs;
+  int Hq, Hkv, G, pairs;  // pairs = G / 2 head pairs per tile
+  int items_per_pair;     // work items per pair of tiles (2k, 2k+1)
   float scale_log2;
   int32_t* status;
 };
@@ -97,19 +103,58 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: (tile, kv head, head pair); expensive tiles (late rows) first
-  const int items_per_tile = p.Hkv * p.pairs;
-  const int w = blockIdx.x;
-  const int tile = p.num_tiles - 1 - w / items_per_tile;
-  const int rem = w % items_per_tile;
-  const int kvh = rem / p.pairs;
-  const int pair = rem % p.pairs;
-  const int h0 = kvh * p.G + 2 * pair;
-  const int nq = (2 * pair + 1 < p.G) ? 2 : 1;
-  const specopd_tile_meta m = p.meta[tile];
+  // ---- work item.  Tiles are taken in pairs (2k, 2k+1), the latest rows (the
+  // costliest) first.  Per pair: for each of its two tiles, KV head and head
+  // pair an item with two heads of that tile; for odd G, per KV head one item
+  // with head G-1 on both tiles (when they belong to the same tree; else one
+  // single-slot item per tile).  Items with nothing to do return at once.
+  int tile_s[2], head_s[2], nq;
+  {
+    const int w = blockIdx.x;
+    const int k = (p.num_tiles + 1) / 2 - 1 - w / p.items_per_pair;
+    const int r = w % p.items_per_pair;
+    const int n_two = 2 * p.Hkv * p.pairs;
+    if (r < n_two) {
+      const int sub = r / (p.Hkv * p.pairs);
+      const int rem = r % (p.Hkv * p.pairs);
+      const int h = (rem / p.pairs) * p.G + 2 * (rem % p.pairs);
+      tile_s[0] = tile_s[1] = 2 * k + 1 - sub;
+      head_s[0] = h;
+      head_s[1] = h + 1;
+      nq = 2;
+    } else {
+      const int sub = (r - n_two) / p.Hkv;
+      const int h = ((r - n_two) % p.Hkv) * p.G + p.G - 1;
+      const bool has1 = 2 * k + 1 < p.num_tiles;
+      const bool same = has1 && p.meta[2 * k].tree_base == p.meta[2 * k + 1].tree_base;
+      head_s[0] = head_s[1] = h;
+      tile_s[0] = 2 * k + sub;
+      tile_s[1] = 2 * k + 1;
+      nq = same ? (sub == 0 ? 2 : 0) : 1;
+    }
+    if (tile_s[0] >= p.num_tiles) nq = 0;
+  }
+  if (nq == 0) return;  // uniform over the CTA, before any barrier or TMEM use
+  // column spans: the union over the CTA's tiles (each slot's rows mask per row)
+  specopd_tile_meta m = p.meta[tile_s[0]];
+  if (nq == 2 && tile_s[1] != tile_s[0]) {
+    const specopd_tile_meta m1 = p.meta[tile_s[1]];
+    m.trunk_hi = max(m.trunk_hi, m1.trunk_hi);
+    m.trunk_full = min(m.trunk_full, m1.trunk_full);
+    if (m1.br_hi > m1.br_lo) {
+      if (m.br_hi > m.br_lo) {
+        m.br_lo = min(m.br_lo, m1.br_lo);
+        m.br_hi = max(m.br_hi, m1.br_hi);
+      } else {
+        m.br_lo = m1.br_lo;
+        m.br_hi = m1.br_hi;
+      }
+    }
+  }
   const int n_trunk = (m.trunk_hi - m.tree_base + kBN - 1) / kBN;
   const int n_br = (m.br_hi > m.br_lo) ? (m.br_hi - m.br_lo + kBN - 1) / kBN : 0;
   const int nblk = n_trunk + n_br;
+  const int kvh = head_s[0] / p.G;
 
   if (threadIdx.x == 0) {
     mbar_init(&sm->q_full, 1);
@@ -150,9 +195,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ================= TMA producer
     if (lane == 0) {
       mbar_arrive_expect_tx(&sm->q_full, nq * kTileBytes);
-      for (int t = 0; t < nq; ++t)
+      for (int t = 0; t < nq; ++t) {
+        const int row0 = p.meta[tile_s[t]].row_start;
         for (int hx = 0; hx < 2; ++hx)
-          tma_load_3d(sm->q[t] + hx * kBoxBytes, &tmQ, hx * 64, h0 + t, m.row_start, &sm->q_full);
+          tma_load_3d(sm->q[t] + hx * kBoxBytes, &tmQ, hx * 64, head_s[t], row0, &sm->q_full);
+      }
       int last_n[kSlots] = {-1, -1, -1, -1};
       for (int n = 0; n < 2 * nblk; ++n) {
         const int slot = n % kSlots;
@@ -232,8 +279,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (t < nq) {
       const int quad = warp & 3;
       const int rloc = quad * 32 + lane;
-      const int r = m.row_start + rloc;
-      const bool valid = r < m.row_end;
+      const int r = p.meta[tile_s[t]].row_start + rloc;
+      const bool valid = r < p.meta[tile_s[t]].row_end;
       int lim = m.tree_base, bstart = 0;
       uint64_t bits = 0;
       if (valid) {
@@ -331,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok && mbar_wait_warp(&sm->o_done[t], (nblk - 1) & 1, abort_flag)) {
         tc_fence_after();
         const float inv = 1.f / l;
-        __nv_bfloat16* orow = p.out + ((long long)r * p.Hq + h0 + t) * kHD;
+        __nv_bfloat16* orow = p.out + ((long long)r * p.Hq + head_s[t]) * kHD;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t orr[32];
@@ -391,14 +438,15 @@ cudaError_t launch_tree_attention_sm100(const AttnArgs& a, cudaStream_t stream) 
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;
   p.G = a.Hq / a.Hkv;
-  p.pairs = (p.G + 1) / 2;
+  p.pairs = p.G / 2;
+  p.items_per_pair = p.Hkv * (2 * p.pairs + 2 * (p.G & 1));
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.status = a.status;
   const size_t smem = sizeof(Smem) + 1024;
   cudaError_t e =
       cudaFuncSetAttribute(tree_attn_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const long long grid = (long long)a.num_tiles * p.Hkv * p.pairs;
+  const long long grid = (long long)((a.num_tiles + 1) / 2) * p.items_per_pair;
   tree_attn_sm100_kernel<<<(unsigned)grid, kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
