@@ -25,8 +25,10 @@ Modules:
                 every row reading the state of its own history
   sparse     -- sparse attention with branch-consistent indexer groups: top-k
                 complete groups per row plus the causal tail
+  conv       -- short causal convolution along each row's own history (the
+                GDN feature path's convolution that follows branch ancestry)
 
 Every function is plain fp64 NumPy written from the definitions; nothing is
 blocked, fused or reordered.
 """
-from . import tree, attention, overlap, lm_head, gdn, sparse  # noqa: F401
+from . import tree, attention, overlap, lm_head, gdn, sparse, conv  # noqa: F401

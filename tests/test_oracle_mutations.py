@@ -222,3 +222,34 @@ def test_sparse_boundary_group_keyed_by_trunk_only_breaks_the_branch_pin():
     bad = (slipped(pt, 12, qi, ki, 4, 1, 0), slipped(pt, 14, qi, ki, 4, 1, 0))
     assert good[0] != good[1]
     assert bad[0][:4] == bad[1][:4] == [0, 1, 2, 3]   # both branches fall back to the trunk group
+
+
+def test_conv_over_packed_neighbours_breaks_the_fir_pin():
+    """Convolving over the packed neighbours r, r-1, ... instead of the row's
+    history puts a sibling's or trunk tail's tokens in a branch row's window;
+    the per-history FIR pin catches it."""
+    from scipy.signal import lfilter
+    from oracle import conv as CV
+
+    def slipped(pt, x, w):
+        out = np.zeros_like(x)
+        for r in range(pt.num_rows):
+            for j in range(w.shape[1]):
+                if r - j >= 0:
+                    out[r] += w[:, j] * x[r - j]
+        return out
+    pt = T.pack([20], [3], [3], [5, 5, 19], 4, True)
+    rng = np.random.default_rng(1)
+    x = rng.normal(size=(pt.num_rows, 3))
+    w = rng.normal(size=(3, 4))
+
+    def fir_mismatch(conv):
+        out = conv(pt, x, w)
+        worst = 0.0
+        for r in range(pt.num_rows):
+            hist = CV.history(pt, r)
+            ref = np.stack([lfilter(w[c], [1.0], x[hist, c]) for c in range(3)], axis=1)[-1]
+            worst = max(worst, float(np.max(np.abs(out[r] - ref))))
+        return worst
+    assert fir_mismatch(CV.tree_causal_conv) < 1e-12
+    assert fir_mismatch(slipped) > 0.1
