@@ -32,7 +32,7 @@ or reuse of group keys across rows.
 """
 from __future__ import annotations
 
-from typing import Iterable, List, Optional
+from typing import Iterable, List, Mapping, Optional, Sequence, Tuple
 
 import numpy as np
 
@@ -45,57 +45,53 @@ def history(pt: _tree.PackedTrees, r: int) -> List[int]:
     return _tree.ancestors(pt, r)[::-1] + [r]
 
 
-def _scores_fp32(qr: np.ndarray, members: List[np.ndarray]) -> np.ndarray:
-    """Indexer scores taken in fp32 in a fixed order: each group key is the
-    sequential fp32 sum of its members' keys divided by g, each score a
-    sequential chain of fused multiply-adds over the key's elements (every step
-    rounded once to fp32)."""
-    out = np.zeros(len(members))
-    q32 = np.asarray(qr, dtype=np.float32)
-    for m, mem in enumerate(members):
-        key = np.zeros(mem.shape[1], dtype=np.float32)
-        for row in np.asarray(mem, dtype=np.float32):
-            key = (key + row).astype(np.float32)
-        key = (key / np.float32(mem.shape[0])).astype(np.float32)
-        acc = np.float32(0.0)
-        for e in range(key.shape[0]):
-            acc = np.float32(float(q32[e]) * float(key[e]) + float(acc))
-        out[m] = float(acc)
-    return out
+def group_scores(pt: _tree.PackedTrees, r: int, qi: np.ndarray, ki: np.ndarray, g: int,
+                 kvh: int) -> np.ndarray:
+    """fp64 indexer scores of row r's complete groups for KV head kvh: group m's
+    key is the mean of the indexer keys of history positions m g .. m g + g - 1
+    (branch-specific when the group holds branch tokens, since the history is
+    the branch's own), and its score is the row's indexer query dotted with it."""
+    hist = history(pt, r)
+    n_complete = len(hist) // g
+    if n_complete == 0:
+        return np.zeros(0)
+    keys = np.stack([np.mean(np.asarray(ki[hist[m * g:(m + 1) * g], kvh], dtype=np.float64), axis=0)
+                     for m in range(n_complete)])
+    return keys @ np.asarray(qi[r, kvh], dtype=np.float64)
+
+
+def top_groups(scores: np.ndarray, topk: int) -> List[int]:
+    """The topk highest scores (ties to the earlier group), ascending; all
+    groups when there are topk or fewer."""
+    order = sorted(range(len(scores)), key=lambda m: (-scores[m], m))
+    return sorted(order[:topk])
 
 
 def selected_columns(pt: _tree.PackedTrees, r: int, qi: np.ndarray, ki: np.ndarray, g: int, topk: int,
-                     kvh: int, decide_fp32: bool = False) -> List[int]:
+                     kvh: int, groups: Optional[Sequence[int]] = None) -> List[int]:
     """Packed columns row r attends to for KV head kvh: the members of its
-    top-k complete groups (by indexer score) and its causal tail.  With
-    decide_fp32 the scores that decide the selection are taken in fp32 (see
-    _scores_fp32) rather than fp64."""
+    top-k complete groups (by fp64 indexer score), or of the given `groups`,
+    followed by its causal tail."""
     hist = history(pt, r)
     p = len(hist) - 1
     n_complete = (p + 1) // g
     tail = hist[n_complete * g:]
     if n_complete == 0:
         return tail
-    if decide_fp32:
-        scores = _scores_fp32(qi[r, kvh], [ki[hist[m * g:(m + 1) * g], kvh] for m in range(n_complete)])
-    else:
-        keys = np.stack([np.mean(np.asarray(ki[hist[m * g:(m + 1) * g], kvh], dtype=np.float64), axis=0)
-                         for m in range(n_complete)])
-        scores = keys @ np.asarray(qi[r, kvh], dtype=np.float64)
-    order = sorted(range(n_complete), key=lambda m: (-scores[m], m))
-    chosen = sorted(order[:topk])
+    chosen = top_groups(group_scores(pt, r, qi, ki, g, kvh), topk) if groups is None else sorted(groups)
     cols = [c for m in chosen for c in hist[m * g:(m + 1) * g]]
     return cols + tail
 
 
 def sparse_tree_attention(pt: _tree.PackedTrees, q: np.ndarray, k: np.ndarray, v: np.ndarray, qi: np.ndarray,
                           ki: np.ndarray, g: int, topk: int, theta: float, scale: Optional[float] = None,
-                          rows: Optional[Iterable[int]] = None, decide_fp32: bool = False) -> np.ndarray:
+                          rows: Optional[Iterable[int]] = None,
+                          selections: Optional[Mapping[Tuple[int, int], Sequence[int]]] = None) -> np.ndarray:
     """O[r, h] over the selected columns of row r for KV head h // (Hq / Hkv).
     q [N, Hq, d], k/v [N, Hkv, d] (RoPE applied here at semantic positions),
-    qi/ki [N, Hkv, di] indexer features.  Returns [len(rows), Hq, d].  The
-    attention is fp64; decide_fp32 takes only the selection's scores in fp32,
-    the precision in which a GPU kernel makes that integer decision."""
+    qi/ki [N, Hkv, di] indexer features.  Returns [len(rows), Hq, d], fp64.
+    `selections` maps (row, kvh) to a group list used instead of the fp64
+    top-k (a selection shown elsewhere to be a valid top-k)."""
     if g < 1 or topk < 1:
         raise ValueError("group size and top-k must be positive")
     N, Hq, d = q.shape
@@ -110,7 +106,8 @@ def sparse_tree_attention(pt: _tree.PackedTrees, q: np.ndarray, k: np.ndarray, v
     out = np.zeros((len(rows), Hq, d))
     for n, r in enumerate(rows):
         for kvh in range(Hkv):
-            cols = selected_columns(pt, r, qi, ki, g, topk, kvh, decide_fp32)
+            given = None if selections is None else selections.get((r, kvh))
+            cols = selected_columns(pt, r, qi, ki, g, topk, kvh, given)
             for h in range(kvh * G, (kvh + 1) * G):
                 out[n, h] = _attn._softmax_attend(qr[r, h], kr[cols, kvh], vv[cols, kvh], scale)
     return out

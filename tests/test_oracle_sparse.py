@@ -103,24 +103,39 @@ def test_tail_bypasses_top_k():
         assert r in cols or (r + 1) % 3 == 0
 
 
-def test_fp32_decision_agrees_with_fp64_away_from_ties():
-    """Taking the scores in fp32 changes no selection unless two scores are
-    within fp32 rounding of each other (random features: none here)."""
-    pt = T.pack([40], [5], [3], [10, 25, 39], 4, True)
-    q, k, v, qi, ki = _inputs(pt.num_rows, 2, 1, 8, 16, 7)
-    for r in range(pt.num_rows):
-        assert SP.selected_columns(pt, r, qi, ki, 4, 2, 0) == SP.selected_columns(pt, r, qi, ki, 4, 2, 0, True)
-
-
-def test_exact_ties_pick_the_earliest_groups_in_both_precisions():
+def test_exact_ties_pick_the_earliest_groups():
     pt = T.pack([33], [0], [1], [20], 4, True)
     N = pt.num_rows
     zeros = np.zeros((N, 1, 8))
     for r in (10, 32, 33, 36):
-        for fp32 in (False, True):
-            cols = SP.selected_columns(pt, r, zeros, zeros, 4, 2, 0, fp32)
-            hist = SP.history(pt, r)
-            p = len(hist) - 1
-            nc = (p + 1) // 4
-            expect = hist[:min(nc, 2) * 4] + hist[nc * 4:]
-            assert cols == expect, (r, fp32)
+        cols = SP.selected_columns(pt, r, zeros, zeros, 4, 2, 0)
+        hist = SP.history(pt, r)
+        p = len(hist) - 1
+        nc = (p + 1) // 4
+        expect = hist[:min(nc, 2) * 4] + hist[nc * 4:]
+        assert cols == expect, r
+
+
+def test_top_groups_order_and_count():
+    s = np.array([0.5, 2.0, -1.0, 2.0, 0.7])
+    assert SP.top_groups(s, 2) == [1, 3]          # the two best, ascending
+    assert SP.top_groups(s, 3) == [1, 3, 4]
+    assert SP.top_groups(np.array([1.0, 1.0, 1.0]), 2) == [0, 1]   # ties to the earlier group
+    assert SP.top_groups(s, 9) == [0, 1, 2, 3, 4]  # k above the count: every group
+
+
+def test_group_scores_are_query_dot_member_mean():
+    """Brute force for one branch row: each complete group's score is the
+    indexer query dotted with the mean of its members' keys, the members
+    being the row's own history (trunk through the anchor, then its branch)."""
+    pt = T.pack([10], [2], [2], [5, 8], 4, True)
+    rng = np.random.default_rng(3)
+    qi = rng.standard_normal((pt.num_rows, 1, 6))
+    ki = rng.standard_normal((pt.num_rows, 1, 6))
+    r = 10 + 4 + 2            # y_{1,3} of the branch at anchor 8: history x_0..x_8, y_{1,1}, y_{1,2}, y_{1,3}
+    hist = list(range(0, 9)) + [14, 15, 16]
+    assert SP.history(pt, r) == hist
+    got = SP.group_scores(pt, r, qi, ki, 3, 0)
+    want = [sum(qi[r, 0, e] * sum(ki[hist[m * 3 + j], 0, e] for j in range(3)) / 3 for e in range(6))
+            for m in range(4)]
+    assert np.allclose(got, want, rtol=0, atol=1e-12)

@@ -11,15 +11,20 @@
 // members' indexer keys; the score is the indexer query dotted with it; the
 // k best per KV head are taken, ties to the earlier group.
 //
-//   sparse_gkey_kernel -- the keys of every complete trunk group (shared by
-//                         all rows of the tree): fp32 mean in position order;
-//   sparse_attn_kernel -- one warp per (row, KV head): scores of the row's
-//                         complete groups (trunk keys from the table, keys of
-//                         groups holding branch tokens formed on the spot, in
-//                         the same order), top-k by repeated warp argmax,
-//                         then an fp32 online softmax over the chosen groups'
-//                         members and the tail for each query head of the KV
-//                         group (RoPE applied beforehand by the RoPE kernel).
+//   sparse_gkey_kernel   -- the keys of every complete trunk group (shared by
+//                           all rows of the tree): fp32 mean in position order;
+//   sparse_select_kernel -- one warp per (row, KV head): scores of the row's
+//                           complete groups (trunk keys from the table, keys of
+//                           groups holding branch tokens formed on the spot, in
+//                           the same order), top-k by repeated warp argmax; it
+//                           writes the chosen groups as an ascending list and
+//                           as bits of the row's selection words;
+//   attention            -- for g a multiple of 64, the tcgen05 tree-attention
+//                           kernel in its sparse mode (tensor cores; every
+//                           query head of the KV group shares the selection);
+//                           otherwise sparse_attn_kernel, one warp per (row,
+//                           KV head) with an fp32 online softmax over the
+//                           chosen groups' members and the tail.
 // Scores are sequential fp32 sums and fused multiply-adds in a fixed order,
 // so the selection is reproducible.
 #include <cuda_bf16.h>
@@ -87,7 +92,7 @@ __global__ void sparse_gkey_kernel(const SparseArgs s) {
   s.gkey[((long long)gidx * s.Hkv + kvh) * s.di + e] = sum / (float)s.g;
 }
 
-__global__ void __launch_bounds__(32 * kSpWarps) sparse_attn_kernel(const SparseArgs s) {
+__global__ void __launch_bounds__(32 * kSpWarps) sparse_select_kernel(const SparseArgs s) {
   __shared__ float score[kSpWarps][kSpMaxGroups];
   __shared__ int sel[kSpWarps][kSpMaxTopk];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -98,7 +103,6 @@ __global__ void __launch_bounds__(32 * kSpWarps) sparse_attn_kernel(const Sparse
   const RowPlace x = place_row(s, r);
   const int t = x.t;
   const int nc = (x.p + 1) / s.g;  // complete groups
-  const int tail0 = nc * s.g;
   const __nv_bfloat16* qi = static_cast<const __nv_bfloat16*>(s.qi) + (r * s.Hkv + kvh) * s.di;
   const __nv_bfloat16* ki = static_cast<const __nv_bfloat16*>(s.ki);
 
@@ -163,7 +167,37 @@ __global__ void __launch_bounds__(32 * kSpWarps) sparse_attn_kernel(const Sparse
   }
   __syncwarp();
 
-  // ---- attention over the chosen groups' members and the tail
+  // ---- outputs: the ascending list (-1 past K) and the selection words
+  int32_t* list = s.sel_list + item * s.topk;
+  for (int i = lane; i < s.topk; i += 32) {
+    const int v = i < K ? sel[w][i] : -1;
+    list[i] = v;
+    if (s.sel_out) s.sel_out[item * s.topk + i] = v;
+  }
+  uint32_t* words = s.sel_mask + item * s.sel_words;
+  for (int wd = lane; wd < s.sel_words; wd += 32) {
+    uint32_t bits = 0;
+    for (int i = 0; i < K; ++i) {
+      const int m = sel[w][i];
+      if ((m >> 5) == wd) bits |= 1u << (m & 31);
+    }
+    words[wd] = bits;
+  }
+}
+
+// fp32 SIMT attention over the chosen groups' members and the tail (group
+// sizes that are not a multiple of 64).
+__global__ void __launch_bounds__(32 * kSpWarps) sparse_attn_kernel(const SparseArgs s) {
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long item = (long long)blockIdx.x * kSpWarps + w;
+  if (item >= s.N * s.Hkv) return;
+  const long long r = item / s.Hkv;
+  const int kvh = (int)(item % s.Hkv);
+  const RowPlace x = place_row(s, r);
+  const int nc = (x.p + 1) / s.g;
+  const int tail0 = nc * s.g;
+  const int K = nc < s.topk ? nc : s.topk;
+  const int32_t* sel = s.sel_list + item * s.topk;
   const int ncols = K * s.g + (x.p + 1 - tail0);
   const __nv_bfloat16* rq = static_cast<const __nv_bfloat16*>(s.rq);
   const __nv_bfloat16* rk = static_cast<const __nv_bfloat16*>(s.rk);
@@ -176,7 +210,7 @@ __global__ void __launch_bounds__(32 * kSpWarps) sparse_attn_kernel(const Sparse
     for (int i = 0; i < 4; ++i) qv[i] = ldbf(rq + (r * s.Hq + h) * kSpD + lane * 4 + i) * s.scale_log2;
     float mx = -INFINITY, l = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
     for (int c = 0; c < ncols; ++c) {
-      const int q = c < K * s.g ? sel[w][c / s.g] * s.g + c % s.g : tail0 + (c - K * s.g);
+      const int q = c < K * s.g ? sel[c / s.g] * s.g + c % s.g : tail0 + (c - K * s.g);
       const long long col = hist_row(x, q);
       const __nv_bfloat16* kp = rk + (col * s.Hkv + kvh) * kSpD + lane * 4;
       float d = 0.f;
@@ -206,6 +240,15 @@ size_t sparse_group_keys(const TreeParams& tp, int g) {
   return n;
 }
 
+int sparse_selection_words(const TreeParams& tp, int g) {
+  int most = 0;
+  for (int t = 0; t < tp.num_trees; ++t) {
+    const int n = (tp.trunk_len[t] + tp.rows_per_branch) / g;  // complete groups of the deepest row
+    if (n > most) most = n;
+  }
+  return (most + 31) / 32 > 0 ? (most + 31) / 32 : 1;
+}
+
 cudaError_t launch_sparse_attention(SparseArgs s, cudaStream_t stream) {
   int off = 0;
   for (int t = 0; t < s.tp.num_trees; ++t) {
@@ -221,7 +264,31 @@ cudaError_t launch_sparse_attention(SparseArgs s, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
   }
   const long long items = s.N * s.Hkv;
-  sparse_attn_kernel<<<(unsigned)((items + kSpWarps - 1) / kSpWarps), 32 * kSpWarps, 0, stream>>>(s);
+  const unsigned blocks = (unsigned)((items + kSpWarps - 1) / kSpWarps);
+  sparse_select_kernel<<<blocks, 32 * kSpWarps, 0, stream>>>(s);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (s.g % 64 == 0) {
+    AttnArgs a;
+    a.q = s.rq;
+    a.k = s.rk;
+    a.v = s.v;
+    a.out = s.out;
+    a.N = s.N;
+    a.Hq = s.Hq;
+    a.Hkv = s.Hkv;
+    a.d = kSpD;
+    a.scale = s.scale;
+    a.pos = s.pos;
+    a.trunk_limit = s.trunk_limit;
+    a.anc_bits = s.anc_bits;
+    a.meta = s.meta;
+    a.num_tiles = s.num_tiles;
+    a.status = s.status;
+    SparseSel sel{s.sel_mask, s.sel_words, s.g};
+    return launch_tree_attention_sm100(a, stream, &sel);
+  }
+  sparse_attn_kernel<<<blocks, 32 * kSpWarps, 0, stream>>>(s);
   return cudaGetLastError();
 }
 

@@ -27,6 +27,15 @@
 //  * TMEM: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512) fp32 columns;
 //    P_t occupies the first 64 columns of S_t as packed bf16 pairs.
 //
+// Sparse mode (the listing's Fig 4: attention reads the selected indexer
+// groups plus the causal tail) runs the same pipeline with one more per-row
+// filter: a column of the row's history is kept only when its semantic
+// position lies in the row's causal tail or in a complete group the indexer
+// selected for the row and KV head (bit m of the row's selection words).  With
+// the group size g a multiple of 64, each 64-column half of a trunk block lies
+// in one group, so the filter costs one flag per half-block; branch columns
+// are filtered once per row into the row's ancestor bits.
+//
 // All waits are bounded (see ptx.cuh); a wait that gives up sets
 // SPECOPD_FLAG_TIMEOUT, and the CTA drains its copies and MMAs, frees TMEM
 // and returns.
@@ -74,7 +83,14 @@ struct Params {
   int items_per_pair;     // work items per pair of tiles (2k, 2k+1)
   float scale_log2;
   int32_t* status;
+  // sparse mode only: per (row, KV head) sel_words words, bit m set iff
+  // complete group m of the row's history is selected; g % 64 == 0
+  const uint32_t* sel_mask;
+  int sel_words;
+  int g;
 };
+
+__device__ __forceinline__ bool group_selected(const uint32_t* w, int m) { return (w[m >> 5] >> (m & 31)) & 1u; }
 
 // bounded wait used only to drain in-flight work before exit: ignores the
 // abort flag, still gives up after the time limit.
@@ -95,6 +111,7 @@ __device__ __forceinline__ int block_col(const specopd_tile_meta& m, int n_trunk
   return j < n_trunk ? m.tree_base + j * kBN : m.br_lo + (j - n_trunk) * kBN;
 }
 
+template <bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
     tree_attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -283,11 +300,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = r < p.meta[tile_s[t]].row_end;
       int lim = m.tree_base, bstart = 0;
       uint64_t bits = 0;
+      int tail0 = 0;                  // sparse: first position of the causal tail
+      const uint32_t* selw = nullptr;  // sparse: the row's selection words
       if (valid) {
         const int tl = p.trunk_limit[r];
+        const int prow = p.pos[r];
         lim = m.tree_base + tl;
-        bstart = r - (p.pos[r] - tl) + 1;
+        bstart = r - (prow - tl) + 1;
         bits = p.anc_bits[r];
+        if (kSparse) {
+          tail0 = (prow + 1) / p.g * p.g;
+          selw = p.sel_mask + ((long long)r * p.Hkv + kvh) * p.sel_words;
+          // branch sample k (position tl + k) stays visible only if its group is selected or in the tail
+          uint64_t keep = 0;
+          for (int k = 1; k <= prow - tl; ++k) {
+            const int q = tl + k;
+            if (q >= tail0 || group_selected(selw, q / p.g)) keep |= 1ull << (k - 1);
+          }
+          bits &= keep;
+        }
       }
       const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
       const uint32_t s_col = t * 128;
@@ -307,6 +338,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         float* s = reinterpret_cast<float*>(sr);
         const int c0 = block_col(m, n_trunk, j);
         const bool trunk = j < n_trunk;
+        if (kSparse && trunk) {
+          // positions of this block: c0 - tree_base + [0, 128); a half below the
+          // tail lies in one complete group (g % 64 == 0, blocks 128-aligned)
+          const int q0 = c0 - m.tree_base;
+          if (!(q0 >= tail0 || group_selected(selw, q0 / p.g))) {
+#pragma unroll
+            for (int e = 0; e < 64; ++e) s[e] = -INFINITY;
+          }
+          if (!(q0 + 64 >= tail0 || group_selected(selw, (q0 + 64) / p.g))) {
+#pragma unroll
+            for (int e = 64; e < 128; ++e) s[e] = -INFINITY;
+          }
+        }
         if (!(trunk && c0 + kBN <= m.trunk_full)) {
           if (trunk) {
 #pragma unroll
@@ -333,7 +377,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_new = fmaxf(m_use, mx * p.scale_log2);
         float corr = 1.f;
         bool rescale = false;
-        if (m_use == -INFINITY || m_new > m_use + kRescaleLog2) {
+        // (a fully masked block before any visible column leaves m_use at -inf)
+        if ((m_use == -INFINITY && m_new != -INFINITY) || m_new > m_use + kRescaleLog2) {
           corr = ex2(m_use - m_new);
           m_use = m_new;
           rescale = j > 0;
@@ -423,7 +468,7 @@ bool make_map(CUtensorMap* tm, const void* ptr, int64_t N, int H) {
 
 }  // namespace
 
-cudaError_t launch_tree_attention_sm100(const AttnArgs& a, cudaStream_t stream) {
+cudaError_t launch_tree_attention_sm100(const AttnArgs& a, cudaStream_t stream, const SparseSel* sel) {
   if (a.num_tiles == 0) return cudaSuccess;
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, a.q, a.N, a.Hq) || !make_map(&tk, a.k, a.N, a.Hkv) || !make_map(&tv, a.v, a.N, a.Hkv))
@@ -442,12 +487,15 @@ cudaError_t launch_tree_attention_sm100(const AttnArgs& a, cudaStream_t stream) 
   p.items_per_pair = p.Hkv * (2 * p.pairs + 2 * (p.G & 1));
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.status = a.status;
+  p.sel_mask = sel ? sel->mask : nullptr;
+  p.sel_words = sel ? sel->words : 0;
+  p.g = sel ? sel->g : 0;
   const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e =
-      cudaFuncSetAttribute(tree_attn_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = sel ? tree_attn_sm100_kernel<true> : tree_attn_sm100_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long long grid = (long long)((a.num_tiles + 1) / 2) * p.items_per_pair;
-  tree_attn_sm100_kernel<<<(unsigned)grid, kThreads, smem, stream>>>(tq, tk, tv, p);
+  kern<<<(unsigned)grid, kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
