@@ -11,9 +11,12 @@ loss, sum_b W) scored per second.
 The default workload is the largest single-GPU one ("scale27b": trunk 32,768,
 512 branches x 16 samples, 40/8 heads of 128, vocabulary 248,320).
 
-N > 1 runs under torchrun: each rank scores its own batch (weak scaling; the
-trees are independent problems, so the data path has no collective), the
-timed region is bracketed by barriers and the slowest rank's time is used.
+N > 1 runs under torchrun and splits one logical batch over the ranks (strong
+scaling): each rank scores a contiguous run of the packed query tiles,
+balanced by visible (row, column) pairs, and a contiguous share of whole
+branches for the overlap / loss / gradient, normalised by the whole batch's
+prediction count; one NCCL all-reduce per step sums the ranks' loss shares.
+The timed region is bracketed by barriers and the slowest rank's time is used.
 `--impl reference` times the fp64 CPU oracle on the host cores instead (rank 0).
 """
 from __future__ import annotations
@@ -244,7 +247,9 @@ def config_dict(case, figs, workload: int, seed: int, world: int) -> dict:
     return {"workload": SY.WORKLOADS[workload], "supervised_tokens_per_step": figs["R"],
             "packed_rows": case.num_rows, "visible_pairs": figs["pairs"], "seed": seed,
             "l2": "inputs larger than L2 (%.2f GB per step > 126 MB); each step streams them from HBM" % (in_bytes / 1e9),
-            "parallelism": f"dp{world} (independent tree batches per rank)"}
+            "parallelism": ("1 GPU" if world == 1 else
+                            f"{world} GPUs, one batch: query tiles split by visible pairs, whole branches split, "
+                            "loss shares summed by one NCCL all-reduce per step")}
 
 
 # ----------------------------------------------------------------- GPU run
@@ -267,8 +272,17 @@ def run_gpu(args):
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
 
-    case = SY.make_workload(args.workload, seed=args.seed + rank, workers=min(8, os.cpu_count() or 1))
+    # the same logical batch on every rank; each scores its share of it
+    case = SY.make_workload(args.workload, seed=args.seed, workers=min(8, os.cpu_count() or 1))
     figs = case_figures(case)
+    nb = int(sum(case.num_branches))
+    count = float(nb * case.W)  # the whole batch's predictions, known on the host
+    costs = PAR.tile_costs(case.trunk_len, case.num_branches, case.anchors, case.W, case.pack_terminal)
+    t0, t1 = PAR.split_tiles(costs, world, rank)
+    trows = PAR.tile_rows(case.trunk_len, case.num_branches, case.W, case.pack_terminal)
+    r0, r1 = (int(trows[t0, 0]), int(trows[t1 - 1, 1])) if t1 > t0 else (0, 0)
+    b0, b1 = PAR.shard_range(nb, world, rank)
+    split = world > 1
     st = ScoringStep(case.trunk_len, case.prompt_len, case.num_branches, case.W, case.Hq, case.Hkv, case.d,
                      torch.bfloat16 if case.dtype == "bf16" else torch.float32, case.vocab, device=dev,
                      pack_terminal=case.pack_terminal, theta=case.theta)
@@ -285,10 +299,17 @@ def run_gpu(args):
         st.build_mask(stream)
         if i is not None:
             marks[i][1].record(stream)
-        st.attention(stream)
+        if split:
+            st.attention(stream, tiles=(t0, t1), rows=(r0, r1))
+        else:
+            st.attention(stream)
         if i is not None:
             marks[i][2].record(stream)
-        st.overlap(stream)
+        if split:
+            st.overlap(stream, count=count, branches=(b0, b1))
+            dist.all_reduce(st.loss)  # sum of the ranks' L_r; L = sum - (world - 1)
+        else:
+            st.overlap(stream)
         if i is not None:
             marks[i][3].record(stream)
 
@@ -320,21 +341,25 @@ def run_gpu(args):
     elapsed_ms = PAR.max_time_ms(elapsed_ms, device=dev)  # slowest rank (identity at N = 1)
 
     # ---- end to end through the public API with host buffers
+    # each rank copies what its share reads: every key/value row, its query
+    # rows, its branches' logits; and reads back the loss and its alphas
     pin = lambda x, dt: (torch.from_numpy(x).view(torch.bfloat16) if dt == "bf16" else torch.from_numpy(x)).pin_memory()
-    h_in = [torch.from_numpy(case.anchors).pin_memory(), pin(case.q, case.dtype), pin(case.k, case.dtype),
-            pin(case.v, case.dtype), pin(case.draft, case.dtype), pin(case.teacher, case.dtype)]
-    d_in = [st.anchors, st.q, st.k, st.v, st.draft, st.teacher]
+    pr0, pr1 = (r0, r1) if split else (0, case.num_rows)
+    lr0, lr1 = (b0 * case.W, b1 * case.W) if split else (0, st.R)
+    h_in = [torch.from_numpy(case.anchors).pin_memory(), pin(case.q[pr0:pr1], case.dtype), pin(case.k, case.dtype),
+            pin(case.v, case.dtype), pin(case.draft[lr0:lr1], case.dtype), pin(case.teacher[lr0:lr1], case.dtype)]
+    d_in = [st.anchors, st.q[pr0:pr1], st.k, st.v, st.draft[lr0:lr1], st.teacher[lr0:lr1]]
     h_loss = torch.empty(1, dtype=torch.float32).pin_memory()
-    h_alpha = torch.empty(st.R, dtype=torch.float32).pin_memory()
+    h_alpha = torch.empty(max(lr1 - lr0, 1), dtype=torch.float32).pin_memory()
     h2d = sum(x.numel() * x.element_size() for x in h_in)
-    d2h = h_loss.numel() * 4 + h_alpha.numel() * 4
+    d2h = h_loss.numel() * 4 + (lr1 - lr0) * 4
 
     def e2e_step():
         for h, d in zip(h_in, d_in):
             d.copy_(h, non_blocking=True)
-        st.run(stream)
+        step()
         h_loss.copy_(st.loss, non_blocking=True)
-        h_alpha.copy_(st.alpha[:st.R], non_blocking=True)
+        h_alpha[:lr1 - lr0].copy_(st.alpha[lr0:lr1], non_blocking=True)
 
     Ke = min(K, 50 if h2d < 2e9 else 10)  # the host copies dominate; a few steps are plenty
     for _ in range(max(1, Wm // 2)):
@@ -350,6 +375,9 @@ def run_gpu(args):
     torch.cuda.synchronize()
     e2e_ms = e_start.elapsed_time(e_end)
     e2e_ms = PAR.max_time_ms(e2e_ms, device=dev)
+    if split:  # bytes moved per step by all ranks together
+        h2d = int(PAR.global_count(h2d, device=dev))
+        d2h = int(PAR.global_count(d2h, device=dev))
     status = st.check_status()
 
     peaks = load_peaks()
@@ -384,11 +412,11 @@ def run_gpu(args):
                 "peak_source": f"{peaks['source']} ({peak_src})"}
     if dom == "tree_attention":
         roofline["frac_burst"] = kd["frac_burst"]
-    tokens = figs["R"] * world
+    tokens = figs["R"]  # one logical batch, whatever the number of ranks
     value = tokens * K / (elapsed_ms * 1e-3)
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": Wm,
-        "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
         "dtype": case.dtype, "data": "synthetic (seeded; no datasets or weights)",
         "config": config_dict(case, figs, args.workload, args.seed, world),
         "roofline": roofline,
@@ -396,9 +424,13 @@ def run_gpu(args):
         "clocks": clk,
         "e2e": {"value": tokens * Ke / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / Ke, "steps": Ke},
-        "gpu_launches": 4 * K,  # mask, RoPE, attention, fused overlap (statistics + gradient)
+        # mask, RoPE (two calls when split: query rows, key rows), attention, fused overlap
+        "gpu_launches": (5 if split else 4) * K,
         "device_status": status,
     }
+    if split:
+        out["loss"] = st.loss.item() - (world - 1)
+        out["shard"] = {"tiles": [t0, t1], "rows": [r0, r1], "branches": [b0, b1]}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(case)
     if world == 1 and not args.no_lm_head:
@@ -588,7 +620,9 @@ def sparse_measure(dev, peaks, seed: int) -> dict:
     (not part of the step), on the shape of the GPU parity test's full-size
     case: the 8B-style tree (T 4,096, 64 branches x W 16), 32/8 heads, d 128,
     64-token groups, top-8, 64-wide indexer features.  Useful FLOPs count the
-    attended (row, column) pairs, 4 d per pair and query head."""
+    attended (row, column) pairs, 4 d per pair and query head; the tensor-core
+    kernel executes the tree's visible key blocks with the unselected groups
+    masked (executed FLOPs count every visible pair)."""
     import torch
     import synthetic as SY
     from tree_attention_masked_b200 import specopd as S
@@ -608,10 +642,10 @@ def sparse_measure(dev, peaks, seed: int) -> dict:
     S.specopd_build_tree_mask(trees, pos, trunk_limit, branch_of, anc_bits, pred_rows, cu_rows, tile_meta, status)
     q, k, v, qi, ki = bf(case.q), bf(case.k), bf(case.v), bf(case.qi), bf(case.ki)
     out = torch.empty(N, 32, 128, dtype=torch.bfloat16, device=dev)
-    ws = torch.empty(S.specopd_sparse_workspace_bytes(trees, 32, 8, 64, g), dtype=torch.uint8, device=dev)
+    ws = torch.empty(S.specopd_sparse_workspace_bytes(trees, 32, 8, 64, g, topk), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    call = lambda: S.specopd_sparse_tree_attention(trees, q, k, v, qi, ki, out, pos, g, topk, 1e4, ws, status,
-                                                   stream=stream)
+    call = lambda: S.specopd_sparse_tree_attention(trees, q, k, v, qi, ki, out, pos, trunk_limit, anc_bits,
+                                                   tile_meta, g, topk, 1e4, ws, status, stream=stream)
     for _ in range(3):
         call()
     torch.cuda.synchronize()
@@ -624,19 +658,22 @@ def sparse_measure(dev, peaks, seed: int) -> dict:
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / n
     # attended pairs: per row, its chosen groups' members and its tail
-    T0, P0, B0 = 4096, 1024, 64
+    T0 = 4096
     pairs = 0
+    vis = 0
     for r in range(N):
         p = r if r < T0 else int(case.anchors[(r - T0) // W]) + 1 + (r - T0) % W
         nc = (p + 1) // g
         pairs += min(nc, topk) * g + (p + 1 - nc * g)
+        vis += p + 1
     flops = 4.0 * 128 * 32 * pairs
     achieved = flops / (ms * 1e-3) / 1e12
-    return {"bound": "latency (SIMT: one warp per row and KV head)", "ms": ms, "achieved": achieved,
+    return {"bound": "tensor (masked tree attention over the selected groups)", "ms": ms, "achieved": achieved,
             "unit": "TFLOP/s", "peak": peaks["bf16"], "frac": achieved / peaks["bf16"], "useful_flops": flops,
-            "attended_pairs": pairs, "device_status": status.item(),
+            "attended_pairs": pairs, "visible_pairs": vis,
+            "executed_tflops": 4.0 * 128 * 32 * vis / (ms * 1e-3) / 1e12, "device_status": status.item(),
             "shape": "T 4096, B 64 x W 16, 32/8 heads, d 128, groups of 64, top-8, indexer width 64, bf16",
-            "launches": 3}
+            "launches": 4}
 
 
 def main():

@@ -150,7 +150,10 @@ int specopd_build_tree_mask(const specopd_tree_desc* desc, int32_t* pos, int32_t
  * a_b + i, not its packed offset.  Element k of each head pairs with element
  * k + d/2 and both rotate by pos[r] * theta^(-2k/d); the angle is formed in
  * fp64.  q [N, Hq, d] -> q_out, k [N, Hkv, d] -> k_out (same dtype, may not
- * alias the inputs).  d even, d <= 256.
+ * alias the inputs).  Hq or Hkv may be 0 (that tensor is skipped and its two
+ * pointers may be null), so a caller can rotate a range of query rows and all
+ * key rows with two calls.  d a multiple of 4 with 4 <= d <= 256 (the kernel
+ * moves each half-head in 2-element pairs); other d return SPECOPD_ERR_SHAPE.
  */
 int specopd_rope(const void* q, const void* k, void* q_out, void* k_out, specopd_dtype dtype, int64_t N,
                  int Hq, int Hkv, int d, const int32_t* pos, float theta, specopd_stream_t stream);
@@ -169,8 +172,13 @@ size_t specopd_attention_workspace_bytes(specopd_dtype dtype, int64_t N, int Hq,
  * q [N, Hq, d], k and v [N, Hkv, d], out [N, Hq, d]: device, dtype `dtype`,
  * 16-byte aligned.  rope_theta > 0 rotates q and k at pos first (into the
  * workspace); rope_theta <= 0 takes q and k as already rotated.
- * softmax_scale <= 0 means 1/sqrt(d).  pos, trunk_limit, anc_bits, tile_meta:
- * outputs of specopd_build_tree_mask for the same trees.
+ * softmax_scale <= 0 means 1/sqrt(d).  pos, trunk_limit, anc_bits: outputs
+ * of specopd_build_tree_mask for the same trees.  tile_meta: num_tiles of its
+ * tile records, all of them or any contiguous run (tile_meta offset by the
+ * run's first tile); only the rows of the given tiles are written to out, so
+ * ranks that split a batch by query rows each pass their own run (q rows
+ * outside the run are not read; every key row the run's rows see must be
+ * present).  num_tiles == 0 does nothing.
  * bf16 with d = 128 runs the tcgen05/TMEM kernel; fp32 (any d) and bf16 with
  * other d (multiple of 32, <= 256) run a SIMT kernel with fp32 arithmetic.
  * Accumulation is fp32 in both.
@@ -244,6 +252,50 @@ int specopd_tv_overlap_e2e(const void* draft, const void* teacher, specopd_dtype
                            double count, float* alpha, float* loss, float* grad_draft, int64_t ld_grad,
                            void* workspace, size_t workspace_bytes, int32_t* status, specopd_stream_t stream);
 
+/*
+ * specopd_diag_overlap_wait_timeout -- failure-detection diagnostic: makes a
+ * bounded in-kernel wait of the fused overlap kernel run out on purpose.
+ *
+ * Launches the bf16 kernel of specopd_tv_overlap_e2e (cooperative, one CTA per
+ * SM) with the gradient of every row requested but no row's statistics, so
+ * no branch's dL/dalpha is ever published: every gradient unit waits for a
+ * publication that never comes.  The wait gives up after its time limit
+ * (about one second), ORs SPECOPD_FLAG_TIMEOUT into *status, raises the CTA's
+ * abort flag so its other waits stop, and the kernel returns; no copy is in
+ * flight at that point and the stream stays usable.  grad_draft is left
+ * unwritten.  Arguments as specopd_tv_overlap_e2e (bf16 only, grad_draft and
+ * workspace required, num_branches >= 1).
+ */
+int specopd_diag_overlap_wait_timeout(const void* draft, const void* teacher, int64_t rows, int64_t V,
+                                      int64_t ld_draft, int64_t ld_teacher, int64_t num_branches, int W,
+                                      float* grad_draft, int64_t ld_grad, void* workspace, size_t workspace_bytes,
+                                      int32_t* status, specopd_stream_t stream);
+
+/*
+ * specopd_tree_causal_conv -- short causal convolution along each packed row's
+ * own history.
+ *
+ * SpecOPD (thelatestinai.com listing), Fig 5: the causal convolution of the
+ * GDN branch path follows branch ancestry, so a branch token's window holds
+ * its own history (the trunk through its anchor, then its branch's earlier
+ * samples), never its packed neighbours or a sibling's tokens.  Reading (the
+ * figure prints no formula): a depthwise convolution of width Kw,
+ *   out[r, c] = act(bias[c] + sum_{j<Kw} weight[c, j] * x[h_j(r), c]),
+ * h_j(r) the row j steps back in r's history (j = 0: r itself), zero before
+ * the start of the history; act is the identity (silu = 0) or SiLU
+ * u / (1 + e^-u) (silu = 1).  fp32 arithmetic.
+ *
+ * x, out [N, C]: device, dtype `dtype` (out in the same dtype), row-major,
+ * 16-byte aligned, C a multiple of 8 (bf16) or 4 (fp32); a feature tensor
+ * [N, H, d] is passed with C = H d.  weight [C, Kw] and bias [C] (nullable):
+ * device fp32.  1 <= Kw <= 8.  pos, trunk_limit, cu_rows (num_trees + 1
+ * entries): outputs of specopd_build_tree_mask for the same trees.  out may
+ * not alias x.  Returns SPECOPD_ERR_* before anything is enqueued.
+ */
+int specopd_tree_causal_conv(const void* x, void* out, specopd_dtype dtype, int64_t N, int C, const float* weight,
+                             const float* bias, int Kw, int silu, const int32_t* pos, const int32_t* trunk_limit,
+                             const int32_t* cu_rows, int num_trees, specopd_stream_t stream);
+
 /* Bytes of workspace specopd_gdn_tree needs: the fp32 trunk checkpoints,
  * (sum over trees of T / 64) * H * 128 * 128 * 4 rounded up to 256 (0 for an
  * invalid description). */
@@ -280,8 +332,10 @@ int specopd_gdn_tree(const specopd_tree_desc* desc, const void* q, const void* k
                      void* workspace, size_t workspace_bytes, int32_t* status, specopd_stream_t stream);
 
 /* Bytes of workspace specopd_sparse_tree_attention needs: rotated Q and K
- * (bf16) and the trunk group keys (fp32), each rounded up to 256 bytes. */
-size_t specopd_sparse_workspace_bytes(const specopd_tree_desc* desc, int Hq, int Hkv, int di, int g);
+ * (bf16), the trunk group keys (fp32), the chosen groups [N][Hkv][topk]
+ * (int32) and the per-row selection words (uint32), each rounded up to 256
+ * bytes (0 for an invalid description). */
+size_t specopd_sparse_workspace_bytes(const specopd_tree_desc* desc, int Hq, int Hkv, int di, int g, int topk);
 
 /*
  * specopd_sparse_tree_attention -- sparse attention with branch-consistent
@@ -299,19 +353,28 @@ size_t specopd_sparse_workspace_bytes(const specopd_tree_desc* desc, int Hq, int
  * sums, fused multiply-adds); the k best per KV head, ties to the earlier
  * group; attention as specopd_tree_attention (rotate-half RoPE at `pos`,
  * scale softmax_scale or 1/sqrt(d) when <= 0) over the chosen members and the
- * tail, fp32 online softmax.
+ * tail, fp32 accumulation.  For g a multiple of 64 the attention runs on the
+ * tensor cores (the tree-attention kernel with a per-row group filter); other
+ * g run a SIMT kernel.
  *
  * q [N, Hq, 128], k, v [N, Hkv, 128], qi, ki [N, Hkv, di] (di <= 256), out
- * [N, Hq, 128]: device bf16, row-major, 16-byte aligned; pos [N] from
- * specopd_build_tree_mask for the same description.  1 <= topk <= 64; a
- * tree's trunk plus one branch must hold at most 1,024 complete groups.
- * workspace >= specopd_sparse_workspace_bytes, 256-byte aligned.  Returns
- * SPECOPD_ERR_SHAPE / _ARG / _ALIGN / _WORKSPACE before anything is
- * enqueued, SPECOPD_ERR_CUDA if a launch fails.
+ * [N, Hq, 128]: device bf16, row-major, 16-byte aligned.  pos, trunk_limit,
+ * anc_bits, tile_meta (num_tiles entries): outputs of specopd_build_tree_mask
+ * for the same description.  1 <= topk <= 64; a tree's trunk plus one branch
+ * must hold at most 1,024 complete groups.  selected (nullable, device int32
+ * [N, Hkv, topk]) receives each (row, KV head)'s chosen complete groups in
+ * ascending order (group m covers positions m g .. m g + g - 1), -1 past the
+ * row's count (min(topk, complete groups)).  workspace >=
+ * specopd_sparse_workspace_bytes, 256-byte aligned.  Returns
+ * SPECOPD_ERR_SHAPE / _ARG / _ALIGN / _WORKSPACE before anything is enqueued,
+ * SPECOPD_ERR_CUDA if a launch fails; a timed-out in-kernel wait sets
+ * SPECOPD_FLAG_TIMEOUT in *status.
  */
 int specopd_sparse_tree_attention(const specopd_tree_desc* desc, const void* q, const void* k, const void* v,
                                   const void* qi, const void* ki, void* out, int64_t N, int Hq, int Hkv, int d,
                                   int di, int g, int topk, float rope_theta, float softmax_scale, const int32_t* pos,
+                                  const int32_t* trunk_limit, const uint64_t* anc_bits,
+                                  const specopd_tile_meta* tile_meta, int64_t num_tiles, int32_t* selected,
                                   void* workspace, size_t workspace_bytes, int32_t* status,
                                   specopd_stream_t stream);
 
@@ -369,8 +432,12 @@ int specopd_lm_head_overlap(const void* h_draft, const void* head_draft, int Hd,
  *     exceeds SPECOPD_STATIC_SCRATCH_BYTES is rejected with
  *     SPECOPD_ERR_WORKSPACE before anything is enqueued (32 MiB holds, e.g.,
  *     1,600 rows of a 151,936-entry vocabulary);
- *   - the first call on a device looks up the array's device address; make
- *     that first call before starting any stream capture;
+ *   - arguments are checked as in specopd_tv_overlap_e2e first, then the
+ *     batch against the fixed size;
+ *   - the first call on a device looks up the array's device address and the
+ *     library keeps it for the life of the process; make that first call
+ *     before starting any stream capture, and do not use this entry point on
+ *     a device after cudaDeviceReset (the kept address would be stale);
  *   - all calls on a device share the one array and it keeps the previous
  *     call's contents (the call clears what must start at zero itself), so
  *     calls that may run at the same time on the GPU -- e.g. on two streams --

@@ -20,7 +20,7 @@ Written from the definition in fp64, one row at a time.
 """
 from __future__ import annotations
 
-from typing import Optional
+from typing import Optional, Sequence
 
 import numpy as np
 
@@ -33,18 +33,20 @@ def history(pt: _tree.PackedTrees, r: int):
 
 
 def tree_causal_conv(pt: _tree.PackedTrees, x: np.ndarray, weight: np.ndarray, bias: Optional[np.ndarray] = None,
-                     silu: bool = False) -> np.ndarray:
-    """x [N, C], weight [C, Kw], bias [C] or None -> [N, C] (fp64)."""
+                     silu: bool = False, rows: Optional[Sequence[int]] = None) -> np.ndarray:
+    """x [N, C], weight [C, Kw], bias [C] or None -> [len(rows), C] (fp64; all
+    rows by default)."""
     x = np.asarray(x, dtype=np.float64)
     w = np.asarray(weight, dtype=np.float64)
     N, C = x.shape
     Kw = w.shape[1]
-    out = np.zeros((N, C))
-    for r in range(N):
+    rows = list(range(N)) if rows is None else list(rows)
+    out = np.zeros((len(rows), C))
+    for n, r in enumerate(rows):
         hist = history(pt, r)
         acc = np.zeros(C) if bias is None else np.array(bias, dtype=np.float64)
         for j in range(Kw):
             if j < len(hist):
                 acc = acc + w[:, j] * x[hist[-1 - j]]
-        out[r] = acc / (1.0 + np.exp(-acc)) if silu else acc
+        out[n] = acc / (1.0 + np.exp(-acc)) if silu else acc
     return out

@@ -425,3 +425,44 @@ def make_sparse_case(name: str, trees: Sequence[Tuple[int, int, int]], W: int, H
                       pack_terminal, np.concatenate(anc) if anc else np.zeros(0, np.int32),
                       f(_TID_SP_Q, Hq, d), f(_TID_SP_K, Hkv, d), f(_TID_SP_V, Hkv, d), f(_TID_SP_QI, Hkv, di),
                       f(_TID_SP_KI, Hkv, di))
+
+
+_TID_CV_X, _TID_CV_W, _TID_CV_B = range(130, 133)
+
+
+@dataclasses.dataclass
+class ConvCase:
+    """Features of the packed rows of some trees and a depthwise filter."""
+    name: str
+    trunk_len: List[int]
+    prompt_len: List[int]
+    num_branches: List[int]
+    W: int
+    pack_terminal: bool
+    anchors: np.ndarray   # int32 [sum B]
+    dtype: str            # "bf16" (uint16 storage) or "f32"
+    x: np.ndarray         # [N, C]
+    weight: np.ndarray    # [C, Kw] fp32
+    bias: np.ndarray      # [C] fp32
+
+    @property
+    def num_rows(self) -> int:
+        return self.x.shape[0]
+
+
+def make_conv_case(name: str, trees: Sequence[Tuple[int, int, int]], W: int, C: int, Kw: int, dtype: str = "bf16",
+                   seed: int = 0, pack_terminal: bool = True) -> ConvCase:
+    """Features x ~ N(0, 1) (drawn in fp32, rounded to bf16 once for bf16),
+    filter weights ~ N(0, 1/Kw) and bias ~ N(0, 0.1^2) in fp32; anchors as for
+    the attention workloads."""
+    rpb = W if pack_terminal else W - 1
+    N = int(sum(T + B * rpb for T, _, B in trees))
+    anc = [_draw_anchors(seed, t, P, T, B, True, False) for t, (T, P, B) in enumerate(trees)]
+    x = _normal_rows(seed, _TID_CV_X, 0, N, C, 1.0)
+    if dtype == "bf16":
+        x = bf16_round(x)
+    w = np.random.default_rng([seed, _TID_CV_W, 0, 0]).normal(0.0, 1.0 / np.sqrt(Kw), size=(C, Kw))
+    b = np.random.default_rng([seed, _TID_CV_B, 0, 0]).normal(0.0, 0.1, size=C)
+    return ConvCase(name, [t[0] for t in trees], [t[1] for t in trees], [t[2] for t in trees], W, pack_terminal,
+                    np.concatenate(anc) if anc else np.zeros(0, np.int32), dtype, x,
+                    w.astype(np.float32), b.astype(np.float32))

@@ -102,6 +102,16 @@ def test_argument_errors_before_launch(S):
     assert lib["specopd_tree_attention"](16, 16, 16, 16, 1, 8, 4, 2, 48, 1e4, 0.0, 16, 16, 16, 16, 1, 256, 1 << 20,
                                          16, None) == -2
     assert lib["specopd_rope"](16, 16, 16, 16, 1, 4, 2, 2, 6, 16, 1e4, None) == -2
+    # one of Hq / Hkv may be 0 (that tensor is skipped and may be null), not both
+    assert lib["specopd_rope"](16, 16, 16, 16, 1, 4, 0, 0, 8, 16, 1e4, None) == -2
+    assert lib["specopd_rope"](None, 16, None, 16, 1, 0, 0, 2, 8, 16, 1e4, None) == 0   # N = 0: nothing enqueued
+    assert lib["specopd_rope"](None, 16, None, 16, 1, 4, 0, 2, 8, None, 1e4, None) == -1  # pos required
+    assert lib["specopd_rope"](None, 16, None, 16, 1, 4, 2, 2, 8, 16, 1e4, None) == -1    # q needed when Hq > 0
+    # attention on a run of tile records: at most one tile per row; none is a no-op
+    assert lib["specopd_tree_attention"](16, 16, 16, 16, 1, 8, 4, 2, 128, 0.0, 0.0, 16, 16, 16, 16, 9, None, 0,
+                                         16, None) == -2
+    assert lib["specopd_tree_attention"](16, 16, 16, 16, 1, 8, 4, 2, 128, 0.0, 0.0, 16, 16, 16, 16, 0, None, 0,
+                                         16, None) == 0
     assert lib["specopd_e2e_tv_loss"](16, 2, 0, 0.0, 16, None, None) == -2
     # LM head: hidden sizes must be multiples of 64, rows = num_branches * W,
     # 16-byte aligned operands, a large enough workspace
@@ -143,28 +153,61 @@ def test_sparse_argument_errors_before_launch(S):
     import torch
     trees = S.Trees([200], [10], [4], 4, torch.zeros(4, dtype=torch.int32))
     N = S.specopd_tree_packed_rows(trees)
-    need = S.specopd_sparse_workspace_bytes(trees, 4, 2, 32, 8)
+    tiles = S.specopd_tree_num_tiles(trees)
+    need = S.specopd_sparse_workspace_bytes(trees, 4, 2, 32, 8, 4)
+    # rotated Q, K; trunk group keys; chosen groups [N][Hkv][topk]; selection words
+    # (the deepest row has (200 + 4) // 8 = 25 complete groups: one word)
     rq, rk, gk = N * 4 * 128 * 2, N * 2 * 128 * 2, (200 // 8) * 2 * 32 * 4
+    lst, words = N * 2 * 4 * 4, N * 2 * 1 * 4
     up = lambda x: (x + 255) // 256 * 256
-    assert need == up(rq) + up(rk) + up(gk)
+    assert need == up(rq) + up(rk) + up(gk) + up(lst) + up(words)
+    assert S.specopd_sparse_workspace_bytes(trees, 4, 2, 32, 8, 0) == 0
     f = S._c["specopd_sparse_tree_attention"]
     args = lambda **kw: [trees.ref(), kw.get("q", 16), 16, 16, 16, 16, 16, kw.get("N", N), 4, kw.get("Hkv", 2),
-                         kw.get("d", 128), 32, kw.get("g", 8), kw.get("topk", 4), 1e4, 0.0, 16, 256,
-                         kw.get("ws", need), 16, None]
+                         kw.get("d", 128), 32, kw.get("g", 8), kw.get("topk", 4), 1e4, 0.0, 16,
+                         kw.get("tl", 16), 16, 16, kw.get("tiles", tiles), None, 256, kw.get("ws", need), 16, None]
     assert f(*args(d=64)) == -2             # d = 128 only
     assert f(*args(Hkv=3)) == -2            # Hq a multiple of Hkv
     assert f(*args(topk=65)) == -2          # top-k at most 64
     assert f(*args(topk=0)) == -2
     assert f(*args(g=0)) == -2
     assert f(*args(N=N + 1)) == -2
+    assert f(*args(tiles=tiles + 1)) == -2  # the mask builder's tile count
     assert f(*args(q=24)) == -6
     assert f(*args(ws=need - 1)) == -5
     assert f(*args(q=0)) == -1
+    assert f(*args(tl=0)) == -1             # the mask fields are required
     # more than 1,024 complete groups in one history
     big = S.Trees([3000], [10], [1], 4, torch.zeros(1, dtype=torch.int32))
     nb = S.specopd_tree_packed_rows(big)
-    assert f(big.ref(), 16, 16, 16, 16, 16, 16, nb, 4, 2, 128, 32, 2, 4, 1e4, 0.0, 16, 256, 1 << 30, 16,
-             None) == -2
+    nt = S.specopd_tree_num_tiles(big)
+    assert f(big.ref(), 16, 16, 16, 16, 16, 16, nb, 4, 2, 128, 32, 2, 4, 1e4, 0.0, 16, 16, 16, 16, nt, None, 256,
+             1 << 30, 16, None) == -2
+
+
+def test_wait_timeout_diagnostic_argument_errors(S):
+    f = S._c["specopd_diag_overlap_wait_timeout"]
+    need = S.specopd_overlap_workspace_bytes(8, 100, 2)
+    ok = dict(rows=8, V=100, ld=104, nb=2, W=4, grad=16, ldg=100, ws=need)
+    args = lambda **kw: [16, 16, kw.get("rows", 8), kw.get("V", 100), kw.get("ld", 104), 104, kw.get("nb", 2),
+                         kw.get("W", 4), kw.get("grad", 16), kw.get("ldg", 100), 256, kw.get("ws", need), 16, None]
+    assert f(*args(nb=3)) == -2       # rows = num_branches * W
+    assert f(*args(nb=0, rows=0)) == -2
+    assert f(*args(grad=None)) == -1  # the gradient buffer is required
+    assert f(*args(ldg=98)) == -6
+    assert f(*args(ld=101)) == -6     # bf16 rows on 16-byte boundaries
+    assert f(*args(ws=need - 1)) == -5
+    assert ok
+
+
+def test_static_scratch_size_matches_the_header(S):
+    import os
+    import re
+    hdr = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                            "specopd.h")).read()
+    m = re.search(r"#define SPECOPD_STATIC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", hdr)
+    assert m, "SPECOPD_STATIC_SCRATCH_BYTES not found"
+    assert S.STATIC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
 
 
 def test_workspace_sizes(S):

@@ -94,6 +94,87 @@ def test_two_gloo_ranks_recombine_loss_and_gradient():
     np.testing.assert_allclose(grad, full_grad, rtol=1e-12, atol=1e-15)
 
 
+def test_tile_split_partitions_the_tiles_by_cost():
+    anchors = np.array([40, 41, 60, 90, 95, 99, 10, 12, 30], np.int32)
+    trunk, nbr, W = [100, 60], [6, 3], 8
+    costs = PAR.tile_costs(trunk, nbr, anchors, W)
+    rows = PAR.tile_rows(trunk, nbr, W)
+    # brute force: visible pairs of every row, summed per tile
+    per_row = []
+    a = 0
+    for T, B in zip(trunk, nbr):
+        per_row += [j + 1 for j in range(T)]
+        for b in range(B):
+            per_row += [int(anchors[a + b]) + 1 + i for i in range(1, W + 1)]
+        a += B
+    assert rows[-1, 1] == len(per_row)
+    assert [int(c) for c in costs] == [sum(per_row[r0:r1]) for r0, r1 in rows]
+    for world in (1, 2, 3, 5):
+        spans = [PAR.split_tiles(costs, world, r) for r in range(world)]
+        assert spans[0][0] == 0 and spans[-1][1] == len(costs)
+        assert all(spans[r][1] == spans[r + 1][0] for r in range(world - 1))
+        if world <= len(costs):
+            share = [costs[t0:t1].sum() for t0, t1 in spans]
+            assert max(share) <= costs.sum() / world + costs.max()
+
+
+def _split_rank_main(rank, world, port, out_dir):
+    """One rank of the split step, the oracle standing in for the kernels: its
+    run of query tiles (attention rows) and its share of whole branches
+    (overlap, loss with the global count, gradient); the loss shares summed
+    over the process group."""
+    import synthetic as SY
+    from oracle import attention as OA
+    from oracle import tree as OT
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        case = SY.make_case("split", [(150, 20, 6), (90, 10, 4)], W=4, Hq=4, Hkv=2, d=16, dtype="f32", vocab=40,
+                            sig_t=3.0, sig_n=1.0, seed=8)
+        nb = int(sum(case.num_branches))
+        costs = PAR.tile_costs(case.trunk_len, case.num_branches, case.anchors, case.W)
+        t0, t1 = PAR.split_tiles(costs, world, rank)
+        trows = PAR.tile_rows(case.trunk_len, case.num_branches, case.W)
+        rows = list(range(int(trows[t0, 0]), int(trows[t1 - 1, 1]))) if t1 > t0 else []
+        pt = OT.pack(case.trunk_len, case.prompt_len, case.num_branches, case.anchors, case.W, True)
+        attn = OA.tree_attention(pt, case.q, case.k, case.v, theta=case.theta, rows=rows) if rows else \
+            np.zeros((0, case.Hq, case.d))
+        b0, b1 = PAR.shard_range(nb, world, rank)
+        lr = slice(b0 * case.W, b1 * case.W)
+        z, t = case.draft[lr].astype(np.float64), case.teacher[lr].astype(np.float64)
+        count = nb * case.W
+        loss = PAR.global_loss(OO.e2e_tv_loss(OO.overlap(z, t), case.W, count=count))
+        grad = OO.e2e_tv_grad_draft(z, t, case.W, count=count)
+        np.savez(os.path.join(out_dir, f"s{rank}.npz"), rows=np.asarray(rows, np.int64), attn=attn, loss=loss,
+                 b0=b0, grad=grad)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_split_one_batch_end_to_end():
+    import synthetic as SY
+    from oracle import attention as OA
+    from oracle import tree as OT
+    world = 2
+    with tempfile.TemporaryDirectory() as out_dir:
+        mp.spawn(_split_rank_main, args=(world, _free_port(), out_dir), nprocs=world, join=True)
+        res = [np.load(os.path.join(out_dir, f"s{r}.npz")) for r in range(world)]
+    case = SY.make_case("split", [(150, 20, 6), (90, 10, 4)], W=4, Hq=4, Hkv=2, d=16, dtype="f32", vocab=40,
+                        sig_t=3.0, sig_n=1.0, seed=8)
+    pt = OT.pack(case.trunk_len, case.prompt_len, case.num_branches, case.anchors, case.W, True)
+    full = OA.tree_attention(pt, case.q, case.k, case.v, theta=case.theta)
+    rows = np.concatenate([r["rows"] for r in res])
+    assert np.array_equal(rows, np.arange(pt.num_rows))       # every row scored exactly once
+    np.testing.assert_allclose(np.concatenate([r["attn"] for r in res]), full, rtol=0, atol=1e-12)
+    z, t = case.draft.astype(np.float64), case.teacher.astype(np.float64)
+    full_loss = OO.e2e_tv_loss(OO.overlap(z, t), case.W)
+    for r in res:
+        assert abs(float(r["loss"]) - full_loss) <= 1e-12
+    grad = np.concatenate([r["grad"] for r in sorted(res, key=lambda r: int(r["b0"]))])
+    np.testing.assert_allclose(grad, OO.e2e_tv_grad_draft(z, t, case.W), rtol=1e-12, atol=1e-15)
+
+
 @pytest.mark.gpu
 def test_branch_shards_on_gpu_recombine():
     """Two shards of one batch, each scored with the global count, against one

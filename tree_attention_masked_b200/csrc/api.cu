@@ -119,8 +119,8 @@ int specopd_build_tree_mask(const specopd_tree_desc* desc, int32_t* pos, int32_t
 int specopd_rope(const void* q, const void* k, void* q_out, void* k_out, specopd_dtype dtype, int64_t N, int Hq,
                  int Hkv, int d, const int32_t* pos, float theta, specopd_stream_t stream) {
   if (dtype != SPECOPD_F32 && dtype != SPECOPD_BF16) return SPECOPD_ERR_DTYPE;
-  if (N < 0 || Hq < 1 || Hkv < 1 || d < 4 || d > 256 || d % 4) return SPECOPD_ERR_SHAPE;
-  if (N > 0 && (!q || !k || !q_out || !k_out || !pos)) return SPECOPD_ERR_ARG;
+  if (N < 0 || Hq < 0 || Hkv < 0 || Hq + Hkv < 1 || d < 4 || d > 256 || d % 4) return SPECOPD_ERR_SHAPE;
+  if (N > 0 && (!pos || (Hq > 0 && (!q || !q_out)) || (Hkv > 0 && (!k || !k_out)))) return SPECOPD_ERR_ARG;
   if (!(theta > 0.f) || !std::isfinite(theta)) return SPECOPD_ERR_ARG;
   return cuda_status(
       launch_rope(q, k, q_out, k_out, dtype, N, Hq, Hkv, d, pos, theta, reinterpret_cast<cudaStream_t>(stream)));
@@ -141,7 +141,8 @@ int specopd_tree_attention(const void* q, const void* k, const void* v, void* ou
   if (N < 0 || num_tiles < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv) return SPECOPD_ERR_SHAPE;
   if (d < 32 || d > 256 || d % 32) return SPECOPD_ERR_SHAPE;
   if (N == 0) return SPECOPD_OK;
-  if (num_tiles < (N + SPECOPD_TILE_ROWS - 1) / SPECOPD_TILE_ROWS || num_tiles > N) return SPECOPD_ERR_SHAPE;
+  if (num_tiles > N) return SPECOPD_ERR_SHAPE;  // every tile holds at least one row
+  if (num_tiles == 0) return SPECOPD_OK;
   if (!q || !k || !v || !out || !pos || !trunk_limit || !anc_bits || !tile_meta || !status) return SPECOPD_ERR_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SPECOPD_ERR_ALIGN;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -233,19 +234,35 @@ int specopd_e2e_tv_loss(const float* alpha, int64_t num_branches, int W, double 
       launch_e2e_loss(alpha, num_branches, W, inv, loss, grad_alpha, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-int specopd_tv_overlap_e2e(const void* draft, const void* teacher, specopd_dtype dtype, int64_t rows, int64_t V,
-                           int64_t ld_draft, int64_t ld_teacher, int64_t num_branches, int W, double count,
-                           float* alpha, float* loss, float* grad_draft, int64_t ld_grad, void* workspace,
-                           size_t workspace_bytes, int32_t* status, specopd_stream_t stream) {
+}  // extern "C"
+
+// Every check of specopd_tv_overlap_e2e's arguments except the workspace.
+int specopd::check_overlap_e2e_args(const void* draft, const void* teacher, specopd_dtype dtype, int64_t rows,
+                                    int64_t V, int64_t ld_draft, int64_t ld_teacher, int64_t num_branches, int W,
+                                    double count, const float* alpha, const float* loss, const float* grad_draft,
+                                    int64_t ld_grad, const int32_t* status) {
   const int c = check_logits(draft, teacher, dtype, rows, V, ld_draft, ld_teacher);
   if (c != SPECOPD_OK) return c;
   if (W < 1 || W > SPECOPD_MAX_W || num_branches < 0 || rows != num_branches * W) return SPECOPD_ERR_SHAPE;
   if (!loss || !status) return SPECOPD_ERR_ARG;
   if (!(count <= 0.0) && !std::isfinite(count)) return SPECOPD_ERR_ARG;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (rows == 0) return cuda_status(cudaMemsetAsync(loss, 0, sizeof(float), st));
+  if (rows == 0) return SPECOPD_OK;
   if (!alpha) return SPECOPD_ERR_ARG;
   if (grad_draft && (ld_grad < V || !aligned16(grad_draft) || (ld_grad * 4) % 16)) return SPECOPD_ERR_ALIGN;
+  return SPECOPD_OK;
+}
+
+extern "C" {
+
+int specopd_tv_overlap_e2e(const void* draft, const void* teacher, specopd_dtype dtype, int64_t rows, int64_t V,
+                           int64_t ld_draft, int64_t ld_teacher, int64_t num_branches, int W, double count,
+                           float* alpha, float* loss, float* grad_draft, int64_t ld_grad, void* workspace,
+                           size_t workspace_bytes, int32_t* status, specopd_stream_t stream) {
+  const int c = check_overlap_e2e_args(draft, teacher, dtype, rows, V, ld_draft, ld_teacher, num_branches, W, count,
+                                       alpha, loss, grad_draft, ld_grad, status);
+  if (c != SPECOPD_OK) return c;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (rows == 0) return cuda_status(cudaMemsetAsync(loss, 0, sizeof(float), st));
   const OverlapLayout L = overlap_layout(rows, V, num_branches);
   if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) % kAlign))
     return SPECOPD_ERR_WORKSPACE;
@@ -294,6 +311,65 @@ int specopd_tv_overlap_e2e(const void* draft, const void* teacher, specopd_dtype
   return SPECOPD_OK;
 }
 
+int specopd_diag_overlap_wait_timeout(const void* draft, const void* teacher, int64_t rows, int64_t V,
+                                      int64_t ld_draft, int64_t ld_teacher, int64_t num_branches, int W,
+                                      float* grad_draft, int64_t ld_grad, void* workspace, size_t workspace_bytes,
+                                      int32_t* status, specopd_stream_t stream) {
+  const int c = check_logits(draft, teacher, SPECOPD_BF16, rows, V, ld_draft, ld_teacher);
+  if (c != SPECOPD_OK) return c;
+  if (W < 1 || W > SPECOPD_MAX_W || num_branches < 1 || rows != num_branches * W) return SPECOPD_ERR_SHAPE;
+  if (!status || !grad_draft) return SPECOPD_ERR_ARG;
+  if (ld_grad < V || !aligned16(grad_draft) || (ld_grad * 4) % 16) return SPECOPD_ERR_ALIGN;
+  const OverlapLayout L = overlap_layout(rows, V, num_branches);
+  if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) % kAlign))
+    return SPECOPD_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  OverlapArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.draft = draft;
+  a.teacher = teacher;
+  a.ld_draft = ld_draft;
+  a.ld_teacher = ld_teacher;
+  a.rows = rows;
+  a.V = V;
+  a.row_begin = 0;  // no statistics rows: no branch is ever published
+  a.row_end = 0;
+  a.grad_begin = 0;
+  a.grad_end = rows;
+  a.mbits = ws + L.mbits;
+  a.mbits_ld = L.mbits_ld;
+  a.lz2 = reinterpret_cast<float*>(ws + L.lz2);
+  a.ql = reinterpret_cast<float*>(ws + L.ql);
+  a.g = reinterpret_cast<float*>(ws + L.g);
+  a.branch_cnt = reinterpret_cast<uint32_t*>(ws + L.counters);
+  a.branch_sum = reinterpret_cast<double*>(ws + L.bsum);
+  a.W = W;
+  a.num_branches = num_branches;
+  a.inv_count = 1.0 / (double)rows;
+  a.grad = grad_draft;
+  a.ld_grad = ld_grad;
+  a.status = status;
+  if (cudaMemsetAsync(a.branch_cnt, 0, L.counters_bytes, st) != cudaSuccess) return SPECOPD_ERR_CUDA;
+  return cuda_status(launch_tv_stats_bf16(a, st));
+}
+
+int specopd_tree_causal_conv(const void* x, void* out, specopd_dtype dtype, int64_t N, int C, const float* weight,
+                             const float* bias, int Kw, int silu, const int32_t* pos, const int32_t* trunk_limit,
+                             const int32_t* cu_rows, int num_trees, specopd_stream_t stream) {
+  if (dtype != SPECOPD_F32 && dtype != SPECOPD_BF16) return SPECOPD_ERR_DTYPE;
+  const int vec = dtype == SPECOPD_BF16 ? 8 : 4;
+  if (N < 0 || N > (1LL << 30) || C < 1 || C % vec || C > (1 << 24) || Kw < 1 || Kw > 8) return SPECOPD_ERR_SHAPE;
+  if (num_trees < 1 || num_trees > SPECOPD_MAX_TREES || (silu != 0 && silu != 1)) return SPECOPD_ERR_ARG;
+  if (N == 0) return SPECOPD_OK;
+  if (!x || !out || !weight || !pos || !trunk_limit || !cu_rows) return SPECOPD_ERR_ARG;
+  if (!aligned16(x) || !aligned16(out) || (reinterpret_cast<uintptr_t>(weight) & 3) ||
+      (reinterpret_cast<uintptr_t>(bias) & 3))
+    return SPECOPD_ERR_ALIGN;
+  return cuda_status(launch_tree_conv(x, out, dtype, N, C, weight, bias, Kw, silu, pos, trunk_limit, cu_rows,
+                                      num_trees, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t specopd_gdn_workspace_bytes(const specopd_tree_desc* desc, int H) {
   TreeParams p;
   if (tree_params(desc, &p) != SPECOPD_OK || H < 1) return 0;
@@ -329,23 +405,37 @@ int specopd_gdn_tree(const specopd_tree_desc* desc, const void* q, const void* k
   return cuda_status(launch_gdn_tree(g, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-static size_t sparse_ws(const TreeParams& p, int Hq, int Hkv, int di, int g, size_t* off_rk, size_t* off_gk) {
+// Sparse attention workspace (all regions 256-byte aligned): rotated Q [N][Hq][128]
+// and K [N][Hkv][128] bf16, trunk group keys [groups][Hkv][di] fp32, the chosen
+// groups [N][Hkv][topk] int32 and the selection words [N][Hkv][words] uint32.
+struct SparseLayout {
+  size_t rk, gk, list, mask, total;
+  int words;
+};
+
+static SparseLayout sparse_layout(const TreeParams& p, int Hq, int Hkv, int di, int g, int topk) {
   const int64_t N = p.row_base[p.num_trees];
-  *off_rk = align_up((size_t)N * Hq * 128 * 2);
-  *off_gk = *off_rk + align_up((size_t)N * Hkv * 128 * 2);
-  return *off_gk + align_up(sparse_group_keys(p, g) * Hkv * di * sizeof(float));
+  SparseLayout L;
+  L.words = sparse_selection_words(p, g);
+  L.rk = align_up((size_t)N * Hq * 128 * 2);
+  L.gk = L.rk + align_up((size_t)N * Hkv * 128 * 2);
+  L.list = L.gk + align_up(sparse_group_keys(p, g) * Hkv * di * sizeof(float));
+  L.mask = L.list + align_up((size_t)N * Hkv * topk * sizeof(int32_t));
+  L.total = L.mask + align_up((size_t)N * Hkv * L.words * sizeof(uint32_t));
+  return L;
 }
 
-size_t specopd_sparse_workspace_bytes(const specopd_tree_desc* desc, int Hq, int Hkv, int di, int g) {
+size_t specopd_sparse_workspace_bytes(const specopd_tree_desc* desc, int Hq, int Hkv, int di, int g, int topk) {
   TreeParams p;
-  if (tree_params(desc, &p) != SPECOPD_OK || Hq < 1 || Hkv < 1 || di < 1 || g < 1) return 0;
-  size_t a, b;
-  return sparse_ws(p, Hq, Hkv, di, g, &a, &b);
+  if (tree_params(desc, &p) != SPECOPD_OK || Hq < 1 || Hkv < 1 || di < 1 || g < 1 || topk < 1) return 0;
+  return sparse_layout(p, Hq, Hkv, di, g, topk).total;
 }
 
 int specopd_sparse_tree_attention(const specopd_tree_desc* desc, const void* q, const void* k, const void* v,
                                   const void* qi, const void* ki, void* out, int64_t N, int Hq, int Hkv, int d,
                                   int di, int g, int topk, float rope_theta, float softmax_scale, const int32_t* pos,
+                                  const int32_t* trunk_limit, const uint64_t* anc_bits,
+                                  const specopd_tile_meta* tile_meta, int64_t num_tiles, int32_t* selected,
                                   void* workspace, size_t workspace_bytes, int32_t* status,
                                   specopd_stream_t stream) {
   SparseArgs a;
@@ -354,16 +444,16 @@ int specopd_sparse_tree_attention(const specopd_tree_desc* desc, const void* q, 
   if (d != 128 || Hq < 1 || Hkv < 1 || Hq % Hkv || di < 1 || di > 256 || g < 1 || topk < 1 ||
       topk > kSpMaxTopk)
     return SPECOPD_ERR_SHAPE;
-  if (N != (int64_t)a.tp.row_base[a.tp.num_trees]) return SPECOPD_ERR_SHAPE;
+  if (N != (int64_t)a.tp.row_base[a.tp.num_trees] || num_tiles != a.tp.num_tiles) return SPECOPD_ERR_SHAPE;
   for (int t = 0; t < a.tp.num_trees; ++t)  // every row's complete groups must fit the score buffer
     if ((a.tp.trunk_len[t] + a.tp.rows_per_branch) / g > kSpMaxGroups) return SPECOPD_ERR_SHAPE;
-  if (!q || !k || !v || !qi || !ki || !out || !pos || !status) return SPECOPD_ERR_ARG;
+  if (!q || !k || !v || !qi || !ki || !out || !pos || !trunk_limit || !anc_bits || !tile_meta || !status)
+    return SPECOPD_ERR_ARG;
   if (a.tp.total_branches > 0 && !desc->anchors) return SPECOPD_ERR_ARG;
   if (!(rope_theta > 0.f) || !std::isfinite(rope_theta)) return SPECOPD_ERR_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SPECOPD_ERR_ALIGN;
-  size_t off_rk, off_gk;
-  const size_t need = sparse_ws(a.tp, Hq, Hkv, di, g, &off_rk, &off_gk);
-  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) % kAlign))
+  const SparseLayout L = sparse_layout(a.tp, Hq, Hkv, di, g, topk);
+  if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) % kAlign))
     return SPECOPD_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.q = q;
@@ -373,8 +463,12 @@ int specopd_sparse_tree_attention(const specopd_tree_desc* desc, const void* q, 
   a.ki = ki;
   a.out = out;
   a.rq = ws;
-  a.rk = ws + off_rk;
-  a.gkey = reinterpret_cast<float*>(ws + off_gk);
+  a.rk = ws + L.rk;
+  a.gkey = reinterpret_cast<float*>(ws + L.gk);
+  a.sel_list = reinterpret_cast<int32_t*>(ws + L.list);
+  a.sel_mask = reinterpret_cast<uint32_t*>(ws + L.mask);
+  a.sel_words = L.words;
+  a.sel_out = selected;
   a.N = N;
   a.Hq = Hq;
   a.Hkv = Hkv;
@@ -382,9 +476,15 @@ int specopd_sparse_tree_attention(const specopd_tree_desc* desc, const void* q, 
   a.g = g;
   a.topk = topk;
   a.theta = rope_theta;
-  a.scale_log2 = (softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(128.f)) * 1.4426950408889634f;
+  a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)d);
+  a.scale_log2 = a.scale * 1.4426950408889634f;
   a.pos = pos;
+  a.trunk_limit = trunk_limit;
+  a.anc_bits = anc_bits;
+  a.meta = tile_meta;
+  a.num_tiles = num_tiles;
   a.anchors = desc->anchors;
+  a.status = status;
   return cuda_status(launch_sparse_attention(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -44,8 +44,16 @@ struct AttnArgs {
   int32_t* status;
 };
 
-// tcgen05 kernel: bf16, d = 128.
-cudaError_t launch_tree_attention_sm100(const AttnArgs& a, cudaStream_t stream);
+// Indexer-group selection read by the tcgen05 kernel's sparse mode: per
+// (row, KV head) `words` uint32 words, bit m set iff complete group m of the
+// row's history is selected; g a multiple of 64.
+struct SparseSel {
+  const uint32_t* mask;
+  int words;
+  int g;
+};
+// tcgen05 kernel: bf16, d = 128; sparse mode when sel is non-null.
+cudaError_t launch_tree_attention_sm100(const AttnArgs& a, cudaStream_t stream, const SparseSel* sel = nullptr);
 // SIMT kernel: fp32 or bf16, d multiple of 32 up to 256.
 cudaError_t launch_tree_attention_simt(const AttnArgs& a, specopd_dtype dtype, cudaStream_t stream);
 
@@ -83,6 +91,12 @@ struct OverlapArgs {
   int32_t* status;
 };
 
+// Every argument check of specopd_tv_overlap_e2e except its workspace (api.cu).
+int check_overlap_e2e_args(const void* draft, const void* teacher, specopd_dtype dtype, int64_t rows, int64_t V,
+                           int64_t ld_draft, int64_t ld_teacher, int64_t num_branches, int W, double count,
+                           const float* alpha, const float* loss, const float* grad_draft, int64_t ld_grad,
+                           const int32_t* status);
+
 cudaError_t launch_tv_stats(const OverlapArgs& a, specopd_dtype dtype, cudaStream_t stream);
 // bf16 kernels (tv_bf16.cu); launch_tv_stats routes bf16 here
 cudaError_t launch_tv_stats_bf16(const OverlapArgs& a, cudaStream_t stream);
@@ -91,6 +105,11 @@ cudaError_t launch_tv_fused_bf16(OverlapArgs a, cudaStream_t stream);
 cudaError_t launch_tv_grad(const OverlapArgs& a, specopd_dtype dtype, cudaStream_t stream);
 cudaError_t launch_e2e_loss(const float* alpha, int64_t num_branches, int W, double inv_count, float* loss,
                             float* grad_alpha, cudaStream_t stream);
+
+// Short causal convolution along each row's history (tree_conv.cu).
+cudaError_t launch_tree_conv(const void* x, void* out, specopd_dtype dtype, int64_t N, int C, const float* w,
+                             const float* bias, int Kw, int silu, const int32_t* pos, const int32_t* trunk_limit,
+                             const int32_t* cu_rows, int num_trees, cudaStream_t stream);
 
 // Gated DeltaNet over a proposal tree with indexed state replay (gdn.cu).
 struct GdnArgs {
@@ -125,13 +144,23 @@ struct SparseArgs {
   float* gkey;          // workspace: [trunk groups][Hkv][di] fp32
   int64_t N;
   int Hq, Hkv, di, g, topk;
-  float theta, scale_log2;
+  float theta, scale, scale_log2;  // softmax scale and scale * log2(e)
   const int32_t* pos;      // [N] semantic positions (specopd_build_tree_mask)
+  const int32_t* trunk_limit;            // [N] (specopd_build_tree_mask)
+  const uint64_t* anc_bits;              // [N]
+  const specopd_tile_meta* meta;         // [num_tiles]
+  int64_t num_tiles;
   const int32_t* anchors;  // [total branches]
+  int32_t* sel_list;       // workspace: [N][Hkv][topk] chosen groups, ascending, -1 padded
+  uint32_t* sel_mask;      // workspace: [N][Hkv][sel_words] bit m = group m chosen
+  int sel_words;
+  int32_t* sel_out;        // nullable caller copy of sel_list
+  int32_t* status;
   TreeParams tp;
   int32_t gk_off[SPECOPD_MAX_TREES + 1];  // first trunk group of each tree (set by the launcher)
 };
 size_t sparse_group_keys(const TreeParams& tp, int g);
+int sparse_selection_words(const TreeParams& tp, int g);
 cudaError_t launch_sparse_attention(SparseArgs s, cudaStream_t stream);
 
 // Overlap statistics from hidden states and LM heads (lm_head_sm100.cu).

@@ -42,7 +42,13 @@ int specopd_tv_overlap_e2e_static(const void* draft, const void* teacher, specop
                                   int64_t V, int64_t ld_draft, int64_t ld_teacher, int64_t num_branches, int W,
                                   double count, float* alpha, float* loss, float* grad_draft, int64_t ld_grad,
                                   int32_t* status, specopd_stream_t stream) {
-  if (rows < 0 || V < 1 || num_branches < 0) return SPECOPD_ERR_SHAPE;
+  // the regular entry point's checks first, so a bad call reports what is wrong with it
+  const int c = specopd::check_overlap_e2e_args(draft, teacher, dtype, rows, V, ld_draft, ld_teacher, num_branches,
+                                                W, count, alpha, loss, grad_draft, ld_grad, status);
+  if (c != SPECOPD_OK) return c;
+  if (rows == 0)  // nothing to score: no scratch needed (the loss is set to 0)
+    return specopd_tv_overlap_e2e(draft, teacher, dtype, rows, V, ld_draft, ld_teacher, num_branches, W, count,
+                                  alpha, loss, grad_draft, ld_grad, nullptr, 0, status, stream);
   if (specopd_overlap_workspace_bytes(rows, V, num_branches) > kStaticScratchBytes) return SPECOPD_ERR_WORKSPACE;
   void* scratch = nullptr;
   const int s = scratch_for_current_device(&scratch);

@@ -1,11 +1,19 @@
 """Host logic for running the scoring step on several GPUs, one process per GPU.
 
-The trees of a batch are independent problems (SpecOPD, Fig 3: each proposal
-tree is packed and scored on its own), so ranks never exchange data inside a
-step.  The only cross-rank quantities are:
+One logical batch of proposal trees is split over the ranks:
+
+* attention by query rows: each rank scores a contiguous run of the packed
+  128-row query tiles, the runs balanced by visible (row, column) pairs (a
+  trunk tile's cost grows with its position; a branch row sees its anchor's
+  prefix plus its own samples).  Every rank holds the keys and values its
+  tiles see; no data moves between ranks;
+* the overlap, E2E-TV loss and gradient by whole branches (all W rows of a
+  branch on one rank, since its prefix products couple them).
+
+The only cross-rank quantities are:
 
 * the slowest rank's step time (the job is as fast as its slowest rank);
-* the E2E-TV loss when one logical batch of branches is split over ranks.
+* the E2E-TV loss of the split batch of branches.
   The daiwk.github.io write-up, section "Equations", normalises L by the total
   number of supervised predictions, L = 1 - (1/count) sum_b sum_j prod_{i<=j}
   alpha_{b,i}.  A rank that scores its own branches with the global `count`
@@ -18,10 +26,13 @@ torch.distributed backend (NCCL on the GPUs, gloo in the CPU tests).
 """
 from __future__ import annotations
 
-from typing import Optional, Tuple
+from typing import List, Optional, Sequence, Tuple
 
+import numpy as np
 import torch
 import torch.distributed as dist
+
+TILE_ROWS = 128
 
 
 def shard_range(n: int, world: int, rank: int) -> Tuple[int, int]:
@@ -32,6 +43,60 @@ def shard_range(n: int, world: int, rank: int) -> Tuple[int, int]:
     base, extra = divmod(n, world)
     lo = rank * base + min(rank, extra)
     return lo, lo + base + (1 if rank < extra else 0)
+
+
+def tile_costs(trunk_len: Sequence[int], num_branches: Sequence[int], anchors: np.ndarray, W: int,
+               pack_terminal: bool = True) -> np.ndarray:
+    """Visible (row, column) pairs of every packed 128-row query tile, in the
+    packing order of specopd_build_tree_mask (per tree: trunk, then each
+    branch's samples; tiles never straddle two trees).  Trunk row j sees j + 1
+    columns; sample i of a branch at anchor a sees a + 1 trunk columns and its
+    own samples 1..i."""
+    rpb = W if pack_terminal else W - 1
+    out: List[np.ndarray] = []
+    a_off = 0
+    for T, B in zip(trunk_len, num_branches):
+        anc = np.asarray(anchors[a_off:a_off + B], dtype=np.int64)
+        a_off += B
+        per_row = np.concatenate([np.arange(1, T + 1, dtype=np.int64),
+                                  (anc[:, None] + 1 + np.arange(1, rpb + 1)[None, :]).reshape(-1)])
+        n = per_row.shape[0]
+        pad = (-n) % TILE_ROWS
+        out.append(np.concatenate([per_row, np.zeros(pad, np.int64)]).reshape(-1, TILE_ROWS).sum(axis=1))
+    return np.concatenate(out) if out else np.zeros(0, np.int64)
+
+
+def tile_rows(trunk_len: Sequence[int], num_branches: Sequence[int], W: int, pack_terminal: bool = True) -> np.ndarray:
+    """[first row, one past the last row] of every packed query tile, in the
+    order of tile_costs."""
+    rpb = W if pack_terminal else W - 1
+    out = []
+    base = 0
+    for T, B in zip(trunk_len, num_branches):
+        n = T + B * rpb
+        for r in range(base, base + n, TILE_ROWS):
+            out.append((r, min(base + n, r + TILE_ROWS)))
+        base += n
+    return np.asarray(out, dtype=np.int64).reshape(-1, 2)
+
+
+def split_tiles(costs: np.ndarray, world: int, rank: int) -> Tuple[int, int]:
+    """[t0, t1) of a contiguous split of the tiles over `world` ranks with about
+    equal cost: rank r ends at the first tile whose running cost reaches
+    (r + 1) / world of the total (the last rank takes the rest)."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError(f"bad split: world={world} rank={rank}")
+    n = int(costs.shape[0])
+    cum = np.cumsum(costs, dtype=np.float64)
+    total = cum[-1] if n else 0.0
+
+    def end(r):
+        if r >= world - 1:
+            return n
+        return min(n, int(np.searchsorted(cum, total * (r + 1) / world, side="left")) + 1)
+
+    t0 = 0 if rank == 0 else end(rank - 1)
+    return min(t0, n), max(min(end(rank), n), min(t0, n))
 
 
 def _world(group) -> int:

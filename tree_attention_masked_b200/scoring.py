@@ -73,13 +73,49 @@ class ScoringStep:
         S.specopd_build_tree_mask(self.trees, self.pos, self.trunk_limit, self.branch_of, self.anc_bits,
                                   self.pred_rows, self.cu_rows, self.tile_meta, self.status, stream)
 
-    def attention(self, stream=None) -> None:
-        S.specopd_tree_attention(self.q, self.k, self.v, self.out, self.pos, self.trunk_limit, self.anc_bits,
-                                 self.tile_meta, self.num_tiles, self.theta, 0.0, self.attn_ws, self.status, stream)
+    def attention(self, stream=None, tiles=None, rows=None) -> None:
+        """RoPE + tree attention.  With `tiles` = (t0, t1) only those query
+        tiles are scored (rows [r0, r1) = `rows`, the tiles' packed rows): the
+        query rows of the range and every key row are rotated into the
+        workspace, then the kernel runs on the tiles' records alone."""
+        if tiles is None:
+            S.specopd_tree_attention(self.q, self.k, self.v, self.out, self.pos, self.trunk_limit, self.anc_bits,
+                                     self.tile_meta, self.num_tiles, self.theta, 0.0, self.attn_ws, self.status,
+                                     stream)
+            return
+        t0, t1 = tiles
+        if t1 <= t0:
+            return
+        r0, r1 = rows
+        qr, kr = self.rotated()
+        S.specopd_rope(self.q[r0:r1], None, qr[r0:r1], None, self.pos[r0:r1], self.theta, stream)
+        S.specopd_rope(None, self.k, None, kr, self.pos, self.theta, stream)
+        S.specopd_tree_attention(qr, kr, self.v, self.out, self.pos, self.trunk_limit, self.anc_bits,
+                                 self.tile_meta[t0:t1], t1 - t0, 0.0, 0.0, None, self.status, stream)
 
-    def overlap(self, stream=None, count: float = 0.0) -> None:
-        S.specopd_tv_overlap_e2e(self.draft, self.teacher, self.vocab, self.num_branches, self.W, count, self.alpha,
-                                 self.loss, self.grad, self.ov_ws, self.status, stream)
+    def rotated(self):
+        """Views of the attention workspace holding rotated Q [N, Hq, d] and K [N, Hkv, d]."""
+        es = self.q.element_size()
+        nq = self.N * self.Hq * self.d
+        kq = -(-nq * es // 256) * 256 // es
+        flat = self.attn_ws.view(self.q.dtype)
+        qr = flat[:nq].view(self.N, self.Hq, self.d)
+        kr = flat[kq:kq + self.N * self.Hkv * self.d].view(self.N, self.Hkv, self.d)
+        return qr, kr
+
+    def overlap(self, stream=None, count: float = 0.0, branches=None) -> None:
+        """Fused overlap / E2E-TV / gradient.  With `branches` = (b0, b1) only
+        those branches' rows are scored, normalised by `count` (the whole
+        batch's predictions when the branches are split over ranks)."""
+        if branches is None:
+            S.specopd_tv_overlap_e2e(self.draft, self.teacher, self.vocab, self.num_branches, self.W, count,
+                                     self.alpha, self.loss, self.grad, self.ov_ws, self.status, stream)
+            return
+        b0, b1 = branches
+        r0, r1 = b0 * self.W, b1 * self.W
+        S.specopd_tv_overlap_e2e(self.draft[r0:r1], self.teacher[r0:r1], self.vocab, b1 - b0, self.W, count,
+                                 self.alpha[r0:r1], self.loss, None if self.grad is None else self.grad[r0:r1],
+                                 self.ov_ws, self.status, stream)
 
     def run(self, stream=None) -> None:
         """One pass of the whole hot path (inputs already resident)."""

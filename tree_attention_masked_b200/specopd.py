@@ -71,13 +71,18 @@ _c = {
                                    _int, _f64, _vp, _vp, _vp, _i64, _vp, _sz, _vp, _vp),
     "specopd_tv_overlap_e2e_static": _sig("specopd_tv_overlap_e2e_static", _int, _vp, _vp, _int, _i64, _i64,
                                           _i64, _i64, _i64, _int, _f64, _vp, _vp, _vp, _i64, _vp, _vp),
+    "specopd_diag_overlap_wait_timeout": _sig("specopd_diag_overlap_wait_timeout", _int, _vp, _vp, _i64, _i64,
+                                              _i64, _i64, _i64, _int, _vp, _i64, _vp, _sz, _vp, _vp),
+    "specopd_tree_causal_conv": _sig("specopd_tree_causal_conv", _int, _vp, _vp, _int, _i64, _int, _vp, _vp, _int,
+                                     _int, _vp, _vp, _vp, _int, _vp),
     "specopd_gdn_workspace_bytes": _sig("specopd_gdn_workspace_bytes", _sz, _desc_p, _int),
     "specopd_gdn_tree": _sig("specopd_gdn_tree", _int, _desc_p, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _int, _int,
                              _int, _vp, _sz, _vp, _vp),
-    "specopd_sparse_workspace_bytes": _sig("specopd_sparse_workspace_bytes", _sz, _desc_p, _int, _int, _int, _int),
+    "specopd_sparse_workspace_bytes": _sig("specopd_sparse_workspace_bytes", _sz, _desc_p, _int, _int, _int, _int,
+                                           _int),
     "specopd_sparse_tree_attention": _sig("specopd_sparse_tree_attention", _int, _desc_p, _vp, _vp, _vp, _vp, _vp,
-                                          _vp, _i64, _int, _int, _int, _int, _int, _int, _f32, _f32, _vp, _vp, _sz,
-                                          _vp, _vp),
+                                          _vp, _i64, _int, _int, _int, _int, _int, _int, _f32, _f32, _vp, _vp, _vp,
+                                          _vp, _i64, _vp, _vp, _sz, _vp, _vp),
     "specopd_lm_head_workspace_bytes": _sig("specopd_lm_head_workspace_bytes", _sz, _i64, _i64),
     "specopd_lm_head_overlap": _sig("specopd_lm_head_overlap", _int, _vp, _vp, _int, _vp, _vp, _int, _i64, _i64,
                                     _i64, _int, _f64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp, _vp),
@@ -171,11 +176,14 @@ def specopd_build_tree_mask(trees: Trees, pos, trunk_limit, branch_of, anc_bits,
 
 
 def specopd_rope(q, k, q_out, k_out, pos, theta: float, stream=None) -> None:
+    """q [N, Hq, d] -> q_out and k [N, Hkv, d] -> k_out; either pair may be None
+    (that tensor is skipped)."""
     _contig(q, k, q_out, k_out, pos)
-    N, Hq, d = q.shape
+    ref = q if q is not None else k
+    N, _, d = ref.shape
     _check("specopd_rope", _c["specopd_rope"](
-        _ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), _dtype(q), N, Hq, k.shape[1], d, _ptr(pos), theta,
-        _stream(stream)))
+        _ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), _dtype(ref), N, 0 if q is None else q.shape[1],
+        0 if k is None else k.shape[1], d, _ptr(pos), theta, _stream(stream)))
 
 
 def specopd_attention_workspace_bytes(dtype: int, N: int, Hq: int, Hkv: int, d: int) -> int:
@@ -252,6 +260,31 @@ def specopd_gdn_workspace_bytes(trees: Trees, H: int) -> int:
     return _c["specopd_gdn_workspace_bytes"](trees.ref(), H)
 
 
+def specopd_diag_overlap_wait_timeout(draft, teacher, num_branches: int, W: int, grad, workspace, status,
+                                      stream=None) -> None:
+    """Failure-detection diagnostic: the fused overlap kernel with no branch
+    ever published, so its bounded gradient waits run out (about a second)
+    and set FLAG_TIMEOUT in status.  draft, teacher [rows, >= V] bf16 (row
+    stride 16-byte aligned), grad [rows, >= V] fp32."""
+    wb = workspace.numel() * workspace.element_size()
+    _check("specopd_diag_overlap_wait_timeout", _c["specopd_diag_overlap_wait_timeout"](
+        _ptr(draft), _ptr(teacher), draft.shape[0], draft.shape[1], draft.stride(0), teacher.stride(0),
+        num_branches, W, _ptr(grad), grad.stride(0), _ptr(workspace), wb, _ptr(status), _stream(stream)))
+
+
+def specopd_tree_causal_conv(x, out, weight, bias, pos, trunk_limit, cu_rows, silu: bool = False,
+                             stream=None) -> None:
+    """Causal convolution along each row's history: x, out [N, ...] (bf16 or
+    fp32, contiguous; the trailing dimensions flattened to C), weight [C, Kw]
+    and bias [C] (or None) fp32."""
+    _contig(x, out, weight, bias)
+    N = x.shape[0]
+    C = x.numel() // max(N, 1)
+    _check("specopd_tree_causal_conv", _c["specopd_tree_causal_conv"](
+        _ptr(x), _ptr(out), _dtype(x), N, C, _ptr(weight), _ptr(bias), weight.shape[1], 1 if silu else 0,
+        _ptr(pos), _ptr(trunk_limit), _ptr(cu_rows), cu_rows.shape[0] - 1, _stream(stream)))
+
+
 def specopd_gdn_tree(trees: Trees, q, k, v, alpha, beta, out, workspace, status, stream=None) -> None:
     """Gated DeltaNet over the packed tree: q, k, v [N, H, 128] bf16, alpha,
     beta [N, H] fp32, out [N, H, 128] fp32 (all contiguous)."""
@@ -262,17 +295,20 @@ def specopd_gdn_tree(trees: Trees, q, k, v, alpha, beta, out, workspace, status,
         q.shape[2], v.shape[2], _ptr(workspace), wb, _ptr(status), _stream(stream)))
 
 
-def specopd_sparse_workspace_bytes(trees: Trees, Hq: int, Hkv: int, di: int, g: int) -> int:
-    return _c["specopd_sparse_workspace_bytes"](trees.ref(), Hq, Hkv, di, g)
+def specopd_sparse_workspace_bytes(trees: Trees, Hq: int, Hkv: int, di: int, g: int, topk: int) -> int:
+    return _c["specopd_sparse_workspace_bytes"](trees.ref(), Hq, Hkv, di, g, topk)
 
 
-def specopd_sparse_tree_attention(trees: Trees, q, k, v, qi, ki, out, pos, g: int, topk: int, rope_theta: float,
-                                  workspace, status, softmax_scale: float = 0.0, stream=None) -> None:
+def specopd_sparse_tree_attention(trees: Trees, q, k, v, qi, ki, out, pos, trunk_limit, anc_bits, tile_meta,
+                                  g: int, topk: int, rope_theta: float, workspace, status, selected=None,
+                                  softmax_scale: float = 0.0, stream=None) -> None:
     """Sparse attention with branch-consistent indexer groups: q [N, Hq, 128],
-    k, v [N, Hkv, 128], qi, ki [N, Hkv, di], out [N, Hq, 128] (bf16, contiguous)."""
-    _contig(q, k, v, qi, ki, out)
+    k, v [N, Hkv, 128], qi, ki [N, Hkv, di], out [N, Hq, 128] (bf16, contiguous);
+    pos, trunk_limit, anc_bits, tile_meta from specopd_build_tree_mask;
+    selected (optional int32 [N, Hkv, topk]) receives the chosen groups."""
+    _contig(q, k, v, qi, ki, out, selected)
     wb = workspace.numel() * workspace.element_size()
     _check("specopd_sparse_tree_attention", _c["specopd_sparse_tree_attention"](
         trees.ref(), _ptr(q), _ptr(k), _ptr(v), _ptr(qi), _ptr(ki), _ptr(out), q.shape[0], q.shape[1], k.shape[1],
-        q.shape[2], qi.shape[2], g, topk, rope_theta, softmax_scale, _ptr(pos), _ptr(workspace), wb, _ptr(status),
-        _stream(stream)))
+        q.shape[2], qi.shape[2], g, topk, rope_theta, softmax_scale, _ptr(pos), _ptr(trunk_limit), _ptr(anc_bits),
+        _ptr(tile_meta), tile_meta.shape[0], _ptr(selected), _ptr(workspace), wb, _ptr(status), _stream(stream)))
