@@ -8,11 +8,11 @@
 // inactive draft entries, the teacher must be finite, bf16 work promotes to fp32.
 //
 // Statistics need two passes over a row (the normalisers before alpha).  A
-// row's logits are read from HBM once: the second pass re-reads them while
-// they are still in the L2 (one row in flight per SM is a small part of it),
-// and every copy goes through a ring of shared-memory slots fed by one
-// producer thread, so HBM reads run ahead of the arithmetic and through the
-// reductions between the passes.  Gradient: dL/dz = g q ([q < p] - q_less)
+// row's logits are read from HBM once: the second pass re-reads them from the
+// L2, walking the row's chunks last to first (the chunks pass 1 read last are
+// the likeliest still to be there), and every copy goes through a ring of
+// shared-memory slots fed by one producer thread, so HBM reads run ahead of
+// the arithmetic and through the reductions between the passes.  Gradient: dL/dz = g q ([q < p] - q_less)
 // from the draft logits and the bits written by pass 2.  The statistics are
 // bound by instruction issue and the gradient by HBM, so the same kernel runs
 // both side by side: gradient warps on every SM stream the gradient of the
@@ -127,8 +127,8 @@ __device__ __forceinline__ uint32_t p2_group(const uint4& zw, const uint4& tw, f
 // ...) and reads it twice through a ring of shared-memory slots:
 //   pass 1 -- the row's draft and teacher logits from HBM (L2 policy
 //             evict_last) into the online base-2 (max, sum) of both softmaxes;
-//   pass 2 -- the same bytes again, an L2 hit (one row per SM is a small part
-//             of the L2), for alpha, q_less and the [q < p] bits.
+//   pass 2 -- the same bytes again, last chunk first, mostly L2 hits, for
+//             alpha, q_less and the [q < p] bits.
 // Warp 0 is the producer, warp 1 the row epilogue and warp 2 the gradient
 // producer.  The producer walks the chunk sequence P1(row), P2(row), P1(next
 // row), ... and bulk-copies each chunk of draft and teacher logits into the
@@ -263,7 +263,8 @@ __global__ void __launch_bounds__(kRThreads, 1) tv_stats_bf16_ring_kernel(const 
         const __nv_bfloat16* zrow = static_cast<const __nv_bfloat16*>(a.draft) + row * a.ld_draft;
         const __nv_bfloat16* trow = static_cast<const __nv_bfloat16*>(a.teacher) + row * a.ld_teacher;
         for (int pass = 0; ok && pass < 2; ++pass) {
-          for (int c = 0; c < nch; ++c, ++n) {
+          for (int cc = 0; cc < nch; ++cc, ++n) {
+            const int c = pass ? nch - 1 - cc : cc;  // pass 2 walks the row backwards
             const int slot = (int)(n % kRSlots);
             if (n >= kRSlots && !mbar_wait(&ctl->empty[slot], (uint32_t)((n / kRSlots) - 1) & 1u, abort_flag)) {
               ok = false;
@@ -399,7 +400,8 @@ __global__ void __launch_bounds__(kRThreads, 1) tv_stats_bf16_ring_kernel(const 
     const float2 nlz = make_float2(live ? -lz2 : 0.f, live ? -lz2 : 0.f), nlt = make_float2(-lt2, -lt2);
     float2 acc_a = make_float2(0.f, 0.f), acc_q = make_float2(0.f, 0.f);
     uint8_t* mrow = a.mbits ? a.mbits + row * a.mbits_ld : nullptr;
-    for (int c = 0; c < nch; ++c, ++n) {
+    for (int cc = 0; cc < nch; ++cc, ++n) {
+      const int c = nch - 1 - cc;  // the producer's order: last chunk first
       const int slot = (int)(n % kRSlots);
       if (ok) ok = mbar_wait_warp(&ctl->full[slot], (uint32_t)(n / kRSlots) & 1u, abort_flag);
       if (ok) {
