@@ -49,7 +49,12 @@ KERNEL_SOURCES = {
     "tv_overlap_e2e": ["tree_attention_masked_b200/csrc/tv_bf16.cu", "tree_attention_masked_b200/csrc/overlap_common.cuh",
                        "tree_attention_masked_b200/csrc/ptx.cuh"],
 }
-MEASURED_TRAFFIC = {}  # {(workload, kernel): {"bytes": B, "sha": digest, "profile": file}}
+MEASURED_TRAFFIC = {  # {(workload, kernel): {"bytes": B, "sha": digest, "profile": file}}
+    (5, "tree_attention"): {"bytes": 3482385664.0 + 453979392.0, "sha": "ec93944992a931ed",
+                            "profile": "profiles/dram_traffic_scale27b.md"},
+    (5, "tv_overlap_e2e"): {"bytes": 17671086848.0 + 8334844672.0, "sha": "05ea75c9d2c9d63c",
+                            "profile": "profiles/dram_traffic_scale27b.md"},
+}
 
 
 def source_digest(kernel: str) -> str:

@@ -349,8 +349,9 @@ size_t specopd_sparse_workspace_bytes(const specopd_tree_desc* desc, int Hq, int
  * prints no formula): groups are g consecutive semantic positions of the
  * row's own history (trunk through the anchor, then its branch); a complete
  * group's key is the mean of its members' indexer keys; the score is the
- * indexer query dotted with it, taken in fp32 in a fixed order (sequential
- * sums, fused multiply-adds); the k best per KV head, ties to the earlier
+ * indexer query dotted with it, taken in fp32 in a fixed order (members
+ * summed in position order, products summed by a fixed reduction tree); the
+ * k best per KV head, ties to the earlier
  * group; attention as specopd_tree_attention (rotate-half RoPE at `pos`,
  * scale softmax_scale or 1/sqrt(d) when <= 0) over the chosen members and the
  * tail, fp32 accumulation.  For g a multiple of 64 the attention runs on the
@@ -414,6 +415,49 @@ int specopd_lm_head_overlap(const void* h_draft, const void* head_draft, int Hd,
                             double count, float* alpha, float* q_less, float* lse_draft, float* lse_teacher,
                             float* loss, float* grad_alpha, float* grad_draft, int64_t ld_grad, void* workspace,
                             size_t workspace_bytes, int32_t* status, specopd_stream_t stream);
+
+/*
+ * specopd_lm_head_shard_phase -- the LM head + overlap of specopd_lm_head_overlap
+ * split over vocabulary shards (one shard per GPU), one phase at a time.
+ *
+ * The write-up's section "Inputs and code mapping" (prediction_logits from
+ * supplied hidden states and head; e2e_tv_loss on the aligned logits), with
+ * the vocabulary split: every rank holds all hidden states and the rows
+ * [v0, v0 + V_shard) of both heads.  alpha needs both full-vocabulary
+ * normalisers before any min, so the phases are separated by three per-row
+ * exchanges of the ranks' partials (gather them in rank order, combine with
+ * specopd_merge_parts):
+ *   phase 0 -- out1 / out2 = the shard's base-2 log-sum-exps of draft /
+ *              teacher logits per row [rows] (gather, merge with mode 1 ->
+ *              the global lz2, lt2);
+ *   phase 1 -- with the global lz2, lt2: out1 / out2 = the shard's alpha /
+ *              q_less shares [rows] (gather, merge with mode 0 -> alpha,
+ *              q_less; then specopd_e2e_tv_loss on alpha gives L and dL/dalpha);
+ *              the [q < p] bits of the shard stay in the workspace;
+ *   phase 2 -- with the global lz2, q_less and dL/dalpha (grad_alpha): out1 =
+ *              dL/dz of the shard's columns, [rows, ld_grad] fp32 (16-byte
+ *              aligned rows), from the bits phase 1 left in the same workspace.
+ * Arguments as specopd_lm_head_overlap, heads of V_shard rows; lz2 / lt2 are
+ * base-2 (log2 of the softmax normaliser).  workspace >=
+ * specopd_lm_head_workspace_bytes(rows, V_shard), kept between phases 1 and 2.
+ * A non-finite logit sets SPECOPD_FLAG_NONFINITE (phase 0).  One GPU runs the
+ * same steps with one shard; the result equals specopd_lm_head_overlap up to
+ * summation order.
+ */
+int specopd_lm_head_shard_phase(int phase, const void* h_draft, const void* head_draft, int Hd, const void* h_teacher,
+                                const void* head_teacher, int Ht, int64_t rows, int64_t V_shard, const float* lz2,
+                                const float* lt2, const float* q_less, const float* grad_alpha, float* out1,
+                                float* out2, int64_t ld_grad, void* workspace, size_t workspace_bytes,
+                                int32_t* status, specopd_stream_t stream);
+
+/*
+ * specopd_merge_parts -- out[i] from parts[k][i], k = 0 .. nparts-1, combined
+ * in part order: mode 0 the sum, mode 1 the base-2 log-sum-exp (the maximum,
+ * then log2 of the sum of 2^(x - maximum); a part of +inf or NaN is passed
+ * on, all -inf gives -inf).  parts [nparts][n], out [n]: device fp32.  Used
+ * between the phases of specopd_lm_head_shard_phase.
+ */
+int specopd_merge_parts(const float* parts, int nparts, int64_t n, int mode, float* out, specopd_stream_t stream);
 
 /*
  * specopd_tv_overlap_e2e_static -- specopd_tv_overlap_e2e without a workspace.

@@ -137,7 +137,11 @@ def test_gdn_argument_errors_before_launch(S):
     trees = S.Trees([200], [10], [4], 4, torch.zeros(4, dtype=torch.int32))
     N = S.specopd_tree_packed_rows(trees)
     need = S.specopd_gdn_workspace_bytes(trees, 2)
-    assert need == 3 * 2 * 128 * 128 * 4    # checkpoints after tokens 63, 127, 191
+    # checkpoints after tokens 63, 127, 191; then per trunk chunk (4 of them,
+    # the last one partial) and head: W^T, U [128 x 64 each], P [64][64], 64
+    # log2 decays, 64 decay ratios and the chunk's decay (padded to 4)
+    up = lambda x: (x + 255) // 256 * 256
+    assert need == up(3 * 2 * 128 * 128 * 4) + up(4 * 2 * (2 * 64 * 128 + 64 * 64 + 64 + 64 + 4) * 4)
     g = S._c["specopd_gdn_tree"]
     args = lambda **kw: [trees.ref(), kw.get("q", 16), 16, 16, 16, 16, 16, kw.get("N", N), 2, kw.get("dk", 128),
                          kw.get("dv", 128), 256, kw.get("ws", need), 16, None]
@@ -208,6 +212,25 @@ def test_static_scratch_size_matches_the_header(S):
     m = re.search(r"#define SPECOPD_STATIC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", hdr)
     assert m, "SPECOPD_STATIC_SCRATCH_BYTES not found"
     assert S.STATIC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
+
+
+def test_lm_head_shard_and_merge_argument_errors(S):
+    f = S._c["specopd_lm_head_shard_phase"]
+    need = S.specopd_lm_head_workspace_bytes(8, 512)
+    args = lambda **kw: [kw.get("phase", 0), 16, 16, kw.get("Hd", 128), 16, 16, 128, 8, kw.get("V", 512),
+                         kw.get("lz2", 16), 16, 16, 16, 16, kw.get("out2", 16), kw.get("ld", 512), 256,
+                         kw.get("ws", need), 16, None]
+    assert f(*args(phase=3)) == -1          # phases 0, 1, 2
+    assert f(*args(Hd=96)) == -2            # hidden sizes in multiples of 64
+    assert f(*args(V=0)) == -2
+    assert f(*args(phase=0, out2=None)) == -1
+    assert f(*args(phase=1, lz2=None)) == -1  # the global normalisers are inputs from phase 1 on
+    assert f(*args(phase=2, ld=510)) == -6    # gradient rows: ld >= V_shard, 16-byte aligned
+    assert f(*args(ws=need - 1)) == -5
+    m = S._c["specopd_merge_parts"]
+    assert m(16, 0, 10, 0, 16, None) == -1    # at least one part
+    assert m(16, 2, 10, 2, 16, None) == -1    # modes 0 and 1
+    assert m(None, 2, 0, 1, None, None) == 0  # nothing to merge
 
 
 def test_workspace_sizes(S):

@@ -138,3 +138,56 @@ def test_full_size_sampled_branches():
     # the loss from the GPU's own alpha, by the definition
     from oracle import overlap as OO
     assert abs(got["loss"][0] - OO.e2e_tv_loss(got["alpha"], 16)) <= 1e-6
+
+
+def test_vocabulary_shards_match_the_fused_call():
+    """The vocabulary-parallel form, as ranks would run it, here one shard
+    after another on one GPU: three shards of the heads' rows, phase 0 on each,
+    the per-row log-sum-exps gathered (stacked in shard order) and merged,
+    phase 1 on each with the global normalisers, the alpha / q_less shares
+    merged, the E2E-TV loss on the merged alpha, phase 2 on each writing its
+    columns of dL/dz.  Against the fused call and the fp64 oracle."""
+    case = SY.make_lm_head_case("shards", 3, 5, 1800, 128, 192, sig_t=3.0, sig_n=1.5, seed=12)
+    dev = torch.device("cuda")
+    t = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    hd, wd, ht, wt = t(case.h_draft), t(case.w_draft), t(case.h_teacher), t(case.w_teacher)
+    R, V = case.rows, case.V
+    cuts = [0, 512, 1536, V]
+    shards = list(zip(cuts[:-1], cuts[1:]))
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = [torch.empty(S.specopd_lm_head_workspace_bytes(R, v1 - v0), dtype=torch.uint8, device=dev)
+          for v0, v1 in shards]
+    f = lambda: torch.empty(R, device=dev)
+    lz_p, lt_p = [f() for _ in shards], [f() for _ in shards]
+    for k, (v0, v1) in enumerate(shards):
+        S.specopd_lm_head_shard_phase(0, hd, wd[v0:v1], ht, wt[v0:v1], ws[k], status, lz_p[k], lt_p[k])
+    lz2, lt2 = f(), f()
+    S.specopd_merge_parts(torch.stack(lz_p), 1, lz2)
+    S.specopd_merge_parts(torch.stack(lt_p), 1, lt2)
+    a_p, q_p = [f() for _ in shards], [f() for _ in shards]
+    for k, (v0, v1) in enumerate(shards):
+        S.specopd_lm_head_shard_phase(1, hd, wd[v0:v1], ht, wt[v0:v1], ws[k], status, a_p[k], q_p[k], lz2=lz2,
+                                      lt2=lt2)
+    alpha, q_less = f(), f()
+    S.specopd_merge_parts(torch.stack(a_p), 0, alpha)
+    S.specopd_merge_parts(torch.stack(q_p), 0, q_less)
+    loss, g = torch.empty(1, device=dev), f()
+    S.specopd_e2e_tv_loss(alpha, case.num_branches, case.W, 0.0, loss, g)
+    ld = (V + 3) // 4 * 4
+    grad = torch.full((R, ld), 7.0, device=dev)
+    for k, (v0, v1) in enumerate(shards):
+        S.specopd_lm_head_shard_phase(2, hd, wd[v0:v1], ht, wt[v0:v1], ws[k], status, grad[:, v0:], lz2=lz2,
+                                      q_less=q_less, grad_alpha=g)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert torch.all(grad[:, V:] == 7.0)
+    fused = run(case)
+    got_a = alpha.cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(got_a - fused["alpha"])) <= 1e-5
+    assert abs(loss.item() - fused["loss"][0]) <= 1e-5
+    ref = oracle(case)
+    assert np.max(np.abs(got_a - ref["alpha"])) <= TOL
+    assert np.max(np.abs(q_less.cpu().numpy() - ref["q_less"])) <= TOL
+    assert abs(loss.item() - ref["loss"]) <= TOL
+    assert rel_l2(grad[:, :V].cpu().numpy().astype(np.float64), ref["grad"]) <= GRAD_TOL
+    np.testing.assert_allclose(lz2.cpu().numpy() * np.log(2), ref["lse_draft"], rtol=0, atol=TOL)

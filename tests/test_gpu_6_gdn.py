@@ -1,7 +1,8 @@
 """Gated DeltaNet over a proposal tree on the GPU (trunk pass with C = 64
 checkpoints, then indexed replay per branch) against the oracle's plain
 sequential recurrence over each row's history: relative L2 <= 1e-4 (fp32 state
-on the GPU, fp64 in the oracle, the same bf16 inputs)."""
+on the GPU, fp64 in the oracle, the same bf16 inputs), and every row within
+1e-3 so that one wrong row cannot hide in the whole-tensor figure."""
 import numpy as np
 import pytest
 import torch
@@ -14,6 +15,7 @@ from tree_attention_masked_b200 import specopd as S
 pytestmark = pytest.mark.gpu
 
 TOL = 1e-4
+ROW_TOL = 1e-3
 
 
 def run(case):
@@ -53,6 +55,16 @@ def rel_l2(a, b):
     return float(np.linalg.norm(a - b) / np.linalg.norm(b))
 
 
+def check(got, ref, rows=None):
+    """Whole-tensor and per-row relative L2 of GPU rows `rows` (all rows by default)."""
+    g = got if rows is None else got[rows]
+    assert np.all(np.isfinite(g))
+    assert rel_l2(g, ref) <= TOL, rel_l2(g, ref)
+    per_row = [rel_l2(g[i], ref[i]) for i in range(g.shape[0])]
+    worst = int(np.argmax(per_row))
+    assert per_row[worst] <= ROW_TOL, (worst if rows is None else rows[worst], per_row[worst])
+
+
 CASES = [
     dict(trees=[(40, 5, 3)], W=4, H=2),                       # trunk below one checkpoint interval
     dict(trees=[(200, 10, 6)], W=4, H=2, anchors=[[63, 127, 128, 10, 199, 64]]),  # anchors on and next to boundaries
@@ -69,8 +81,7 @@ def test_gdn_tree_matches_oracle(cfg):
     case = SY.make_gdn_case("gdn", cfg.pop("trees"), seed=7, anchors=anchors, **cfg)
     got, status, _, _ = run(case)
     assert status == 0
-    ref = oracle_rows(case)
-    assert rel_l2(got, ref) <= TOL, rel_l2(got, ref)
+    check(got, oracle_rows(case))
 
 
 def test_checkpoints_hold_the_boundary_states():
@@ -96,6 +107,7 @@ def test_full_size_sampled_rows():
     case = SY.make_gdn_case("gdn-full", [(4096, 1024, 64)], W=16, H=8, seed=0)
     got, status, _, _ = run(case)
     assert status == 0
-    rows = [0, 63, 64, 4095, 4096, 4096 + 15, 4096 + 16 * 37 + 7, 5119]
-    ref = oracle_rows(case, rows)
-    assert rel_l2(got[rows], ref) <= TOL, rel_l2(got[rows], ref)
+    rng = np.random.default_rng(5)
+    rows = sorted({0, 63, 64, 4095, 4096, 4096 + 15, 4096 + 16 * 37 + 7, 5119} |
+                  set(rng.choice(5120, size=16, replace=False).tolist()))
+    check(got, oracle_rows(case, rows), rows)

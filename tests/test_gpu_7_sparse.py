@@ -7,8 +7,9 @@ top-k: a chosen set may differ from the fp64 one only by swapping groups whose
 fp64 scores lie within fp32 rounding of each other.  The bound used is the
 standard one for the kernel's arithmetic: a group key is a sequential fp32 sum
 of g exactly representable bf16 keys, divided by g (error <= gamma_g * mean|k|
-per element), and the score a sequential chain of di fused multiply-adds
-(error <= gamma_di * sum |q| |key|), with gamma_n = n u / (1 - n u) and
+per element), and the score di products summed in a fixed order with at most
+di roundings on any path (error <= gamma_di * sum |q| |key|, whatever the
+order), with gamma_n = n u / (1 - n u) and
 u = 2^-24, so |score_fp32 - score| <= (gamma_di + gamma_g + gamma_di gamma_g)
 * sum_e |q_e| mean_j |k_je|.  Rows whose set differs validly are compared
 against the oracle's attention over the kernel's set; every other row against

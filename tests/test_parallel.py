@@ -175,6 +175,66 @@ def test_two_gloo_ranks_split_one_batch_end_to_end():
     np.testing.assert_allclose(grad, OO.e2e_tv_grad_draft(z, t, case.W), rtol=1e-12, atol=1e-15)
 
 
+def test_vocab_range_partitions_in_tile_blocks():
+    for V in (1, 255, 256, 1000, 151936, 248320):
+        for world in (1, 2, 3, 8):
+            spans = [PAR.vocab_range(V, world, r) for r in range(world)]
+            assert spans[0][0] == 0 and spans[-1][1] == V
+            assert all(spans[r][1] == spans[r + 1][0] for r in range(world - 1))
+            assert all(lo % 256 == 0 or lo == hi == V for lo, hi in spans)   # empty shards sit at V
+
+
+def _vocab_rank_main(rank, world, port, out_dir):
+    """One rank of the vocabulary-parallel LM head, the oracle standing in for
+    the three phases: log-sum-exps of its logit columns, gathered and merged;
+    alpha / q_less shares with the global normalisers, gathered and summed;
+    the loss from the merged alpha; dL/dz of its columns."""
+    import synthetic as SY
+    from oracle import lm_head as LM
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        case = SY.make_lm_head_case("vp", 2, 3, 700, 64, 64, sig_t=3.0, sig_n=1.0, seed=4)
+        f = lambda a: SY.to_f64(a, "bf16")
+        v0, v1 = PAR.vocab_range(case.V, world, rank)
+        z = LM.prediction_logits(f(case.h_draft), f(case.w_draft)[v0:v1])
+        t = LM.prediction_logits(f(case.h_teacher), f(case.w_teacher)[v0:v1])
+        lse = lambda x: x.max(axis=1) + np.log(np.exp(x - x.max(axis=1, keepdims=True)).sum(axis=1))
+        gz = PAR.gather_rows(torch.from_numpy(lse(z))).numpy()
+        gt = PAR.gather_rows(torch.from_numpy(lse(t))).numpy()
+        lz = np.logaddexp.reduce(gz, axis=0)
+        lt = np.logaddexp.reduce(gt, axis=0)
+        q, p = np.exp(z - lz[:, None]), np.exp(t - lt[:, None])
+        alpha = PAR.gather_rows(torch.from_numpy(np.minimum(q, p).sum(axis=1))).numpy().sum(axis=0)
+        qless = PAR.gather_rows(torch.from_numpy(np.where(q < p, q, 0.0).sum(axis=1))).numpy().sum(axis=0)
+        loss = OO.e2e_tv_loss(alpha, case.W)
+        g = OO.e2e_tv_grad_alpha(alpha, case.W)
+        grad = g[:, None] * q * ((q < p).astype(np.float64) - qless[:, None])
+        np.savez(os.path.join(out_dir, f"v{rank}.npz"), v0=v0, v1=v1, alpha=alpha, loss=loss, grad=grad)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_split_the_vocabulary():
+    import synthetic as SY
+    from oracle import lm_head as LM
+    world = 2
+    with tempfile.TemporaryDirectory() as out_dir:
+        mp.spawn(_vocab_rank_main, args=(world, _free_port(), out_dir), nprocs=world, join=True)
+        res = [np.load(os.path.join(out_dir, f"v{r}.npz")) for r in range(world)]
+    case = SY.make_lm_head_case("vp", 2, 3, 700, 64, 64, sig_t=3.0, sig_n=1.0, seed=4)
+    f = lambda a: SY.to_f64(a, "bf16")
+    hd, wd, ht, wt = f(case.h_draft), f(case.w_draft), f(case.h_teacher), f(case.w_teacher)
+    full = LM.lm_head_overlap(hd, wd, ht, wt, case.W)
+    grad = OO.e2e_tv_grad_draft(LM.prediction_logits(hd, wd), LM.prediction_logits(ht, wt), case.W)
+    for r in res:
+        np.testing.assert_allclose(r["alpha"], full["alpha"], rtol=0, atol=1e-12)
+        assert abs(float(r["loss"]) - full["loss"]) <= 1e-12
+    got = np.concatenate([r["grad"] for r in sorted(res, key=lambda r: int(r["v0"]))], axis=1)
+    np.testing.assert_allclose(got, grad, rtol=1e-10, atol=1e-14)
+
+
 @pytest.mark.gpu
 def test_branch_shards_on_gpu_recombine():
     """Two shards of one batch, each scored with the global count, against one

@@ -373,7 +373,7 @@ int specopd_tree_causal_conv(const void* x, void* out, specopd_dtype dtype, int6
 size_t specopd_gdn_workspace_bytes(const specopd_tree_desc* desc, int H) {
   TreeParams p;
   if (tree_params(desc, &p) != SPECOPD_OK || H < 1) return 0;
-  return align_up(gdn_checkpoint_floats(p, H) * sizeof(float));
+  return align_up(gdn_checkpoint_floats(p, H) * sizeof(float)) + align_up(gdn_chunk_floats(p, H) * sizeof(float));
 }
 
 int specopd_gdn_tree(const specopd_tree_desc* desc, const void* q, const void* k, const void* v,
@@ -389,8 +389,9 @@ int specopd_gdn_tree(const specopd_tree_desc* desc, const void* q, const void* k
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (reinterpret_cast<uintptr_t>(alpha) & 3) ||
       (reinterpret_cast<uintptr_t>(beta) & 3))
     return SPECOPD_ERR_ALIGN;
-  const size_t need = align_up(gdn_checkpoint_floats(g.tp, H) * sizeof(float));
-  if (need > 0 && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) % kAlign)))
+  const size_t ck_bytes = align_up(gdn_checkpoint_floats(g.tp, H) * sizeof(float));
+  const size_t need = ck_bytes + align_up(gdn_chunk_floats(g.tp, H) * sizeof(float));
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) % kAlign))
     return SPECOPD_ERR_WORKSPACE;
   g.q = q;
   g.k = k;
@@ -401,6 +402,7 @@ int specopd_gdn_tree(const specopd_tree_desc* desc, const void* q, const void* k
   g.H = H;
   g.anchors = desc->anchors;
   g.ckpt = static_cast<float*>(workspace);
+  g.chunk_data = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ck_bytes);
   g.status = status;
   return cuda_status(launch_gdn_tree(g, reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -537,6 +539,52 @@ int specopd_lm_head_overlap(const void* h_draft, const void* head_draft, int Hd,
   a.workspace = workspace;
   a.status = status;
   return cuda_status(launch_lm_head_overlap(a, st));
+}
+
+int specopd_lm_head_shard_phase(int phase, const void* h_draft, const void* head_draft, int Hd, const void* h_teacher,
+                                const void* head_teacher, int Ht, int64_t rows, int64_t V_shard, const float* lz2,
+                                const float* lt2, const float* q_less, const float* grad_alpha, float* out1,
+                                float* out2, int64_t ld_grad, void* workspace, size_t workspace_bytes,
+                                int32_t* status, specopd_stream_t stream) {
+  if (phase < 0 || phase > 2) return SPECOPD_ERR_ARG;
+  if (rows < 0 || V_shard < 1 || V_shard > (1LL << 31) - 256 || Hd < 64 || Ht < 64 || Hd % 64 || Ht % 64 ||
+      Hd > (1 << 20) || Ht > (1 << 20) || rows > (1LL << 31) - 128)
+    return SPECOPD_ERR_SHAPE;
+  if (!status) return SPECOPD_ERR_ARG;
+  if (rows == 0) return SPECOPD_OK;
+  if (!h_draft || !head_draft || !h_teacher || !head_teacher || !out1) return SPECOPD_ERR_ARG;
+  if (phase <= 1 && !out2) return SPECOPD_ERR_ARG;
+  if (phase >= 1 && !lz2) return SPECOPD_ERR_ARG;
+  if (phase == 1 && !lt2) return SPECOPD_ERR_ARG;
+  if (phase == 2 && (!q_less || !grad_alpha)) return SPECOPD_ERR_ARG;
+  if (!aligned16(h_draft) || !aligned16(head_draft) || !aligned16(h_teacher) || !aligned16(head_teacher))
+    return SPECOPD_ERR_ALIGN;
+  if (phase == 2 && (ld_grad < V_shard || !aligned16(out1) || (ld_grad * 4) % 16)) return SPECOPD_ERR_ALIGN;
+  const LmHeadLayout L = lm_head_layout(rows, V_shard);
+  if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) % kAlign))
+    return SPECOPD_ERR_WORKSPACE;
+  LmHeadArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.h_draft = h_draft;
+  a.w_draft = head_draft;
+  a.h_teacher = h_teacher;
+  a.w_teacher = head_teacher;
+  a.rows = rows;
+  a.V = V_shard;
+  a.Hd = Hd;
+  a.Ht = Ht;
+  a.ld_grad = ld_grad;
+  a.workspace = workspace;
+  a.status = status;
+  return cuda_status(launch_lm_head_phase(a, phase, lz2, lt2, q_less, grad_alpha, out1, out2,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int specopd_merge_parts(const float* parts, int nparts, int64_t n, int mode, float* out, specopd_stream_t stream) {
+  if (nparts < 1 || n < 0 || (mode != 0 && mode != 1)) return SPECOPD_ERR_ARG;
+  if (n == 0) return SPECOPD_OK;
+  if (!parts || !out) return SPECOPD_ERR_ARG;
+  return cuda_status(launch_merge_parts(parts, nparts, n, mode, out, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 const char* specopd_status_string(int status) {

@@ -12,18 +12,25 @@
 //   S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,  o_t = S_t q_t,
 // so row i of S evolves on its own:
 //   u = S_i . k,  S_i <- alpha S_i + beta (v_i - alpha u) k,  o_i = S_i . q.
-// Four threads own a row (32 of its 128 columns each, fp32 in registers) and
-// join their partial dot products with two shuffles, in a fixed order.  Each
-// token's features (k, q, v, alpha, beta) are staged kGdnDepth tokens ahead
-// in a shared-memory ring with cp.async, so a step waits on the arithmetic
-// and one CTA barrier rather than on a global load.
 //
-//   gdn_trunk_kernel  -- one CTA per (tree, head, 32 state rows): the trunk in order; writes
-//                        every trunk row's output and the state after tokens
-//                        64 j - 1 (the checkpoints);
-//   gdn_branch_kernel -- one CTA per (branch, head, 32 state rows): the checkpoint at or
-//                        before the anchor, replay to the anchor, then the
-//                        branch's rows, writing their outputs.
+// The trunk runs in the chunked form of the rule (C = 64 tokens, the
+// checkpoint interval): within a chunk with start state S0, cumulative decays
+// g_t and update vectors U (S_t = alpha_t S_{t-1} + u_t k_t^T), the delta rule
+// is the unit lower-triangular system
+//   (I + A) U = diag(beta) (V - diag(g) K S0^T),  A_ti = beta_t (g_t/g_i) (k_t . k_i), i < t,
+// and  O = diag(g) Q S0^T + (L o Q K^T) U,  S_C = g_C S0 + (diag(g_C/g) U)^T K.
+// Four kernels, fp32 arithmetic throughout:
+//   gdn_prep_kernel   -- per (chunk, head), in parallel: A, and W = (I+A)^-1 diag(beta g) K,
+//                        U' = (I+A)^-1 diag(beta) V by forward substitution (so U = U' - W S0^T);
+//   gdn_scan_kernel   -- per (tree, head, 16 state rows): the only sequential part, chunk by
+//                        chunk: stores the checkpoint at each chunk start, U = U' - W S0^T,
+//                        S <- g_C S + (diag(g_C/g) U)^T K;
+//   gdn_out_kernel    -- per (chunk, head), in parallel: the trunk rows' outputs;
+//   gdn_branch_kernel -- per (branch, head, 32 state rows): the checkpoint of the anchor's
+//                        chunk plus that chunk's first m + 1 update vectors (the indexed state
+//                        replay of the figure, without a token-by-token pass), then the
+//                        branch's own tokens one by one (four threads own a row, 32 of its
+//                        columns each, features staged kGdnDepth tokens ahead with cp.async).
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -171,19 +178,365 @@ __device__ __forceinline__ void gdn_run(float (&S)[kGdnCols], GdnRing* ring, con
   cp_async_wait<0>();
 }
 
-__global__ void __launch_bounds__(kGdnThreads) gdn_trunk_kernel(const GdnArgs g) {
-  __shared__ GdnRing ring;
-  const int t = blockIdx.x, h = blockIdx.y;
-  const int row = blockIdx.z * kGdnRows + threadIdx.x / kGdnTpr, part = threadIdx.x % kGdnTpr;
-  float S[kGdnCols];
-#pragma unroll
-  for (int j = 0; j < kGdnCols; ++j) S[j] = 0.f;
-  // this tree's checkpoints, head h: [T / C][H][dv][dk] starting at ck_off[t]
-  float* ck = g.ckpt + ((long long)g.ck_off[t] * g.H + h) * kGdnD * kGdnD;
-  const long long base = g.tp.row_base[t];
-  gdn_run(S, &ring, g, h, row, part, base, base + g.tp.trunk_len[t], base, ck, 0);
+// ---------------------------------------------------------------- chunked trunk pass
+// Per (trunk chunk, head) the workspace holds (fp32): W^T [128][64], U [64][128]
+// (U' from phase A, then U from phase B), P [64][64], log2 decays [64], the
+// chunk-end decay ratios g_n/g_t [64] and g_n (padded to 4): kGdnChunkFloats.
+constexpr int kOffW = 0;
+constexpr int kOffU = kOffW + kGdnD * kGdnC;
+constexpr int kOffP = kOffU + kGdnC * kGdnD;
+constexpr int kOffLg = kOffP + kGdnC * kGdnC;
+constexpr int kOffCoef = kOffLg + kGdnC;
+constexpr int kOffGn = kOffCoef + kGdnC;
+constexpr int kGdnChunkFloats = kOffGn + 4;
+
+__device__ __forceinline__ float* chunk_ptr(const GdnArgs& g, long long chunk, int h) {
+  return g.chunk_data + (chunk * g.H + h) * (long long)kGdnChunkFloats;
 }
 
+// Phase A: one CTA per (trunk chunk of C tokens, head), 256 threads.  With the
+// chunk's cumulative decays g_t = prod_{i<=t} alpha_i (as log2 g):
+//   Gram K K^T and Q K^T in 4 x 4 register tiles over transposed K, Q;
+//   A_ti = beta_t (g_t/g_i) (k_t . k_i), i < t;   P_ti = (g_t/g_i)(q_t . k_i), i <= t;
+//   (I + A) X = B by forward substitution, one right-hand-side column per
+//   thread in registers: B = diag(beta g) K gives W, B = diag(beta) V gives U'
+//   (so a start state S0 gives the chunk's update vectors U = U' - W S0^T);
+//   coef_t = g_n / g_t, the decay from token t to the chunk's end.
+constexpr int kPrepThreads = 2 * kGdnD;
+constexpr int kTP = kGdnC + 4;  // padded row of a transposed [128][64] tile
+
+struct PrepSmem {
+  float Kt[kGdnD][kTP];
+  float Qt[kGdnD][kTP];
+  float As[kGdnC][kGdnC];
+  float lg_s[kGdnC], beta_s[kGdnC];
+};
+
+__global__ void __launch_bounds__(kPrepThreads) gdn_prep_kernel(const GdnArgs g) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  PrepSmem& ps = *reinterpret_cast<PrepSmem*>(smem_raw);
+  const int chunk = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+  int t = 0;
+  while (t + 1 < g.tp.num_trees && g.ch_off[t + 1] <= chunk) ++t;
+  const int c = chunk - g.ch_off[t];
+  const long long r0 = g.tp.row_base[t] + (long long)c * kGdnC;
+  const int n = min(kGdnC, g.tp.trunk_len[t] - c * kGdnC);
+  const __nv_bfloat16* kk = static_cast<const __nv_bfloat16*>(g.k);
+  const __nv_bfloat16* qq = static_cast<const __nv_bfloat16*>(g.q);
+  const __nv_bfloat16* vv = static_cast<const __nv_bfloat16*>(g.v);
+  float* cd = chunk_ptr(g, chunk, h);
+  for (int idx = tid; idx < kGdnC * kGdnD; idx += kPrepThreads) {
+    const int tt = idx / kGdnD, e = idx % kGdnD;
+    const bool in = tt < n;
+    ps.Kt[e][tt] = in ? __bfloat162float(kk[((r0 + tt) * g.H + h) * kGdnD + e]) : 0.f;
+    ps.Qt[e][tt] = in ? __bfloat162float(qq[((r0 + tt) * g.H + h) * kGdnD + e]) : 0.f;
+  }
+  if (tid < kGdnC) {
+    const bool in = tid < n;
+    ps.lg_s[tid] = in ? log2f(g.alpha[(r0 + tid) * g.H + h]) : 0.f;
+    ps.beta_s[tid] = in ? g.beta[(r0 + tid) * g.H + h] : 0.f;
+  }
+  __syncthreads();
+  if (tid == 0)
+    for (int tt = 1; tt < kGdnC; ++tt) ps.lg_s[tt] += ps.lg_s[tt - 1];
+  __syncthreads();
+  // K K^T and Q K^T: thread (ty, tx) owns rows 4 ty .. 4 ty + 3, columns 4 tx .. 4 tx + 3
+  {
+    const int ty = tid / 16, tx = tid % 16;
+    float gk[4][4] = {}, qk[4][4] = {};
+    for (int e = 0; e < kGdnD; ++e) {
+      const float4 kr = *reinterpret_cast<const float4*>(&ps.Kt[e][4 * ty]);
+      const float4 qr = *reinterpret_cast<const float4*>(&ps.Qt[e][4 * ty]);
+      const float4 kc = *reinterpret_cast<const float4*>(&ps.Kt[e][4 * tx]);
+      const float a[4] = {kr.x, kr.y, kr.z, kr.w}, q[4] = {qr.x, qr.y, qr.z, qr.w}, b[4] = {kc.x, kc.y, kc.z, kc.w};
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          gk[x][y] = fmaf(a[x], b[y], gk[x][y]);
+          qk[x][y] = fmaf(q[x], b[y], qk[x][y]);
+        }
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const int tt = 4 * ty + x;
+      float4 prow;
+      float* pv = &prow.x;
+#pragma unroll
+      for (int y = 0; y < 4; ++y) {
+        const int i = 4 * tx + y;
+        const float ratio = exp2f(ps.lg_s[tt] - ps.lg_s[i]);
+        ps.As[tt][i] = (i < tt && tt < n) ? ps.beta_s[tt] * ratio * gk[x][y] : 0.f;
+        pv[y] = (i <= tt && tt < n) ? ratio * qk[x][y] : 0.f;
+      }
+      *reinterpret_cast<float4*>(cd + kOffP + tt * kGdnC + 4 * tx) = prow;
+    }
+  }
+  __syncthreads();
+  // forward substitution, column j of [W | U'] per thread, in registers
+  const int j = tid;
+  float X[kGdnC];
+#pragma unroll
+  for (int tt = 0; tt < kGdnC; ++tt) {
+    float b = 0.f;
+    if (tt < n)
+      b = j < kGdnD ? ps.beta_s[tt] * exp2f(ps.lg_s[tt]) * ps.Kt[j][tt]
+                    : ps.beta_s[tt] * __bfloat162float(vv[((r0 + tt) * g.H + h) * kGdnD + (j - kGdnD)]);
+    float a0 = b, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+    for (int i = 0; i + 3 < tt; i += 4) {
+      const float4 av = *reinterpret_cast<const float4*>(&ps.As[tt][i]);
+      a0 = fmaf(-av.x, X[i], a0);
+      a1 = fmaf(-av.y, X[i + 1], a1);
+      a2 = fmaf(-av.z, X[i + 2], a2);
+      a3 = fmaf(-av.w, X[i + 3], a3);
+    }
+#pragma unroll
+    for (int i = tt & ~3; i < tt; ++i) a0 = fmaf(-ps.As[tt][i], X[i], a0);
+    X[tt] = (a0 + a1) + (a2 + a3);
+  }
+  if (j < kGdnD) {  // W^T row j: the j-th key element of every token's W row
+    float4* dst = reinterpret_cast<float4*>(cd + kOffW + j * kGdnC);
+#pragma unroll
+    for (int tt = 0; tt < kGdnC; tt += 4) dst[tt / 4] = make_float4(X[tt], X[tt + 1], X[tt + 2], X[tt + 3]);
+  } else {
+    float* dst = cd + kOffU + (j - kGdnD);
+#pragma unroll
+    for (int tt = 0; tt < kGdnC; ++tt) dst[tt * kGdnD] = X[tt];
+  }
+  if (tid < kGdnC) {
+    cd[kOffLg + tid] = ps.lg_s[tid];
+    cd[kOffCoef + tid] = exp2f(ps.lg_s[n - 1] - ps.lg_s[tid]);
+  }
+  if (tid < 4) cd[kOffGn + tid] = tid == 0 ? exp2f(ps.lg_s[n - 1]) : 0.f;
+}
+
+// Phase B: the state scan, the only sequential part.  One CTA per (tree, head,
+// 32 rows of S), 256 threads; the rows of S evolve independently, so a CTA
+// carries its rows through the trunk's chunks alone, S^T of its rows in
+// shared memory.  Per chunk c: store the rows of the state at the chunk start
+// (the checkpoint after token C c - 1), then
+//   U = U' - W S^T              (64 tokens x 32 rows; tiles of 4 x 2 per thread),
+//   S <- g_n S + sum_t coef_t U_t k_t^T   (32 rows x 128; tiles of 4 x 4).
+// The next chunk's W^T, K, U' columns and coefficients are copied (cp.async)
+// into the other half of a double buffer during the current chunk.
+constexpr int kScanRows = 32;
+constexpr int kScanThreads = 256;
+constexpr int kSR = kScanRows + 4;  // padded row of a [.][32] tile
+
+struct ScanBuf {
+  float Wt[kGdnD][kTP];
+  __nv_bfloat16 K[kGdnC][kGdnD];
+  float U[kGdnC][kSR];
+  float coef[kGdnC + 4];  // g_n / g_t, then g_n
+};
+struct ScanSmem {
+  float St[kGdnD][kSR];  // S^T of this CTA's rows: St[e][r]
+  ScanBuf buf[2];
+};
+
+__device__ __forceinline__ void scan_fetch(ScanBuf& b, const GdnArgs& g, int t, int h, int c, int tid) {
+  const int T = g.tp.trunk_len[t];
+  const int n = min(kGdnC, T - c * kGdnC);
+  const long long chunk = g.ch_off[t] + c;
+  const float* cd = chunk_ptr(g, chunk, h);
+  const __nv_bfloat16* kk = static_cast<const __nv_bfloat16*>(g.k);
+  const long long r0 = g.tp.row_base[t] + (long long)c * kGdnC;
+  for (int i = tid; i < kGdnD * (kGdnC / 4); i += kScanThreads) {  // W^T rows: 16 pieces of 4 tokens each
+    const int e = i / (kGdnC / 4), pc = i % (kGdnC / 4);
+    cp_async16(&b.Wt[e][4 * pc], cd + kOffW + e * kGdnC + 4 * pc);
+  }
+  for (int i = tid; i < n * (kGdnD / 8); i += kScanThreads) {  // K: 8 bf16 per piece
+    const int tt = i / (kGdnD / 8), pc = i % (kGdnD / 8);
+    cp_async16(&b.K[tt][8 * pc], kk + ((r0 + tt) * g.H + h) * kGdnD + 8 * pc);
+  }
+  for (int i = tid; i < n * (kScanRows / 4); i += kScanThreads) {  // U' of this CTA's rows
+    const int tt = i / (kScanRows / 4), pc = i % (kScanRows / 4);
+    cp_async16(&b.U[tt][4 * pc], cd + kOffU + tt * kGdnD + blockIdx.z * kScanRows + 4 * pc);
+  }
+  for (int i = tid; i < (kGdnC + 4) / 4; i += kScanThreads) cp_async16(&b.coef[4 * i], cd + kOffCoef + 4 * i);
+}
+
+__global__ void __launch_bounds__(kScanThreads) gdn_scan_kernel(const GdnArgs g) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  ScanSmem& sm = *reinterpret_cast<ScanSmem*>(smem_raw);
+  const int t = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+  const int row0 = blockIdx.z * kScanRows;
+  const int T = g.tp.trunk_len[t];
+  const int nch = (T + kGdnC - 1) / kGdnC;
+  // step-1 tile: tokens 4 ut .. 4 ut + 3, rows 2 ur, 2 ur + 1
+  const int ut = tid / 16, ur = tid % 16;
+  // step-2 tile: key elements 4 se .. 4 se + 3, rows 4 sr .. 4 sr + 3
+  const int se = tid / 8, sr = tid % 8;
+  for (int i = tid; i < kGdnD * kSR; i += kScanThreads) (&sm.St[0][0])[i] = 0.f;
+  auto store_ckpt = [&](int j) {  // rows 4 sr .. 4 sr + 3, elements 4 se .. 4 se + 3 of the state after token C j - 1
+    float* dst = g.ckpt + ((long long)(g.ck_off[t] + j - 1) * g.H + h) * kGdnD * kGdnD;
+#pragma unroll
+    for (int y = 0; y < 4; ++y) {
+      const int r = 4 * sr + y;
+      *reinterpret_cast<float4*>(dst + (long long)(row0 + r) * kGdnD + 4 * se) =
+          make_float4(sm.St[4 * se][r], sm.St[4 * se + 1][r], sm.St[4 * se + 2][r], sm.St[4 * se + 3][r]);
+    }
+  };
+  if (nch > 0) scan_fetch(sm.buf[0], g, t, h, 0, tid);
+  cp_async_commit();
+  for (int c = 0; c < nch; ++c) {
+    __syncthreads();  // St of the previous chunk is final
+    if (c > 0) store_ckpt(c);
+    if (c + 1 < nch) scan_fetch(sm.buf[(c + 1) & 1], g, t, h, c + 1, tid);
+    cp_async_commit();
+    cp_async_wait<1>();  // chunk c has landed
+    __syncthreads();
+    ScanBuf& b = sm.buf[c & 1];
+    const int n = min(kGdnC, T - c * kGdnC);
+    float* Ug = chunk_ptr(g, g.ch_off[t] + c, h) + kOffU;
+    // step 1: U = U' - W S^T for tokens 4 ut .., rows 2 ur ..
+    {
+      float acc[4][2] = {};
+      for (int e = 0; e < kGdnD; ++e) {
+        const float4 w = *reinterpret_cast<const float4*>(&b.Wt[e][4 * ut]);
+        const float2 sv = *reinterpret_cast<const float2*>(&sm.St[e][2 * ur]);
+        const float wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          acc[x][0] = fmaf(wv[x], sv.x, acc[x][0]);
+          acc[x][1] = fmaf(wv[x], sv.y, acc[x][1]);
+        }
+      }
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const int tt = 4 * ut + x;
+        if (tt < n) {
+          const float u0 = b.U[tt][2 * ur] - acc[x][0], u1 = b.U[tt][2 * ur + 1] - acc[x][1];
+          *reinterpret_cast<float2*>(Ug + tt * kGdnD + row0 + 2 * ur) = make_float2(u0, u1);
+          // keep coef_t U_t for the state update
+          b.U[tt][2 * ur] = b.coef[tt] * u0;
+          b.U[tt][2 * ur + 1] = b.coef[tt] * u1;
+        } else {
+          b.U[tt][2 * ur] = 0.f;
+          b.U[tt][2 * ur + 1] = 0.f;
+        }
+      }
+    }
+    __syncthreads();
+    // step 2: S^T[e][r] = g_n S^T[e][r] + sum_t K[t][e] (coef_t U[t][r])
+    {
+      float acc[4][4];
+      const float gnv = b.coef[kGdnC];
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) acc[x][y] = gnv * sm.St[4 * se + x][4 * sr + y];
+      for (int tt = 0; tt < n; ++tt) {
+        const uint2 kw = *reinterpret_cast<const uint2*>(&b.K[tt][4 * se]);
+        const float kv[4] = {__uint_as_float(kw.x << 16), __uint_as_float(kw.x & 0xFFFF0000u),
+                             __uint_as_float(kw.y << 16), __uint_as_float(kw.y & 0xFFFF0000u)};
+        const float4 u = *reinterpret_cast<const float4*>(&b.U[tt][4 * sr]);
+        const float uv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+          for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(kv[x], uv[y], acc[x][y]);
+      }
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+        *reinterpret_cast<float4*>(&sm.St[4 * se + x][4 * sr]) = make_float4(acc[x][0], acc[x][1], acc[x][2], acc[x][3]);
+    }
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  if (T % kGdnC == 0 && nch > 0) store_ckpt(nch);
+}
+
+// Phase C: outputs of the trunk rows, one CTA per (chunk, head, half of the
+// 128 value columns), 256 threads: with S0 the state at the chunk start (zero,
+// or its checkpoint),  O = diag(g) Q S0^T + P U  on the half's 64 columns.
+// fp32 products in registers: each thread owns 4 tokens x 4 columns.
+constexpr int kOutThreads = 256;
+constexpr int kOutCols = kGdnD / 2;
+
+struct OutSmem {
+  float St[kGdnD][kTP];    // S0^T of the half's columns: St[e][j]
+  float Qt[kGdnD][kTP];    // Q^T
+  float P[kGdnC][kGdnC + 4];
+  float U[kGdnC][kTP];     // the half's columns of U
+  float lg[kGdnC];
+};
+
+__global__ void __launch_bounds__(kOutThreads) gdn_out_kernel(const GdnArgs g) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  OutSmem& sm = *reinterpret_cast<OutSmem*>(smem_raw);
+  const int chunk = blockIdx.x, h = blockIdx.y, half = blockIdx.z, tid = threadIdx.x;
+  int t = 0;
+  while (t + 1 < g.tp.num_trees && g.ch_off[t + 1] <= chunk) ++t;
+  const int c = chunk - g.ch_off[t];
+  const long long r0 = g.tp.row_base[t] + (long long)c * kGdnC;
+  const int n = min(kGdnC, g.tp.trunk_len[t] - c * kGdnC);
+  const __nv_bfloat16* qq = static_cast<const __nv_bfloat16*>(g.q);
+  const float* cd = chunk_ptr(g, chunk, h);
+  const int j0 = half * kOutCols;
+  const float* S0 = c > 0 ? g.ckpt + ((long long)(g.ck_off[t] + c - 1) * g.H + h) * kGdnD * kGdnD : nullptr;
+  for (int idx = tid; idx < kOutCols * kGdnD; idx += kOutThreads) {  // S0 rows j0 .. j0 + 63
+    const int j = idx / kGdnD, e = idx % kGdnD;
+    sm.St[e][j] = S0 ? S0[(long long)(j0 + j) * kGdnD + e] : 0.f;
+  }
+  for (int idx = tid; idx < kGdnC * kGdnD; idx += kOutThreads) {
+    const int tt = idx / kGdnD, e = idx % kGdnD;
+    sm.Qt[e][tt] = tt < n ? __bfloat162float(qq[((r0 + tt) * g.H + h) * kGdnD + e]) : 0.f;
+  }
+  for (int idx = tid; idx < kGdnC * kGdnC / 4; idx += kOutThreads) {
+    const int tt = idx / (kGdnC / 4), pc = idx % (kGdnC / 4);
+    *reinterpret_cast<float4*>(&sm.P[tt][4 * pc]) = *reinterpret_cast<const float4*>(cd + kOffP + tt * kGdnC + 4 * pc);
+  }
+  for (int idx = tid; idx < kGdnC * kOutCols / 4; idx += kOutThreads) {
+    const int tt = idx / (kOutCols / 4), pc = idx % (kOutCols / 4);
+    *reinterpret_cast<float4*>(&sm.U[tt][4 * pc]) =
+        tt < n ? *reinterpret_cast<const float4*>(cd + kOffU + tt * kGdnD + j0 + 4 * pc) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  if (tid < kGdnC) sm.lg[tid] = cd[kOffLg + tid];
+  __syncthreads();
+  const int ty = tid / 16, tx = tid % 16;  // tokens 4 ty .., columns 4 tx ..
+  float acc[4][4] = {};
+  for (int e = 0; e < kGdnD; ++e) {  // Q S0^T
+    const float4 a = *reinterpret_cast<const float4*>(&sm.Qt[e][4 * ty]);
+    const float4 b = *reinterpret_cast<const float4*>(&sm.St[e][4 * tx]);
+    const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
+  }
+#pragma unroll
+  for (int x = 0; x < 4; ++x) {
+    const float gt = exp2f(sm.lg[4 * ty + x]);
+#pragma unroll
+    for (int y = 0; y < 4; ++y) acc[x][y] *= gt;
+  }
+  const int imax = min(n, 4 * ty + 4);  // P is zero past the diagonal
+  for (int i = 0; i < imax; ++i) {      // + P U
+    const float4 b = *reinterpret_cast<const float4*>(&sm.U[i][4 * tx]);
+    const float bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const float p = sm.P[4 * ty + x][i];
+#pragma unroll
+      for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(p, bv[y], acc[x][y]);
+    }
+  }
+#pragma unroll
+  for (int x = 0; x < 4; ++x) {
+    const int tt = 4 * ty + x;
+    if (tt < n)
+      *reinterpret_cast<float4*>(g.out + ((r0 + tt) * g.H + h) * kGdnD + j0 + 4 * tx) =
+          make_float4(acc[x][0], acc[x][1], acc[x][2], acc[x][3]);
+  }
+}
+
+// Phase D: branches, one CTA per (branch, head, 32 state rows).  The state
+// after the anchor a (in chunk c, m = a - C c) comes from the chunk's cached
+// data without a token-by-token replay: S = g_m S0 + sum_{t<=m} (g_m/g_t) U_t k_t^T,
+// S0 the chunk's start state; then the branch's own tokens run through the
+// recurrence one by one, writing their outputs.
 __global__ void __launch_bounds__(kGdnThreads) gdn_branch_kernel(const GdnArgs g) {
   __shared__ GdnRing ring;
   const int gb = blockIdx.x, h = blockIdx.y;
@@ -201,7 +554,7 @@ __global__ void __launch_bounds__(kGdnThreads) gdn_branch_kernel(const GdnArgs g
     a = a < P ? P : T - 1;
   }
   const long long base = g.tp.row_base[t];
-  const int c = (a + 1) / kGdnC;  // checkpoints at or before the anchor
+  const int c = a / kGdnC, m = a - c * kGdnC;
   float S[kGdnCols];
   if (c > 0) {
     const float* src = g.ckpt + ((long long)(g.ck_off[t] + c - 1) * g.H + h) * kGdnD * kGdnD + row * kGdnD +
@@ -218,8 +571,42 @@ __global__ void __launch_bounds__(kGdnThreads) gdn_branch_kernel(const GdnArgs g
 #pragma unroll
     for (int j = 0; j < kGdnCols; ++j) S[j] = 0.f;
   }
-  // replay the trunk from the checkpoint to the anchor (no outputs)
-  gdn_run(S, &ring, g, h, row, part, base + (long long)c * kGdnC, base + a + 1, base + a + 1, nullptr, 0);
+  // the chunk's first m + 1 keys, update-vector entries of this CTA's rows and
+  // decays, staged in shared memory by all threads at once
+  __shared__ __align__(16) __nv_bfloat16 kst[kGdnC][kGdnD];
+  __shared__ float ust[kGdnC][kGdnRows];
+  __shared__ float lgs[kGdnC];
+  const long long chunk = g.ch_off[t] + c;
+  const float* lg = chunk_ptr(g, chunk, h) + kOffLg;
+  const float* Uc = chunk_ptr(g, chunk, h) + kOffU;
+  const __nv_bfloat16* kk = static_cast<const __nv_bfloat16*>(g.k);
+  for (int i = threadIdx.x; i <= m * (kGdnD / 8) + (kGdnD / 8 - 1); i += kGdnThreads) {
+    const int tt = i / (kGdnD / 8), pc = i % (kGdnD / 8);
+    cp_async16(&kst[tt][8 * pc], kk + ((base + (long long)c * kGdnC + tt) * g.H + h) * kGdnD + 8 * pc);
+  }
+  for (int i = threadIdx.x; i <= m * (kGdnRows / 4) + (kGdnRows / 4 - 1); i += kGdnThreads) {
+    const int tt = i / (kGdnRows / 4), pc = i % (kGdnRows / 4);
+    cp_async16(&ust[tt][4 * pc], Uc + tt * kGdnD + blockIdx.z * kGdnRows + 4 * pc);
+  }
+  for (int i = threadIdx.x; i <= m; i += kGdnThreads) cp_async4(&lgs[i], lg + i);
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+  const int lrow = threadIdx.x / kGdnTpr;
+  const float lgm = lgs[m];
+  const float gm = exp2f(lgm);
+#pragma unroll
+  for (int j = 0; j < kGdnCols; ++j) S[j] *= gm;
+  for (int tt = 0; tt <= m; ++tt) {
+    const float coef = exp2f(lgm - lgs[tt]) * ust[tt][lrow];
+    uint4 kw[kGdnCols / 8];
+#pragma unroll
+    for (int i = 0; i < kGdnCols / 8; ++i) kw[i] = reinterpret_cast<const uint4*>(&kst[tt][part * kGdnCols])[i];
+    float kf[kGdnCols];
+    unpack16(kw, kf);
+#pragma unroll
+    for (int j = 0; j < kGdnCols; ++j) S[j] = fmaf(coef, kf[j], S[j]);
+  }
   // the branch's own rows
   const long long first = base + T + (long long)(gb - g.tp.branch_base[t]) * g.tp.rows_per_branch;
   gdn_run(S, &ring, g, h, row, part, first, first + g.tp.rows_per_branch, first, nullptr, 0);
@@ -233,15 +620,37 @@ size_t gdn_checkpoint_floats(const TreeParams& tp, int H) {
   return (size_t)n * H * kGdnD * kGdnD;
 }
 
+size_t gdn_chunk_floats(const TreeParams& tp, int H) {
+  long long n = 0;
+  for (int t = 0; t < tp.num_trees; ++t) n += (tp.trunk_len[t] + kGdnC - 1) / kGdnC;
+  return (size_t)n * H * kGdnChunkFloats;
+}
+
 cudaError_t launch_gdn_tree(GdnArgs g, cudaStream_t stream) {
   if (g.tp.num_trees == 0) return cudaSuccess;
-  int off = 0;
+  int off = 0, coff = 0;
   for (int t = 0; t < g.tp.num_trees; ++t) {
     g.ck_off[t] = off;
+    g.ch_off[t] = coff;
     off += g.tp.trunk_len[t] / kGdnC;
+    coff += (g.tp.trunk_len[t] + kGdnC - 1) / kGdnC;
   }
-  gdn_trunk_kernel<<<dim3(g.tp.num_trees, g.H, kGdnD / kGdnRows), kGdnThreads, 0, stream>>>(g);
-  cudaError_t e = cudaGetLastError();
+  g.ch_off[g.tp.num_trees] = coff;
+  cudaError_t e = cudaFuncSetAttribute(gdn_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)sizeof(PrepSmem));
+  if (e != cudaSuccess) return e;
+  gdn_prep_kernel<<<dim3(coff, g.H), kPrepThreads, sizeof(PrepSmem), stream>>>(g);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(gdn_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ScanSmem));
+  if (e != cudaSuccess) return e;
+  gdn_scan_kernel<<<dim3(g.tp.num_trees, g.H, kGdnD / kScanRows), kScanThreads, sizeof(ScanSmem), stream>>>(g);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(gdn_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(OutSmem));
+  if (e != cudaSuccess) return e;
+  gdn_out_kernel<<<dim3(coff, g.H, kGdnD / kOutCols), kOutThreads, sizeof(OutSmem), stream>>>(g);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (g.tp.total_branches == 0) return cudaSuccess;
   gdn_branch_kernel<<<dim3(g.tp.total_branches, g.H, kGdnD / kGdnRows), kGdnThreads, 0, stream>>>(g);

@@ -122,11 +122,14 @@ struct GdnArgs {
   int H;
   const int32_t* anchors;  // device [total branches], zero-based within the tree
   float* ckpt;             // [sum_t T_t / 64][H][128][128] fp32 checkpoints
+  float* chunk_data;       // per trunk chunk and head: the chunked form's data (gdn.cu)
   int32_t* status;
   TreeParams tp;
-  int32_t ck_off[SPECOPD_MAX_TREES];  // first checkpoint of each tree (set by the launcher)
+  int32_t ck_off[SPECOPD_MAX_TREES];      // first checkpoint of each tree (set by the launcher)
+  int32_t ch_off[SPECOPD_MAX_TREES + 1];  // first trunk chunk of each tree (set by the launcher)
 };
 size_t gdn_checkpoint_floats(const TreeParams& tp, int H);
+size_t gdn_chunk_floats(const TreeParams& tp, int H);
 cudaError_t launch_gdn_tree(GdnArgs g, cudaStream_t stream);
 
 // Sparse attention with branch-consistent indexer groups (sparse_attn.cu).
@@ -191,5 +194,10 @@ struct LmHeadLayout {
 };
 LmHeadLayout lm_head_layout(int64_t rows, int64_t V);
 cudaError_t launch_lm_head_overlap(const LmHeadArgs& a, cudaStream_t stream);
+// one phase over a vocabulary shard (lm_head_sm100.cu): 0 stats, 1 alpha/q_less shares, 2 dL/dz
+cudaError_t launch_lm_head_phase(LmHeadArgs a, int phase, const float* lz2, const float* lt2, const float* q_less,
+                                 const float* g, float* out1, float* out2, cudaStream_t stream);
+// parts [nparts][n] combined in part order: mode 0 sum, mode 1 base-2 log-sum-exp
+cudaError_t launch_merge_parts(const float* parts, int nparts, int64_t n, int mode, float* out, cudaStream_t stream);
 
 }  // namespace specopd

@@ -423,15 +423,15 @@ LmHeadLayout lm_head_layout(int64_t rows, int64_t V) {
   return L;
 }
 
-cudaError_t launch_lm_head_overlap(const LmHeadArgs& a, cudaStream_t stream) {
-  if (a.rows <= 0) return cudaSuccess;
-  CUtensorMap thd, twd, tht, twt;
-  if (!make_map_2d(&thd, a.h_draft, a.rows, a.Hd, kLBM) || !make_map_2d(&twd, a.w_draft, a.V, a.Hd, kLBN) ||
-      !make_map_2d(&tht, a.h_teacher, a.rows, a.Ht, kLBM) || !make_map_2d(&twt, a.w_teacher, a.V, a.Ht, kLBN))
+// Tensor maps and kernel parameters shared by the fused call and the shard phases.
+static cudaError_t lm_setup(const LmHeadArgs& a, CUtensorMap* thd, CUtensorMap* twd, CUtensorMap* tht,
+                            CUtensorMap* twt, LmParams* pp, unsigned* grid, size_t* smem) {
+  if (!make_map_2d(thd, a.h_draft, a.rows, a.Hd, kLBM) || !make_map_2d(twd, a.w_draft, a.V, a.Hd, kLBN) ||
+      !make_map_2d(tht, a.h_teacher, a.rows, a.Ht, kLBM) || !make_map_2d(twt, a.w_teacher, a.V, a.Ht, kLBN))
     return cudaErrorInvalidValue;
   const LmHeadLayout L = lm_head_layout(a.rows, a.V);
   uint8_t* ws = static_cast<uint8_t*>(a.workspace);
-  LmParams p;
+  LmParams& p = *pp;
   p.rows = a.rows;
   p.V = a.V;
   p.Hd = a.Hd;
@@ -440,16 +440,12 @@ cudaError_t launch_lm_head_overlap(const LmHeadArgs& a, cudaStream_t stream) {
   p.n_tiles = (int)L.n_tiles;
   p.part_a = reinterpret_cast<float4*>(ws + L.part_a);
   p.part_b = reinterpret_cast<float2*>(ws + L.part_b);
-  float* lz2 = reinterpret_cast<float*>(ws + L.lz2);
-  float* lt2 = reinterpret_cast<float*>(ws + L.lt2);
-  p.lz2 = lz2;
-  p.lt2 = lt2;
+  p.lz2 = reinterpret_cast<float*>(ws + L.lz2);
+  p.lt2 = reinterpret_cast<float*>(ws + L.lt2);
   p.n_words = L.n_tiles * (kLBN / 32);
   p.bits = a.grad_draft ? reinterpret_cast<uint32_t*>(ws + L.bits) : nullptr;
-  float* q_less = a.q_less ? a.q_less : reinterpret_cast<float*>(ws + L.q_less);
-  float* g = a.grad_alpha ? a.grad_alpha : reinterpret_cast<float*>(ws + L.g);
-  p.ql = q_less;
-  p.g = g;
+  p.ql = a.q_less ? a.q_less : reinterpret_cast<float*>(ws + L.q_less);
+  p.g = a.grad_alpha ? a.grad_alpha : reinterpret_cast<float*>(ws + L.g);
   p.grad = a.grad_draft;
   p.ld_grad = a.ld_grad;
   p.status = a.status;
@@ -458,15 +454,32 @@ cudaError_t launch_lm_head_overlap(const LmHeadArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  const size_t smem = sizeof(LmSmem) + 1024;
-  e = cudaFuncSetAttribute(lm_head_tile_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  *smem = sizeof(LmSmem) + 1024;
+  e = cudaFuncSetAttribute(lm_head_tile_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)*smem);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(lm_head_tile_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = cudaFuncSetAttribute(lm_head_tile_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)*smem);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(lm_head_tile_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = cudaFuncSetAttribute(lm_head_tile_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)*smem);
   if (e != cudaSuccess) return e;
   const long long total = (long long)p.m_tiles * p.n_tiles;
-  const unsigned grid = (unsigned)(total < sms ? total : sms);
+  *grid = (unsigned)(total < sms ? total : sms);
+  return cudaSuccess;
+}
+
+cudaError_t launch_lm_head_overlap(const LmHeadArgs& a, cudaStream_t stream) {
+  if (a.rows <= 0) return cudaSuccess;
+  CUtensorMap thd, twd, tht, twt;
+  LmParams p;
+  unsigned grid;
+  size_t smem;
+  cudaError_t e = lm_setup(a, &thd, &twd, &tht, &twt, &p, &grid, &smem);
+  if (e != cudaSuccess) return e;
+  const LmHeadLayout L = lm_head_layout(a.rows, a.V);
+  uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+  float* lz2 = const_cast<float*>(p.lz2);
+  float* lt2 = const_cast<float*>(p.lt2);
+  float* q_less = const_cast<float*>(p.ql);
+  float* g = const_cast<float*>(p.g);
   const unsigned rb = (unsigned)((a.rows + 7) / 8);  // one warp per row, 8 per block
   lm_head_tile_kernel<0><<<grid, kLThreads, smem, stream>>>(thd, twd, tht, twt, p);
   lm_reduce_a_kernel<<<rb, 256, 0, stream>>>(p.part_a, p.n_tiles, a.rows, lz2, lt2, a.lse_draft, a.lse_teacher,
@@ -480,6 +493,77 @@ cudaError_t launch_lm_head_overlap(const LmHeadArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess || !a.grad_draft) return e;
   // pass C: the draft logits once more, now with dL/dalpha known, into dL/dz
   lm_head_tile_kernel<2><<<grid, kLThreads, smem, stream>>>(thd, twd, tht, twt, p);
+  return cudaGetLastError();
+}
+
+// One phase over a vocabulary shard (the heads' rows [0, a.V) of the shard):
+//   phase 0 -- pass A + merge: out1/out2 = the shard's base-2 log-sum-exps of
+//              draft / teacher logits per row;
+//   phase 1 -- pass B with the global normalisers lz2, lt2 + merge: out1/out2
+//              = the shard's alpha / q_less shares; the [q < p] bits stay in
+//              the workspace for phase 2;
+//   phase 2 -- pass C with the global lz2, q_less and dL/dalpha: dL/dz of the
+//              shard's columns into a.grad_draft.
+cudaError_t launch_lm_head_phase(LmHeadArgs a, int phase, const float* lz2, const float* lt2, const float* q_less,
+                                 const float* g, float* out1, float* out2, cudaStream_t stream) {
+  if (a.rows <= 0) return cudaSuccess;
+  CUtensorMap thd, twd, tht, twt;
+  LmParams p;
+  unsigned grid;
+  size_t smem;
+  cudaError_t e = lm_setup(a, &thd, &twd, &tht, &twt, &p, &grid, &smem);
+  if (e != cudaSuccess) return e;
+  // the [q < p] bits: written by phase 1, read by phase 2 (same workspace)
+  p.bits = phase >= 1
+               ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(a.workspace) + lm_head_layout(a.rows, a.V).bits)
+               : nullptr;
+  const unsigned rb = (unsigned)((a.rows + 7) / 8);
+  if (phase == 0) {
+    lm_head_tile_kernel<0><<<grid, kLThreads, smem, stream>>>(thd, twd, tht, twt, p);
+    lm_reduce_a_kernel<<<rb, 256, 0, stream>>>(p.part_a, p.n_tiles, a.rows, out1, out2, nullptr, nullptr,
+                                                 a.status);
+  } else if (phase == 1) {
+    p.lz2 = lz2;
+    p.lt2 = lt2;
+    lm_head_tile_kernel<1><<<grid, kLThreads, smem, stream>>>(thd, twd, tht, twt, p);
+    lm_reduce_b_kernel<<<rb, 256, 0, stream>>>(p.part_b, p.n_tiles, a.rows, out1, out2);
+  } else {
+    p.lz2 = lz2;
+    p.ql = q_less;
+    p.g = g;
+    p.grad = out1;
+    lm_head_tile_kernel<2><<<grid, kLThreads, smem, stream>>>(thd, twd, tht, twt, p);
+  }
+  return cudaGetLastError();
+}
+
+namespace {
+// out[i] = the parts' values at i combined in part order: a sum (mode 0) or
+// a base-2 log-sum-exp (mode 1: max, then the sum of 2^(x - max)).
+__global__ void merge_parts_kernel(const float* __restrict__ parts, int nparts, int64_t n, int mode, float* out) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  if (mode == 0) {
+    float acc = 0.f;
+    for (int k = 0; k < nparts; ++k) acc += parts[(long long)k * n + i];
+    out[i] = acc;
+    return;
+  }
+  float m = -INFINITY;
+  for (int k = 0; k < nparts; ++k) m = fmaxf(m, parts[(long long)k * n + i]);
+  if (m == -INFINITY || m != m || m == INFINITY) {  // no entry, or a non-finite part: pass it on
+    out[i] = m;
+    return;
+  }
+  float acc = 0.f;
+  for (int k = 0; k < nparts; ++k) acc += ex2(parts[(long long)k * n + i] - m);
+  out[i] = m + log2f(acc);
+}
+}  // namespace
+
+cudaError_t launch_merge_parts(const float* parts, int nparts, int64_t n, int mode, float* out, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  merge_parts_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(parts, nparts, n, mode, out);
   return cudaGetLastError();
 }
 

@@ -16,7 +16,9 @@
 //   sparse_select_kernel -- one warp per (row, KV head): scores of the row's
 //                           complete groups (trunk keys from the table, keys of
 //                           groups holding branch tokens formed on the spot, in
-//                           the same order), top-k by repeated warp argmax; it
+//                           the same order; the lanes split a key's elements and
+//                           a fixed shuffle tree sums the products), top-k by
+//                           repeated warp argmax; it
 //                           writes the chosen groups as an ascending list and
 //                           as bits of the row's selection words;
 //   attention            -- for g a multiple of 64, the tcgen05 tree-attention
@@ -25,8 +27,8 @@
 //                           otherwise sparse_attn_kernel, one warp per (row,
 //                           KV head) with an fp32 online softmax over the
 //                           chosen groups' members and the tail.
-// Scores are sequential fp32 sums and fused multiply-adds in a fixed order,
-// so the selection is reproducible.
+// Scores are fp32 sums and fused multiply-adds in a fixed order, so the
+// selection is reproducible.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -106,20 +108,36 @@ __global__ void __launch_bounds__(32 * kSpWarps) sparse_select_kernel(const Spar
   const __nv_bfloat16* qi = static_cast<const __nv_bfloat16*>(s.qi) + (r * s.Hkv + kvh) * s.di;
   const __nv_bfloat16* ki = static_cast<const __nv_bfloat16*>(s.ki);
 
-  // ---- indexer scores of the complete groups
-  for (int m = lane; m < nc; m += 32) {
-    float acc = 0.f;
+  // ---- indexer scores of the complete groups: the lanes split each key's
+  // elements (lane + 32 i), then a fixed xor-shuffle tree sums the products
+  constexpr int kQi = 8;  // di <= 256
+  float qv[kQi];
+#pragma unroll
+  for (int i = 0; i < kQi; ++i) qv[i] = (lane + 32 * i < s.di) ? ldbf(qi + lane + 32 * i) : 0.f;
+  for (int m = 0; m < nc; ++m) {
+    float part = 0.f;
     if (m * s.g + s.g - 1 <= x.a) {  // trunk group: the shared key
       const float* key = s.gkey + ((long long)(s.gk_off[t] + m) * s.Hkv + kvh) * s.di;
-      for (int e = 0; e < s.di; ++e) acc = fmaf(ldbf(qi + e), key[e], acc);
-    } else {                          // holds branch tokens: this branch's key
-      for (int e = 0; e < s.di; ++e) {
-        float sum = 0.f;
-        for (int j = 0; j < s.g; ++j) sum += ldbf(ki + (hist_row(x, m * s.g + j) * s.Hkv + kvh) * s.di + e);
-        acc = fmaf(ldbf(qi + e), sum / (float)s.g, acc);
+#pragma unroll
+      for (int i = 0; i < kQi; ++i)
+        if (lane + 32 * i < s.di) part = fmaf(qv[i], key[lane + 32 * i], part);
+    } else {                          // holds branch tokens: this branch's key, members summed in order
+      float sum[kQi];
+#pragma unroll
+      for (int i = 0; i < kQi; ++i) sum[i] = 0.f;
+      for (int j = 0; j < s.g; ++j) {
+        const __nv_bfloat16* kr = ki + (hist_row(x, m * s.g + j) * s.Hkv + kvh) * s.di;
+#pragma unroll
+        for (int i = 0; i < kQi; ++i)
+          if (lane + 32 * i < s.di) sum[i] += ldbf(kr + lane + 32 * i);
       }
+#pragma unroll
+      for (int i = 0; i < kQi; ++i)
+        if (lane + 32 * i < s.di) part = fmaf(qv[i], sum[i] / (float)s.g, part);
     }
-    score[w][m] = acc;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+    if (lane == (m & 31)) score[w][m] = part;
   }
   __syncwarp();
 

@@ -129,3 +129,57 @@ def max_time_ms(local_ms: float, group=None, device: Optional[torch.device] = No
     t = torch.tensor([float(local_ms)], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
     return t.item()
+
+
+# ---------------------------------------------------------------- vocabulary-parallel LM head
+def vocab_range(V: int, world: int, rank: int, align: int = 256) -> Tuple[int, int]:
+    """[v0, v1) of a contiguous split of the vocabulary over `world` ranks in
+    blocks of `align` entries (the LM-head tile width; a shard's gradient
+    columns then start on 16-byte boundaries); the last rank ends at V."""
+    blocks = (V + align - 1) // align
+    b0, b1 = shard_range(blocks, world, rank)
+    return min(V, b0 * align), min(V, b1 * align)
+
+
+def gather_rows(x: torch.Tensor, group=None) -> torch.Tensor:
+    """Every rank's [n] tensor stacked in rank order: [world, n] (the tensor
+    itself, unsqueezed, on one rank)."""
+    world = _world(group)
+    if world == 1:
+        return x.unsqueeze(0)
+    parts = [torch.empty_like(x) for _ in range(world)]
+    dist.all_gather(parts, x.contiguous(), group=group)
+    return torch.stack(parts)
+
+
+def lm_head_vocab_parallel(h_draft, head_draft_shard, h_teacher, head_teacher_shard, num_branches: int, W: int,
+                           grad_shard, workspace, status, group=None, stream=None):
+    """The LM head + overlap with the vocabulary split over the ranks of
+    `group` (each rank holds all hidden states and its rows of both heads):
+    phase 0, a gather and merge of the per-row log-sum-exps, phase 1, a gather
+    and merge of the alpha / q_less shares, the E2E-TV loss on the merged
+    alpha (every rank), phase 2 for the rank's gradient columns.  Three per-row
+    exchanges; every merge is the library's, in rank order, so every rank gets
+    identical alpha, L and dL/dalpha.  Returns (alpha, q_less, loss, grad_alpha)."""
+    from . import specopd as S
+    R = h_draft.shape[0]
+    dev = h_draft.device
+    f = lambda: torch.empty(R, device=dev, dtype=torch.float32)
+    lz_l, lt_l = f(), f()
+    S.specopd_lm_head_shard_phase(0, h_draft, head_draft_shard, h_teacher, head_teacher_shard, workspace, status,
+                                  lz_l, lt_l, stream=stream)
+    lz2, lt2 = f(), f()
+    S.specopd_merge_parts(gather_rows(lz_l, group), 1, lz2, stream=stream)
+    S.specopd_merge_parts(gather_rows(lt_l, group), 1, lt2, stream=stream)
+    a_l, q_l = f(), f()
+    S.specopd_lm_head_shard_phase(1, h_draft, head_draft_shard, h_teacher, head_teacher_shard, workspace, status,
+                                  a_l, q_l, lz2=lz2, lt2=lt2, stream=stream)
+    alpha, q_less = f(), f()
+    S.specopd_merge_parts(gather_rows(a_l, group), 0, alpha, stream=stream)
+    S.specopd_merge_parts(gather_rows(q_l, group), 0, q_less, stream=stream)
+    loss, g = torch.empty(1, device=dev, dtype=torch.float32), f()
+    S.specopd_e2e_tv_loss(alpha, num_branches, W, 0.0, loss, g, stream=stream)
+    if grad_shard is not None:
+        S.specopd_lm_head_shard_phase(2, h_draft, head_draft_shard, h_teacher, head_teacher_shard, workspace, status,
+                                      grad_shard, lz2=lz2, q_less=q_less, grad_alpha=g, stream=stream)
+    return alpha, q_less, loss, g

@@ -86,6 +86,9 @@ _c = {
     "specopd_lm_head_workspace_bytes": _sig("specopd_lm_head_workspace_bytes", _sz, _i64, _i64),
     "specopd_lm_head_overlap": _sig("specopd_lm_head_overlap", _int, _vp, _vp, _int, _vp, _vp, _int, _i64, _i64,
                                     _i64, _int, _f64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp, _vp),
+    "specopd_lm_head_shard_phase": _sig("specopd_lm_head_shard_phase", _int, _int, _vp, _vp, _int, _vp, _vp, _int,
+                                        _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp, _vp),
+    "specopd_merge_parts": _sig("specopd_merge_parts", _int, _vp, _int, _i64, _int, _vp, _vp),
     "specopd_status_string": _sig("specopd_status_string", ctypes.c_char_p, _int),
 }
 
@@ -312,3 +315,26 @@ def specopd_sparse_tree_attention(trees: Trees, q, k, v, qi, ki, out, pos, trunk
         trees.ref(), _ptr(q), _ptr(k), _ptr(v), _ptr(qi), _ptr(ki), _ptr(out), q.shape[0], q.shape[1], k.shape[1],
         q.shape[2], qi.shape[2], g, topk, rope_theta, softmax_scale, _ptr(pos), _ptr(trunk_limit), _ptr(anc_bits),
         _ptr(tile_meta), tile_meta.shape[0], _ptr(selected), _ptr(workspace), wb, _ptr(status), _stream(stream)))
+
+
+def specopd_lm_head_shard_phase(phase: int, h_draft, head_draft, h_teacher, head_teacher, workspace, status,
+                                out1, out2=None, lz2=None, lt2=None, q_less=None, grad_alpha=None,
+                                stream=None) -> None:
+    """One phase of the LM head + overlap over a vocabulary shard: heads
+    [V_shard, H] bf16.  Phase 0: out1/out2 = the shard's base-2 log-sum-exps;
+    phase 1 (lz2, lt2 global): out1/out2 = alpha / q_less shares; phase 2
+    (lz2, q_less, grad_alpha global): out1 = dL/dz of the shard's columns."""
+    _contig(h_draft, head_draft, h_teacher, head_teacher)
+    wb = workspace.numel() * workspace.element_size()
+    ld = out1.stride(0) if phase == 2 else 0
+    _check("specopd_lm_head_shard_phase", _c["specopd_lm_head_shard_phase"](
+        phase, _ptr(h_draft), _ptr(head_draft), h_draft.shape[1], _ptr(h_teacher), _ptr(head_teacher),
+        h_teacher.shape[1], h_draft.shape[0], head_draft.shape[0], _ptr(lz2), _ptr(lt2), _ptr(q_less),
+        _ptr(grad_alpha), _ptr(out1), _ptr(out2), ld, _ptr(workspace), wb, _ptr(status), _stream(stream)))
+
+
+def specopd_merge_parts(parts, mode: int, out, stream=None) -> None:
+    """parts [nparts, n] fp32 -> out [n]: mode 0 sum, mode 1 base-2 log-sum-exp, in part order."""
+    _contig(parts, out)
+    _check("specopd_merge_parts", _c["specopd_merge_parts"](_ptr(parts), parts.shape[0], parts.shape[1], mode,
+                                                            _ptr(out), _stream(stream)))
