@@ -10,27 +10,30 @@
 // pages name GDN and print no formula; the gated delta rule), per head with
 // S in R^{dv x dk}:
 //   S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,  o_t = S_t q_t,
-// so row i of S evolves on its own:
-//   u = S_i . k,  S_i <- alpha S_i + beta (v_i - alpha u) k,  o_i = S_i . q.
+// so row i of S evolves on its own.
 //
-// The trunk runs in the chunked form of the rule (C = 64 tokens, the
+// Everything runs in the chunked form of the rule (C = 64 tokens, the
 // checkpoint interval): within a chunk with start state S0, cumulative decays
 // g_t and update vectors U (S_t = alpha_t S_{t-1} + u_t k_t^T), the delta rule
 // is the unit lower-triangular system
 //   (I + A) U = diag(beta) (V - diag(g) K S0^T),  A_ti = beta_t (g_t/g_i) (k_t . k_i), i < t,
 // and  O = diag(g) Q S0^T + (L o Q K^T) U,  S_C = g_C S0 + (diag(g_C/g) U)^T K.
 // Four kernels, fp32 arithmetic throughout:
-//   gdn_prep_kernel   -- per (chunk, head), in parallel: A, and W = (I+A)^-1 diag(beta g) K,
-//                        U' = (I+A)^-1 diag(beta) V by forward substitution (so U = U' - W S0^T);
-//   gdn_scan_kernel   -- per (tree, head, 16 state rows): the only sequential part, chunk by
-//                        chunk: stores the checkpoint at each chunk start, U = U' - W S0^T,
-//                        S <- g_C S + (diag(g_C/g) U)^T K;
-//   gdn_out_kernel    -- per (chunk, head), in parallel: the trunk rows' outputs;
-//   gdn_branch_kernel -- per (branch, head, 32 state rows): the checkpoint of the anchor's
-//                        chunk plus that chunk's first m + 1 update vectors (the indexed state
-//                        replay of the figure, without a token-by-token pass), then the
-//                        branch's own tokens one by one (four threads own a row, 32 of its
-//                        columns each, features staged kGdnDepth tokens ahead with cp.async).
+//   gdn_prep_kernel   -- per (trunk chunk, head), in parallel: A, W = (I+A)^-1 diag(beta g) K and
+//                        U' = (I+A)^-1 diag(beta) V (so U = U' - W S0^T), the decay-
+//                        weighted Q K^T and the decay ratios;
+//   gdn_scan_kernel   -- per (tree, head, 32 state rows): the only sequential part,
+//                        chunk by chunk: the checkpoint at each chunk start,
+//                        U = U' - W S0^T, S <- g_C S + (diag(g_C/g) U)^T K;
+//   gdn_out_kernel    -- per (trunk chunk, head, half of the columns), in parallel:
+//                        the trunk rows' outputs;
+//   gdn_branch_kernel -- per (branch, head, 32 state rows): the state after the
+//                        anchor from the checkpoint of its chunk plus that chunk's
+//                        first m + 1 update vectors (the indexed state replay of the
+//                        figure, without a token-by-token pass), then the branch's
+//                        own tokens one by one (four threads own a row, 32 of its
+//                        columns each, features staged kGdnDepth tokens ahead with
+//                        cp.async).
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -194,7 +197,7 @@ __device__ __forceinline__ float* chunk_ptr(const GdnArgs& g, long long chunk, i
   return g.chunk_data + (chunk * g.H + h) * (long long)kGdnChunkFloats;
 }
 
-// Phase A: one CTA per (trunk chunk of C tokens, head), 256 threads.  With the
+// Phase A: one CTA per (trunk chunk of at most C tokens, head), 256 threads.  With the
 // chunk's cumulative decays g_t = prod_{i<=t} alpha_i (as log2 g):
 //   Gram K K^T and Q K^T in 4 x 4 register tiles over transposed K, Q;
 //   A_ti = beta_t (g_t/g_i) (k_t . k_i), i < t;   P_ti = (g_t/g_i)(q_t . k_i), i <= t;
@@ -209,7 +212,8 @@ struct PrepSmem {
   float Kt[kGdnD][kTP];
   float Qt[kGdnD][kTP];
   float As[kGdnC][kGdnC];
-  float lg_s[kGdnC], beta_s[kGdnC];
+  __nv_bfloat16 V[kGdnC][kGdnD];
+  float lg_s[kGdnC], beta_s[kGdnC], bg_s[kGdnC];  // log2 g_t, beta_t, beta_t g_t
 };
 
 __global__ void __launch_bounds__(kPrepThreads) gdn_prep_kernel(const GdnArgs g) {
@@ -225,11 +229,28 @@ __global__ void __launch_bounds__(kPrepThreads) gdn_prep_kernel(const GdnArgs g)
   const __nv_bfloat16* qq = static_cast<const __nv_bfloat16*>(g.q);
   const __nv_bfloat16* vv = static_cast<const __nv_bfloat16*>(g.v);
   float* cd = chunk_ptr(g, chunk, h);
-  for (int idx = tid; idx < kGdnC * kGdnD; idx += kPrepThreads) {
-    const int tt = idx / kGdnD, e = idx % kGdnD;
-    const bool in = tt < n;
-    ps.Kt[e][tt] = in ? __bfloat162float(kk[((r0 + tt) * g.H + h) * kGdnD + e]) : 0.f;
-    ps.Qt[e][tt] = in ? __bfloat162float(qq[((r0 + tt) * g.H + h) * kGdnD + e]) : 0.f;
+  // 8 consecutive elements (16 bytes) of a token's k, q and v per step; the
+  // lanes of a warp take consecutive tokens, so the transposed stores hit
+  // consecutive banks
+#pragma unroll 2
+  for (int idx = tid; idx < kGdnC * (kGdnD / 8); idx += kPrepThreads) {
+    const int tt = idx % kGdnC, e0 = 8 * (idx / kGdnC);
+    uint4 kw = make_uint4(0u, 0u, 0u, 0u), qw = kw, vw = kw;
+    if (tt < n) {
+      const long long off = ((r0 + tt) * g.H + h) * kGdnD + e0;
+      kw = *reinterpret_cast<const uint4*>(kk + off);
+      qw = *reinterpret_cast<const uint4*>(qq + off);
+      vw = *reinterpret_cast<const uint4*>(vv + off);
+    }
+    *reinterpret_cast<uint4*>(&ps.V[tt][e0]) = vw;
+    const uint32_t ku[4] = {kw.x, kw.y, kw.z, kw.w}, qu[4] = {qw.x, qw.y, qw.z, qw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      ps.Kt[e0 + 2 * i][tt] = __uint_as_float(ku[i] << 16);
+      ps.Kt[e0 + 2 * i + 1][tt] = __uint_as_float(ku[i] & 0xFFFF0000u);
+      ps.Qt[e0 + 2 * i][tt] = __uint_as_float(qu[i] << 16);
+      ps.Qt[e0 + 2 * i + 1][tt] = __uint_as_float(qu[i] & 0xFFFF0000u);
+    }
   }
   if (tid < kGdnC) {
     const bool in = tid < n;
@@ -240,11 +261,15 @@ __global__ void __launch_bounds__(kPrepThreads) gdn_prep_kernel(const GdnArgs g)
   if (tid == 0)
     for (int tt = 1; tt < kGdnC; ++tt) ps.lg_s[tt] += ps.lg_s[tt - 1];
   __syncthreads();
+  if (tid < kGdnC) ps.bg_s[tid] = ps.beta_s[tid] * exp2f(ps.lg_s[tid]);
   // K K^T and Q K^T: thread (ty, tx) owns rows 4 ty .. 4 ty + 3, columns 4 tx .. 4 tx + 3
+  // (tiles wholly past the chunk's n tokens or above the diagonal are zero)
   {
     const int ty = tid / 16, tx = tid % 16;
     float gk[4][4] = {}, qk[4][4] = {};
-    for (int e = 0; e < kGdnD; ++e) {
+    const bool live = 4 * ty < n && tx <= ty;
+#pragma unroll 4
+    for (int e = 0; live && e < kGdnD; ++e) {
       const float4 kr = *reinterpret_cast<const float4*>(&ps.Kt[e][4 * ty]);
       const float4 qr = *reinterpret_cast<const float4*>(&ps.Qt[e][4 * ty]);
       const float4 kc = *reinterpret_cast<const float4*>(&ps.Kt[e][4 * tx]);
@@ -278,10 +303,11 @@ __global__ void __launch_bounds__(kPrepThreads) gdn_prep_kernel(const GdnArgs g)
   float X[kGdnC];
 #pragma unroll
   for (int tt = 0; tt < kGdnC; ++tt) {
-    float b = 0.f;
-    if (tt < n)
-      b = j < kGdnD ? ps.beta_s[tt] * exp2f(ps.lg_s[tt]) * ps.Kt[j][tt]
-                    : ps.beta_s[tt] * __bfloat162float(vv[((r0 + tt) * g.H + h) * kGdnD + (j - kGdnD)]);
+    if (tt >= n) {  // rows past n are zero (zero right-hand side, zero A)
+      X[tt] = 0.f;
+      continue;
+    }
+    const float b = j < kGdnD ? ps.bg_s[tt] * ps.Kt[j][tt] : ps.beta_s[tt] * __bfloat162float(ps.V[tt][j - kGdnD]);
     float a0 = b, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
     for (int i = 0; i + 3 < tt; i += 4) {
@@ -393,6 +419,7 @@ __global__ void __launch_bounds__(kScanThreads) gdn_scan_kernel(const GdnArgs g)
     // step 1: U = U' - W S^T for tokens 4 ut .., rows 2 ur ..
     {
       float acc[4][2] = {};
+#pragma unroll 8
       for (int e = 0; e < kGdnD; ++e) {
         const float4 w = *reinterpret_cast<const float4*>(&b.Wt[e][4 * ut]);
         const float2 sv = *reinterpret_cast<const float2*>(&sm.St[e][2 * ur]);
@@ -427,6 +454,7 @@ __global__ void __launch_bounds__(kScanThreads) gdn_scan_kernel(const GdnArgs g)
       for (int x = 0; x < 4; ++x)
 #pragma unroll
         for (int y = 0; y < 4; ++y) acc[x][y] = gnv * sm.St[4 * se + x][4 * sr + y];
+#pragma unroll 4
       for (int tt = 0; tt < n; ++tt) {
         const uint2 kw = *reinterpret_cast<const uint2*>(&b.K[tt][4 * se]);
         const float kv[4] = {__uint_as_float(kw.x << 16), __uint_as_float(kw.x & 0xFFFF0000u),
@@ -476,13 +504,27 @@ __global__ void __launch_bounds__(kOutThreads) gdn_out_kernel(const GdnArgs g) {
   const float* cd = chunk_ptr(g, chunk, h);
   const int j0 = half * kOutCols;
   const float* S0 = c > 0 ? g.ckpt + ((long long)(g.ck_off[t] + c - 1) * g.H + h) * kGdnD * kGdnD : nullptr;
-  for (int idx = tid; idx < kOutCols * kGdnD; idx += kOutThreads) {  // S0 rows j0 .. j0 + 63
-    const int j = idx / kGdnD, e = idx % kGdnD;
-    sm.St[e][j] = S0 ? S0[(long long)(j0 + j) * kGdnD + e] : 0.f;
+#pragma unroll 4
+  for (int idx = tid; idx < kOutCols * (kGdnD / 4); idx += kOutThreads) {  // S0 rows j0 .. j0 + 63
+    const int j = idx % kOutCols, e0 = 4 * (idx / kOutCols);  // lanes: consecutive rows
+    const float4 v = S0 ? *reinterpret_cast<const float4*>(S0 + (long long)(j0 + j) * kGdnD + e0)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    sm.St[e0][j] = v.x;
+    sm.St[e0 + 1][j] = v.y;
+    sm.St[e0 + 2][j] = v.z;
+    sm.St[e0 + 3][j] = v.w;
   }
-  for (int idx = tid; idx < kGdnC * kGdnD; idx += kOutThreads) {
-    const int tt = idx / kGdnD, e = idx % kGdnD;
-    sm.Qt[e][tt] = tt < n ? __bfloat162float(qq[((r0 + tt) * g.H + h) * kGdnD + e]) : 0.f;
+#pragma unroll 2
+  for (int idx = tid; idx < kGdnC * (kGdnD / 8); idx += kOutThreads) {
+    const int tt = idx % kGdnC, e0 = 8 * (idx / kGdnC);  // lanes: consecutive tokens
+    uint4 qw = make_uint4(0u, 0u, 0u, 0u);
+    if (tt < n) qw = *reinterpret_cast<const uint4*>(qq + ((r0 + tt) * g.H + h) * kGdnD + e0);
+    const uint32_t qu[4] = {qw.x, qw.y, qw.z, qw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      sm.Qt[e0 + 2 * i][tt] = __uint_as_float(qu[i] << 16);
+      sm.Qt[e0 + 2 * i + 1][tt] = __uint_as_float(qu[i] & 0xFFFF0000u);
+    }
   }
   for (int idx = tid; idx < kGdnC * kGdnC / 4; idx += kOutThreads) {
     const int tt = idx / (kGdnC / 4), pc = idx % (kGdnC / 4);
@@ -497,6 +539,7 @@ __global__ void __launch_bounds__(kOutThreads) gdn_out_kernel(const GdnArgs g) {
   __syncthreads();
   const int ty = tid / 16, tx = tid % 16;  // tokens 4 ty .., columns 4 tx ..
   float acc[4][4] = {};
+#pragma unroll 8
   for (int e = 0; e < kGdnD; ++e) {  // Q S0^T
     const float4 a = *reinterpret_cast<const float4*>(&sm.Qt[e][4 * ty]);
     const float4 b = *reinterpret_cast<const float4*>(&sm.St[e][4 * tx]);
@@ -513,6 +556,7 @@ __global__ void __launch_bounds__(kOutThreads) gdn_out_kernel(const GdnArgs g) {
     for (int y = 0; y < 4; ++y) acc[x][y] *= gt;
   }
   const int imax = min(n, 4 * ty + 4);  // P is zero past the diagonal
+#pragma unroll 4
   for (int i = 0; i < imax; ++i) {      // + P U
     const float4 b = *reinterpret_cast<const float4*>(&sm.U[i][4 * tx]);
     const float bv[4] = {b.x, b.y, b.z, b.w};
