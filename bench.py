@@ -96,6 +96,36 @@ def visible_pairs(case) -> int:
     return total
 
 
+def attention_executed_flops(meta: np.ndarray, Hkv: int, G: int, d: int) -> float:
+    """FLOPs the tensor-core tree attention issues for one run of query-tile
+    records (the kernel's own metadata, in launch order): per (query head, tile
+    slot) and visited 128-column key block, Q K^T and P V of 128 x 128 x d each.
+    Work items follow the kernel: per pair of tiles (2k, 2k+1), two heads of one
+    tile per item, and for odd G the last head of each KV group on both tiles of
+    a pair over the union of their column spans (one tile at a time when the
+    pair straddles two trees).  Columns come in whole blocks: the trunk span
+    [tree_base, max trunk_hi) and the branch span [min br_lo, max br_hi)."""
+    def nblk(ms):
+        base = int(ms[0][2])
+        n = -(-(max(int(m[3]) for m in ms) - base) // 128)
+        br = [(int(m[5]), int(m[6])) for m in ms if m[6] > m[5]]
+        if br:
+            n += -(-(max(h for _, h in br) - min(lo for lo, _ in br)) // 128)
+        return n
+    nt = len(meta)
+    slots = 0
+    for k in range((nt + 1) // 2):
+        tiles = [t for t in (2 * k, 2 * k + 1) if t < nt]
+        for t in tiles:
+            slots += 2 * (G // 2) * Hkv * nblk([meta[t]])
+        if G % 2:
+            if len(tiles) == 2 and meta[tiles[0]][2] == meta[tiles[1]][2]:
+                slots += 2 * Hkv * nblk([meta[t] for t in tiles])
+            else:
+                slots += sum(Hkv * nblk([meta[t]]) for t in tiles)
+    return 4.0 * d * 128 * 128 * slots
+
+
 def case_figures(case):
     pairs = visible_pairs(case)
     flops = 4.0 * case.d * case.Hq * pairs
@@ -323,6 +353,11 @@ def run_gpu(args):
     torch.cuda.synchronize()
     if st.check_status() != 0:
         raise RuntimeError(f"device status {st.check_status()}")
+    # the attention's executed FLOPs, from the tile records its launch reads
+    meta = st.tile_meta[t0:t1] if split else st.tile_meta[:st.num_tiles]
+    attn_exec = attention_executed_flops(meta.cpu().numpy(), case.Hkv, case.Hq // case.Hkv, case.d)
+    if split:
+        attn_exec = float(PAR.global_count(attn_exec, device=dev))
 
     clocks = ClockSampler(dev.index if dev.index is not None else 0)
     clocks.start()
@@ -391,7 +426,9 @@ def run_gpu(args):
     kernels = {
         "tree_attention": {"bound": "tensor", "ms": t_attn, "achieved": attn_tflops, "unit": "TFLOP/s",
                            "peak": peaks["bf16"], "frac": attn_tflops / peaks["bf16"],
-                           "useful_flops": figs["flops"], "visible_pairs": figs["pairs"]},
+                           "useful_flops": figs["flops"], "visible_pairs": figs["pairs"],
+                           "executed_flops": attn_exec, "useful_over_executed": figs["flops"] / attn_exec,
+                           "executed_tflops": attn_exec / (t_attn * 1e-3) / 1e12},
         "tv_overlap_e2e": {"bound": "hbm", "ms": t_ov, "achieved": ov_gbs, "unit": "GB/s", "peak": peaks["hbm"],
                            "frac": ov_gbs / peaks["hbm"], "algorithmic_bytes": figs["ov_bytes"]},
         "build_tree_mask": {"ms": t_mask},

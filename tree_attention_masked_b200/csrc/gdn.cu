@@ -18,7 +18,8 @@
 // is the unit lower-triangular system
 //   (I + A) U = diag(beta) (V - diag(g) K S0^T),  A_ti = beta_t (g_t/g_i) (k_t . k_i), i < t,
 // and  O = diag(g) Q S0^T + (L o Q K^T) U,  S_C = g_C S0 + (diag(g_C/g) U)^T K.
-// Four kernels, fp32 arithmetic throughout:
+// Four kernels; fp32 arithmetic throughout, the output phase's products on the
+// tensor cores with fp32 operands split into bf16 pairs:
 //   gdn_prep_kernel   -- per (trunk chunk, head), in parallel: A, W = (I+A)^-1 diag(beta g) K and
 //                        U' = (I+A)^-1 diag(beta) V (so U = U' - W S0^T), the decay-
 //                        weighted Q K^T and the decay ratios;
@@ -26,7 +27,7 @@
 //                        chunk by chunk: the checkpoint at each chunk start,
 //                        U = U' - W S0^T, S <- g_C S + (diag(g_C/g) U)^T K;
 //   gdn_out_kernel    -- per (trunk chunk, head, half of the columns), in parallel:
-//                        the trunk rows' outputs;
+//                        the trunk rows' outputs (tcgen05 MMAs, TMEM accumulators);
 //   gdn_branch_kernel -- per (branch, head, 32 state rows): the state after the
 //                        anchor from the checkpoint of its chunk plus that chunk's
 //                        first m + 1 update vectors (the indexed state replay of the
@@ -37,6 +38,7 @@
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace specopd {
 namespace {
@@ -476,25 +478,56 @@ __global__ void __launch_bounds__(kScanThreads) gdn_scan_kernel(const GdnArgs g)
   if (T % kGdnC == 0 && nch > 0) store_ckpt(nch);
 }
 
-// Phase C: outputs of the trunk rows, one CTA per (chunk, head, half of the
-// 128 value columns), 256 threads: with S0 the state at the chunk start (zero,
-// or its checkpoint),  O = diag(g) Q S0^T + P U  on the half's 64 columns.
-// fp32 products in registers: each thread owns 4 tokens x 4 columns.
+// Phase C: outputs of the trunk rows on the tensor cores, one CTA per (chunk,
+// head, half of the 128 value columns), 256 threads.  With S0 the state at
+// the chunk start (zero, or its checkpoint):  O = diag(g) Q S0^T + P U.  Q is
+// exact in bf16; S0, P and U are fp32 and enter the MMAs as bf16 pairs
+// x = hi + lo (hi = bf16(x), lo = bf16(x - hi), together about 16 mantissa
+// bits), so
+//   Q S0^T = Q S0hi^T + Q S0lo^T,    P U = Phi Uhi + Phi Ulo + Plo Uhi
+// (the dropped Plo Ulo term is about 2^-16 of P U), accumulated in fp32 in
+// TMEM: R1 = Q S0^T (columns 0..63), R2 = P U (columns 64..127).  All threads
+// stage the operands into K-major 128-byte-swizzled panels (8-row x 128-byte
+// atoms, 16-byte chunk j of row r at chunk j ^ (r mod 8)), first Q and S0,
+// then, once those MMAs are done, P and U in the same 64 KB (three CTAs share
+// an SM); M is 128 with the rows past the chunk's 64 tokens zero.  One thread
+// issues the MMAs (kind::f16, bf16 in, fp32 accumulate) and commits each
+// group to an mbarrier; the warps that own TMEM lanes 0..63 form g_t R1 + R2.
 constexpr int kOutThreads = 256;
-constexpr int kOutCols = kGdnD / 2;
+constexpr uint32_t kPanel = 128 * 128;  // [128 rows][64 bf16] swizzled panel, bytes
+constexpr uint32_t kHalfPanel = 64 * 128;
 
-struct OutSmem {
-  float St[kGdnD][kTP];    // S0^T of the half's columns: St[e][j]
-  float Qt[kGdnD][kTP];    // Q^T
-  float P[kGdnC][kGdnC + 4];
-  float U[kGdnC][kTP];     // the half's columns of U
+struct OutTcSmem {
+  // GEMM 1: Q (two panels, K = 128) | S0 rows of the half, hi and lo (two 64-row panels each)
+  // GEMM 2: P hi, lo (one panel each, K = 64) | U^T rows of the half, hi and lo (one 64-row panel each)
+  uint8_t buf[4 * kPanel];
+  uint64_t done;
+  uint32_t tmem;
+  int abort_flag;
   float lg[kGdnC];
 };
+constexpr uint32_t kOutAq = 0, kOutBsHi = 2 * kPanel, kOutBsLo = 3 * kPanel;
+constexpr uint32_t kOutApHi = 0, kOutApLo = kPanel, kOutBuHi = 2 * kPanel, kOutBuLo = 2 * kPanel + kHalfPanel;
+
+__device__ __forceinline__ uint32_t swz(int r, int j) { return (uint32_t)r * 128u + (uint32_t)((j ^ (r & 7)) << 4); }
+
+// eight fp32 values -> bf16 hi (rounded) and lo (rounded remainder), packed
+__device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    h[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+    l[i] = pack_bf16x2(x[2 * i] - __uint_as_float(h[i] << 16), x[2 * i + 1] - __uint_as_float(h[i] & 0xFFFF0000u));
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
 
 __global__ void __launch_bounds__(kOutThreads) gdn_out_kernel(const GdnArgs g) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  OutSmem& sm = *reinterpret_cast<OutSmem*>(smem_raw);
-  const int chunk = blockIdx.x, h = blockIdx.y, half = blockIdx.z, tid = threadIdx.x;
+  extern __shared__ uint8_t smem_raw[];
+  OutTcSmem& sm = *reinterpret_cast<OutTcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int chunk = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int v0 = blockIdx.z * 64;
   int t = 0;
   while (t + 1 < g.tp.num_trees && g.ch_off[t + 1] <= chunk) ++t;
   const int c = chunk - g.ch_off[t];
@@ -502,77 +535,142 @@ __global__ void __launch_bounds__(kOutThreads) gdn_out_kernel(const GdnArgs g) {
   const int n = min(kGdnC, g.tp.trunk_len[t] - c * kGdnC);
   const __nv_bfloat16* qq = static_cast<const __nv_bfloat16*>(g.q);
   const float* cd = chunk_ptr(g, chunk, h);
-  const int j0 = half * kOutCols;
   const float* S0 = c > 0 ? g.ckpt + ((long long)(g.ck_off[t] + c - 1) * g.H + h) * kGdnD * kGdnD : nullptr;
-#pragma unroll 4
-  for (int idx = tid; idx < kOutCols * (kGdnD / 4); idx += kOutThreads) {  // S0 rows j0 .. j0 + 63
-    const int j = idx % kOutCols, e0 = 4 * (idx / kOutCols);  // lanes: consecutive rows
-    const float4 v = S0 ? *reinterpret_cast<const float4*>(S0 + (long long)(j0 + j) * kGdnD + e0)
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
-    sm.St[e0][j] = v.x;
-    sm.St[e0 + 1][j] = v.y;
-    sm.St[e0 + 2][j] = v.z;
-    sm.St[e0 + 3][j] = v.w;
+  uint8_t* buf = sm.buf;
+  const uint32_t sb = smem_u32(buf);
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 64, false);
+  if (tid == 0) {
+    mbar_init(&sm.done, 1);
+    sm.abort_flag = 0;
+    fence_barrier_init();
   }
-#pragma unroll 2
-  for (int idx = tid; idx < kGdnC * (kGdnD / 8); idx += kOutThreads) {
-    const int tt = idx % kGdnC, e0 = 8 * (idx / kGdnC);  // lanes: consecutive tokens
-    uint4 qw = make_uint4(0u, 0u, 0u, 0u);
-    if (tt < n) qw = *reinterpret_cast<const uint4*>(qq + ((r0 + tt) * g.H + h) * kGdnD + e0);
-    const uint32_t qu[4] = {qw.x, qw.y, qw.z, qw.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      sm.Qt[e0 + 2 * i][tt] = __uint_as_float(qu[i] << 16);
-      sm.Qt[e0 + 2 * i + 1][tt] = __uint_as_float(qu[i] & 0xFFFF0000u);
-    }
-  }
-  for (int idx = tid; idx < kGdnC * kGdnC / 4; idx += kOutThreads) {
-    const int tt = idx / (kGdnC / 4), pc = idx % (kGdnC / 4);
-    *reinterpret_cast<float4*>(&sm.P[tt][4 * pc]) = *reinterpret_cast<const float4*>(cd + kOffP + tt * kGdnC + 4 * pc);
-  }
-  for (int idx = tid; idx < kGdnC * kOutCols / 4; idx += kOutThreads) {
-    const int tt = idx / (kOutCols / 4), pc = idx % (kOutCols / 4);
-    *reinterpret_cast<float4*>(&sm.U[tt][4 * pc]) =
-        tt < n ? *reinterpret_cast<const float4*>(cd + kOffU + tt * kGdnD + j0 + 4 * pc) : make_float4(0.f, 0.f, 0.f, 0.f);
+  if (warp == 0) {
+    tmem_alloc(&sm.tmem, 128);
+    tmem_relinquish();
   }
   if (tid < kGdnC) sm.lg[tid] = cd[kOffLg + tid];
+  uint32_t phase = 0;
+  bool ok = true;
+  if (S0) {
+    // ---- GEMM 1 operands: Q rows (rows >= n zero), S0 rows v0 .. v0 + 63
+    for (int idx = tid; idx < 128 * 16; idx += kOutThreads) {
+      const int r = idx >> 4, j = idx & 15;
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (r < n) w = *reinterpret_cast<const uint4*>(qq + ((r0 + r) * g.H + h) * kGdnD + 8 * j);
+      *reinterpret_cast<uint4*>(buf + kOutAq + (j >> 3) * kPanel + swz(r, j & 7)) = w;
+    }
+#pragma unroll 2
+    for (int idx = tid; idx < 64 * 16; idx += kOutThreads) {
+      const int v = idx >> 4, j = idx & 15;
+      const float* src = S0 + (v0 + v) * kGdnD + 8 * j;
+      const float4 a = *reinterpret_cast<const float4*>(src);
+      const float4 b = *reinterpret_cast<const float4*>(src + 4);
+      const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      uint4 hi, lo;
+      split8(x, hi, lo);
+      const uint32_t off = (j >> 3) * kHalfPanel + swz(v, j & 7);
+      *reinterpret_cast<uint4*>(buf + kOutBsHi + off) = hi;
+      *reinterpret_cast<uint4*>(buf + kOutBsLo + off) = lo;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+      const uint32_t tmem = sm.tmem;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {  // K = 128 in steps of 16: panel ks / 4, 32 bytes per step
+        const uint64_t a = smem_desc_sw128(sb + kOutAq + (ks >> 2) * kPanel + (ks & 3) * 32, 16, 1024);
+        const uint32_t boff = (ks >> 2) * kHalfPanel + (ks & 3) * 32;
+        mma_ss(tmem, a, smem_desc_sw128(sb + kOutBsHi + boff, 16, 1024), idesc, ks > 0 ? 1u : 0u);
+        mma_ss(tmem, a, smem_desc_sw128(sb + kOutBsLo + boff, 16, 1024), idesc, 1u);
+      }
+      mma_commit(&sm.done);
+    }
+    // the buffer is reused: every thread waits for GEMM 1 to finish reading it
+    ok = mbar_wait_warp(&sm.done, 0, &sm.abort_flag);
+    tc_fence_after();
+    phase = 1;
+  }
+  // ---- GEMM 2 operands: P rows (rows >= n zero), U^T rows v0 .. v0 + 63 (tokens >= n zero)
+  for (int idx = tid; idx < 128 * 8; idx += kOutThreads) {
+    const int r = idx >> 3, j = idx & 7;
+    float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (r < n) {
+      const float4 a = *reinterpret_cast<const float4*>(cd + kOffP + r * kGdnC + 8 * j);
+      const float4 b = *reinterpret_cast<const float4*>(cd + kOffP + r * kGdnC + 8 * j + 4);
+      x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    }
+    uint4 hi, lo;
+    split8(x, hi, lo);
+    *reinterpret_cast<uint4*>(buf + kOutApHi + swz(r, j)) = hi;
+    *reinterpret_cast<uint4*>(buf + kOutApLo + swz(r, j)) = lo;
+  }
+  for (int idx = tid; idx < 64 * 8; idx += kOutThreads) {
+    const int v = idx & 63, j = idx >> 6;
+    float x[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int i = 8 * j + q;
+      x[q] = i < n ? cd[kOffU + i * kGdnD + v0 + v] : 0.f;
+    }
+    uint4 hi, lo;
+    split8(x, hi, lo);
+    *reinterpret_cast<uint4*>(buf + kOutBuHi + swz(v, j)) = hi;
+    *reinterpret_cast<uint4*>(buf + kOutBuLo + swz(v, j)) = lo;
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
   __syncthreads();
-  const int ty = tid / 16, tx = tid % 16;  // tokens 4 ty .., columns 4 tx ..
-  float acc[4][4] = {};
-#pragma unroll 8
-  for (int e = 0; e < kGdnD; ++e) {  // Q S0^T
-    const float4 a = *reinterpret_cast<const float4*>(&sm.Qt[e][4 * ty]);
-    const float4 b = *reinterpret_cast<const float4*>(&sm.St[e][4 * tx]);
-    const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem;
+  if (tid == 0) {
 #pragma unroll
-    for (int x = 0; x < 4; ++x)
-#pragma unroll
-      for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
+    for (int ks = 0; ks < 4; ++ks) {  // K = 64
+      const uint32_t off = ks * 32;
+      const uint64_t ph = smem_desc_sw128(sb + kOutApHi + off, 16, 1024);
+      const uint64_t pl = smem_desc_sw128(sb + kOutApLo + off, 16, 1024);
+      const uint64_t uh = smem_desc_sw128(sb + kOutBuHi + off, 16, 1024);
+      const uint64_t ul = smem_desc_sw128(sb + kOutBuLo + off, 16, 1024);
+      mma_ss(tmem + 64, ph, uh, idesc, ks > 0 ? 1u : 0u);
+      mma_ss(tmem + 64, ph, ul, idesc, 1u);
+      mma_ss(tmem + 64, pl, uh, idesc, 1u);
+    }
+    mma_commit(&sm.done);
   }
+  // ---- epilogue: warps 0, 1 (columns 0..31 of the half) and 4, 5 (32..63) own TMEM lanes 0..63
+  if ((warp & 3) < 2) {
+    if (ok && mbar_wait_warp(&sm.done, phase, &sm.abort_flag)) {
+      tc_fence_after();
+      const int row = 32 * (warp & 3) + lane;
+      const int cb = warp >= 4 ? 32 : 0;
+      const uint32_t ta = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+      uint32_t a[32], b[32];
+      tmem_ld32(ta + 64 + cb, b);
+      if (S0) tmem_ld32(ta + cb, a);
+      tmem_ld_wait();
+      if (row < n) {
+        const float gt = exp2f(sm.lg[row]);
+        float* orow = g.out + ((r0 + row) * g.H + h) * kGdnD + v0 + cb;
 #pragma unroll
-  for (int x = 0; x < 4; ++x) {
-    const float gt = exp2f(sm.lg[4 * ty + x]);
-#pragma unroll
-    for (int y = 0; y < 4; ++y) acc[x][y] *= gt;
-  }
-  const int imax = min(n, 4 * ty + 4);  // P is zero past the diagonal
-#pragma unroll 4
-  for (int i = 0; i < imax; ++i) {      // + P U
-    const float4 b = *reinterpret_cast<const float4*>(&sm.U[i][4 * tx]);
-    const float bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int x = 0; x < 4; ++x) {
-      const float p = sm.P[4 * ty + x][i];
-#pragma unroll
-      for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(p, bv[y], acc[x][y]);
+        for (int e = 0; e < 32; e += 4) {
+          float4 o;
+          o.x = S0 ? fmaf(gt, __uint_as_float(a[e]), __uint_as_float(b[e])) : __uint_as_float(b[e]);
+          o.y = S0 ? fmaf(gt, __uint_as_float(a[e + 1]), __uint_as_float(b[e + 1])) : __uint_as_float(b[e + 1]);
+          o.z = S0 ? fmaf(gt, __uint_as_float(a[e + 2]), __uint_as_float(b[e + 2])) : __uint_as_float(b[e + 2]);
+          o.w = S0 ? fmaf(gt, __uint_as_float(a[e + 3]), __uint_as_float(b[e + 3])) : __uint_as_float(b[e + 3]);
+          *reinterpret_cast<float4*>(orow + e) = o;
+        }
+      }
+    } else if (lane == 0) {
+      atomicOr(reinterpret_cast<unsigned*>(g.status), SPECOPD_FLAG_TIMEOUT);
     }
   }
-#pragma unroll
-  for (int x = 0; x < 4; ++x) {
-    const int tt = 4 * ty + x;
-    if (tt < n)
-      *reinterpret_cast<float4*>(g.out + ((r0 + tt) * g.H + h) * kGdnD + j0 + 4 * tx) =
-          make_float4(acc[x][0], acc[x][1], acc[x][2], acc[x][3]);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
   }
 }
 
@@ -691,9 +789,9 @@ cudaError_t launch_gdn_tree(GdnArgs g, cudaStream_t stream) {
   gdn_scan_kernel<<<dim3(g.tp.num_trees, g.H, kGdnD / kScanRows), kScanThreads, sizeof(ScanSmem), stream>>>(g);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(gdn_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(OutSmem));
+  e = cudaFuncSetAttribute(gdn_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(OutTcSmem) + 1024);
   if (e != cudaSuccess) return e;
-  gdn_out_kernel<<<dim3(coff, g.H, kGdnD / kOutCols), kOutThreads, sizeof(OutSmem), stream>>>(g);
+  gdn_out_kernel<<<dim3(coff, g.H, 2), kOutThreads, sizeof(OutTcSmem) + 1024, stream>>>(g);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (g.tp.total_branches == 0) return cudaSuccess;
