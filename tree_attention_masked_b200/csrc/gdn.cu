@@ -201,27 +201,37 @@ __device__ __forceinline__ float* chunk_ptr(const GdnArgs& g, long long chunk, i
 
 // Phase A: one CTA per (trunk chunk of at most C tokens, head), 256 threads.  With the
 // chunk's cumulative decays g_t = prod_{i<=t} alpha_i (as log2 g):
-//   Gram K K^T and Q K^T in 4 x 4 register tiles over transposed K, Q;
+//   Gram [K; Q] K^T on the tensor cores (bf16 products are exact in fp32): one
+//   M = 128, N = 64, K = 128 MMA group, the K panel serving as both operands;
 //   A_ti = beta_t (g_t/g_i) (k_t . k_i), i < t;   P_ti = (g_t/g_i)(q_t . k_i), i <= t;
 //   (I + A) X = B by forward substitution, one right-hand-side column per
 //   thread in registers: B = diag(beta g) K gives W, B = diag(beta) V gives U'
 //   (so a start state S0 gives the chunk's update vectors U = U' - W S0^T);
 //   coef_t = g_n / g_t, the decay from token t to the chunk's end.
 constexpr int kPrepThreads = 2 * kGdnD;
-constexpr int kTP = kGdnC + 4;  // padded row of a transposed [128][64] tile
+constexpr int kAsP = kGdnC + 4;  // padded row of A (16-byte aligned rows, 4 banks apart)
+constexpr uint32_t kPanel = 128 * 128;  // [128 rows][64 bf16] 128-byte-swizzled panel, bytes
 
 struct PrepSmem {
-  float Kt[kGdnD][kTP];
-  float Qt[kGdnD][kTP];
-  float As[kGdnC][kGdnC];
+  uint8_t kq[2 * kPanel];  // rows 0..63: K, rows 64..127: Q (zero past n); K = 128 in two panels
+  float As[kGdnC][kAsP];
   __nv_bfloat16 V[kGdnC][kGdnD];
   float lg_s[kGdnC], beta_s[kGdnC], bg_s[kGdnC];  // log2 g_t, beta_t, beta_t g_t
+  uint64_t done;
+  uint32_t tmem;
+  int abort_flag;
 };
 
+// byte offset of element (r, k) of a [rows][128] bf16 operand in two 128-byte-swizzled panels
+__device__ __forceinline__ uint32_t swz(int r, int j) { return (uint32_t)r * 128u + (uint32_t)((j ^ (r & 7)) << 4); }
+__device__ __forceinline__ uint32_t swz_elem(int r, int k) {
+  return (uint32_t)(k >> 6) * kPanel + swz(r, (k & 63) >> 3) + (uint32_t)(k & 7) * 2u;
+}
+
 __global__ void __launch_bounds__(kPrepThreads) gdn_prep_kernel(const GdnArgs g) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  PrepSmem& ps = *reinterpret_cast<PrepSmem*>(smem_raw);
-  const int chunk = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+  extern __shared__ uint8_t smem_raw[];
+  PrepSmem& ps = *reinterpret_cast<PrepSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int chunk = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int t = 0;
   while (t + 1 < g.tp.num_trees && g.ch_off[t + 1] <= chunk) ++t;
   const int c = chunk - g.ch_off[t];
@@ -231,75 +241,94 @@ __global__ void __launch_bounds__(kPrepThreads) gdn_prep_kernel(const GdnArgs g)
   const __nv_bfloat16* qq = static_cast<const __nv_bfloat16*>(g.q);
   const __nv_bfloat16* vv = static_cast<const __nv_bfloat16*>(g.v);
   float* cd = chunk_ptr(g, chunk, h);
-  // 8 consecutive elements (16 bytes) of a token's k, q and v per step; the
-  // lanes of a warp take consecutive tokens, so the transposed stores hit
-  // consecutive banks
+  if (tid == 0) {
+    mbar_init(&ps.done, 1);
+    ps.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&ps.tmem, 64);
+    tmem_relinquish();
+  }
+  // 16 bytes of a token's k, q and v per step
 #pragma unroll 2
   for (int idx = tid; idx < kGdnC * (kGdnD / 8); idx += kPrepThreads) {
-    const int tt = idx % kGdnC, e0 = 8 * (idx / kGdnC);
+    const int tt = idx >> 4, j = idx & 15;
     uint4 kw = make_uint4(0u, 0u, 0u, 0u), qw = kw, vw = kw;
     if (tt < n) {
-      const long long off = ((r0 + tt) * g.H + h) * kGdnD + e0;
+      const long long off = ((r0 + tt) * g.H + h) * kGdnD + 8 * j;
       kw = *reinterpret_cast<const uint4*>(kk + off);
       qw = *reinterpret_cast<const uint4*>(qq + off);
       vw = *reinterpret_cast<const uint4*>(vv + off);
     }
-    *reinterpret_cast<uint4*>(&ps.V[tt][e0]) = vw;
-    const uint32_t ku[4] = {kw.x, kw.y, kw.z, kw.w}, qu[4] = {qw.x, qw.y, qw.z, qw.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      ps.Kt[e0 + 2 * i][tt] = __uint_as_float(ku[i] << 16);
-      ps.Kt[e0 + 2 * i + 1][tt] = __uint_as_float(ku[i] & 0xFFFF0000u);
-      ps.Qt[e0 + 2 * i][tt] = __uint_as_float(qu[i] << 16);
-      ps.Qt[e0 + 2 * i + 1][tt] = __uint_as_float(qu[i] & 0xFFFF0000u);
-    }
+    *reinterpret_cast<uint4*>(ps.kq + (j >> 3) * kPanel + swz(tt, j & 7)) = kw;
+    *reinterpret_cast<uint4*>(ps.kq + (j >> 3) * kPanel + swz(kGdnC + tt, j & 7)) = qw;
+    *reinterpret_cast<uint4*>(&ps.V[tt][8 * j]) = vw;
   }
   if (tid < kGdnC) {
     const bool in = tid < n;
     ps.lg_s[tid] = in ? log2f(g.alpha[(r0 + tid) * g.H + h]) : 0.f;
     ps.beta_s[tid] = in ? g.beta[(r0 + tid) * g.H + h] : 0.f;
   }
+  fence_proxy_async_smem();
+  tc_fence_before();
   __syncthreads();
-  if (tid == 0)
+  tc_fence_after();
+  const uint32_t tmem = ps.tmem;
+  if (tid == 0) {
+    constexpr uint32_t idesc = idesc_bf16_f32(128, 64, false);
+    const uint32_t base = smem_u32(ps.kq);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {  // K = 128 in steps of 16: panel ks / 4, 32 bytes per step
+      const uint64_t d = smem_desc_sw128(base + (ks >> 2) * kPanel + (ks & 3) * 32, 16, 1024);
+      mma_ss(tmem, d, d, idesc, ks > 0 ? 1u : 0u);  // B: the panel's first 64 rows (K)
+    }
+    mma_commit(&ps.done);
+  }
+  if (tid == 32)
     for (int tt = 1; tt < kGdnC; ++tt) ps.lg_s[tt] += ps.lg_s[tt - 1];
   __syncthreads();
   if (tid < kGdnC) ps.bg_s[tid] = ps.beta_s[tid] * exp2f(ps.lg_s[tid]);
-  // K K^T and Q K^T: thread (ty, tx) owns rows 4 ty .. 4 ty + 3, columns 4 tx .. 4 tx + 3
-  // (tiles wholly past the chunk's n tokens or above the diagonal are zero)
-  {
-    const int ty = tid / 16, tx = tid % 16;
-    float gk[4][4] = {}, qk[4][4] = {};
-    const bool live = 4 * ty < n && tx <= ty;
-#pragma unroll 4
-    for (int e = 0; live && e < kGdnD; ++e) {
-      const float4 kr = *reinterpret_cast<const float4*>(&ps.Kt[e][4 * ty]);
-      const float4 qr = *reinterpret_cast<const float4*>(&ps.Qt[e][4 * ty]);
-      const float4 kc = *reinterpret_cast<const float4*>(&ps.Kt[e][4 * tx]);
-      const float a[4] = {kr.x, kr.y, kr.z, kr.w}, q[4] = {qr.x, qr.y, qr.z, qr.w}, b[4] = {kc.x, kc.y, kc.z, kc.w};
+  // TMEM lanes 0..63 hold K K^T (warps 0, 1), lanes 64..127 Q K^T (warps 2, 3)
+  if (warp < 4) {
+    if (mbar_wait_warp(&ps.done, 0, &ps.abort_flag)) {
+      tc_fence_after();
+      const int tt = (32 * warp + lane) & (kGdnC - 1);
+      const bool qrow = warp >= 2;
+      const float lgt = ps.lg_s[tt], bt = ps.beta_s[tt];
+      float* prow = cd + kOffP + tt * kGdnC;
 #pragma unroll
-      for (int x = 0; x < 4; ++x)
+      for (int half = 0; half < 2; ++half) {
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + 32 * half, v);
+        tmem_ld_wait();
 #pragma unroll
-        for (int y = 0; y < 4; ++y) {
-          gk[x][y] = fmaf(a[x], b[y], gk[x][y]);
-          qk[x][y] = fmaf(q[x], b[y], qk[x][y]);
+        for (int e = 0; e < 32; e += 4) {
+          float o[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i = 32 * half + e + u;
+            const float ratio = exp2f(lgt - ps.lg_s[i]);
+            const float x = __uint_as_float(v[e + u]);
+            o[u] = qrow ? ((i <= tt && tt < n) ? ratio * x : 0.f) : ((i < tt && tt < n) ? bt * ratio * x : 0.f);
+          }
+          const float4 o4 = make_float4(o[0], o[1], o[2], o[3]);
+          if (qrow)
+            *reinterpret_cast<float4*>(prow + 32 * half + e) = o4;
+          else
+            *reinterpret_cast<float4*>(&ps.As[tt][32 * half + e]) = o4;
         }
-    }
-#pragma unroll
-    for (int x = 0; x < 4; ++x) {
-      const int tt = 4 * ty + x;
-      float4 prow;
-      float* pv = &prow.x;
-#pragma unroll
-      for (int y = 0; y < 4; ++y) {
-        const int i = 4 * tx + y;
-        const float ratio = exp2f(ps.lg_s[tt] - ps.lg_s[i]);
-        ps.As[tt][i] = (i < tt && tt < n) ? ps.beta_s[tt] * ratio * gk[x][y] : 0.f;
-        pv[y] = (i <= tt && tt < n) ? ratio * qk[x][y] : 0.f;
       }
-      *reinterpret_cast<float4*>(cd + kOffP + tt * kGdnC + 4 * tx) = prow;
+    } else if (lane == 0) {
+      atomicOr(reinterpret_cast<unsigned*>(g.status), SPECOPD_FLAG_TIMEOUT);
     }
   }
+  tc_fence_before();
   __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
+  }
   // forward substitution, column j of [W | U'] per thread, in registers
   const int j = tid;
   float X[kGdnC];
@@ -309,7 +338,8 @@ __global__ void __launch_bounds__(kPrepThreads) gdn_prep_kernel(const GdnArgs g)
       X[tt] = 0.f;
       continue;
     }
-    const float b = j < kGdnD ? ps.bg_s[tt] * ps.Kt[j][tt] : ps.beta_s[tt] * __bfloat162float(ps.V[tt][j - kGdnD]);
+    const float b = j < kGdnD ? ps.bg_s[tt] * __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(ps.kq + swz_elem(tt, j)))
+                              : ps.beta_s[tt] * __bfloat162float(ps.V[tt][j - kGdnD]);
     float a0 = b, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
     for (int i = 0; i + 3 < tt; i += 4) {
@@ -323,10 +353,10 @@ __global__ void __launch_bounds__(kPrepThreads) gdn_prep_kernel(const GdnArgs g)
     for (int i = tt & ~3; i < tt; ++i) a0 = fmaf(-ps.As[tt][i], X[i], a0);
     X[tt] = (a0 + a1) + (a2 + a3);
   }
-  if (j < kGdnD) {  // W^T row j: the j-th key element of every token's W row
-    float4* dst = reinterpret_cast<float4*>(cd + kOffW + j * kGdnC);
+  if (j < kGdnD) {  // column j (key element j) of every token's W row
+    float* dst = cd + kOffW + j;
 #pragma unroll
-    for (int tt = 0; tt < kGdnC; tt += 4) dst[tt / 4] = make_float4(X[tt], X[tt + 1], X[tt + 2], X[tt + 3]);
+    for (int tt = 0; tt < kGdnC; ++tt) dst[tt * kGdnD] = X[tt];
   } else {
     float* dst = cd + kOffU + (j - kGdnD);
 #pragma unroll
@@ -339,143 +369,261 @@ __global__ void __launch_bounds__(kPrepThreads) gdn_prep_kernel(const GdnArgs g)
   if (tid < 4) cd[kOffGn + tid] = tid == 0 ? exp2f(ps.lg_s[n - 1]) : 0.f;
 }
 
-// Phase B: the state scan, the only sequential part.  One CTA per (tree, head,
-// 32 rows of S), 256 threads; the rows of S evolve independently, so a CTA
-// carries its rows through the trunk's chunks alone, S^T of its rows in
-// shared memory.  Per chunk c: store the rows of the state at the chunk start
-// (the checkpoint after token C c - 1), then
-//   U = U' - W S^T              (64 tokens x 32 rows; tiles of 4 x 2 per thread),
-//   S <- g_n S + sum_t coef_t U_t k_t^T   (32 rows x 128; tiles of 4 x 4).
-// The next chunk's W^T, K, U' columns and coefficients are copied (cp.async)
-// into the other half of a double buffer during the current chunk.
-constexpr int kScanRows = 32;
+// Phase B: the state scan, the only sequential part, on the tensor cores.  One
+// CTA per (tree, head), 256 threads.  The state S (128 value rows x 128 key
+// elements, fp32) lives in TMEM as an MMA accumulator (lane r = row r).  TMEM
+// columns: S [0, 128), its bf16 split Shi [128, 192) and Slo [192, 256) (two
+// bf16 per column), D = S W^T [256, 320), the split of (coef U)^T: Uhi
+// [320, 352) and Ulo [352, 384).  Per chunk c of n tokens:
+//   warps 0-3, one state row per thread: store the checkpoint (the state at
+//     the chunk start), split S into Shi + Slo, scale S in place by g_n, the
+//     chunk's total decay, and take the row's U' column into registers;
+//   warps 4-7: split the chunk's W into bf16 panels, transpose K into a bf16
+//     panel (exact);
+//   MMA group 1 (A from TMEM):  D = Shi Whi^T + Shi Wlo^T + Slo Whi^T    (M 128, N 64, K 128);
+//   meanwhile every thread prefetches the next chunk's W, U', K and decays
+//     (cp.async) into a raw staging buffer;
+//   warps 0-3:    U = U' - D^T (stored for phases C and D), then coef_t U_t split into Uhi + Ulo;
+//   MMA group 2 (A from TMEM):  S += Uhi^T K + Ulo^T K                   (M 128, N 128, K 64).
+// The fp32 operands enter as bf16 pairs x = hi + lo (about 16 mantissa bits;
+// the dropped lo x lo term is about 2^-16 of a product); K is exact in bf16.
+// Shared-memory operand panels are K-major with the 128-byte swizzle (16-byte
+// chunk j of row r at chunk j ^ (r mod 8)).  Every wait is bounded.
 constexpr int kScanThreads = 256;
-constexpr int kSR = kScanRows + 4;  // padded row of a [.][32] tile
+constexpr uint32_t kHalfPanel = 64 * 128;  // [64 rows][64 bf16] swizzled panel, bytes
+constexpr uint32_t kScS = 0, kScShi = 128, kScSlo = 192, kScD = 256, kScUhi = 320, kScUlo = 352;
 
-struct ScanBuf {
-  float Wt[kGdnD][kTP];
-  __nv_bfloat16 K[kGdnC][kGdnD];
-  float U[kGdnC][kSR];
+struct ScanRaw {  // one chunk record's W, U', decays, and the chunk's K rows, as copied
+  float w[kGdnC][kGdnD];
+  float u[kGdnC][kGdnD];
   float coef[kGdnC + 4];  // g_n / g_t, then g_n
+  __nv_bfloat16 k[kGdnC][kGdnD];
 };
 struct ScanSmem {
-  float St[kGdnD][kSR];  // S^T of this CTA's rows: St[e][r]
-  ScanBuf buf[2];
+  uint8_t w_hi[2 * kHalfPanel], w_lo[2 * kHalfPanel];  // B of group 1: W rows (tokens), K = 128
+  uint8_t kt[kPanel];                                  // B of group 2: K^T rows (key elements), K = 64 tokens
+  ScanRaw raw;
+  float coef[kGdnC];
+  uint64_t bar1, bar2;
+  uint32_t tmem;
+  int abort_flag;
 };
 
-__device__ __forceinline__ void scan_fetch(ScanBuf& b, const GdnArgs& g, int t, int h, int c, int tid) {
-  const int T = g.tp.trunk_len[t];
-  const int n = min(kGdnC, T - c * kGdnC);
-  const long long chunk = g.ch_off[t] + c;
-  const float* cd = chunk_ptr(g, chunk, h);
-  const __nv_bfloat16* kk = static_cast<const __nv_bfloat16*>(g.k);
-  const long long r0 = g.tp.row_base[t] + (long long)c * kGdnC;
-  for (int i = tid; i < kGdnD * (kGdnC / 4); i += kScanThreads) {  // W^T rows: 16 pieces of 4 tokens each
-    const int e = i / (kGdnC / 4), pc = i % (kGdnC / 4);
-    cp_async16(&b.Wt[e][4 * pc], cd + kOffW + e * kGdnC + 4 * pc);
+// eight fp32 values -> bf16 hi (rounded) and lo (rounded remainder), packed
+__device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    h[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+    l[i] = pack_bf16x2(x[2 * i] - __uint_as_float(h[i] << 16), x[2 * i + 1] - __uint_as_float(h[i] & 0xFFFF0000u));
   }
-  for (int i = tid; i < n * (kGdnD / 8); i += kScanThreads) {  // K: 8 bf16 per piece
-    const int tt = i / (kGdnD / 8), pc = i % (kGdnD / 8);
-    cp_async16(&b.K[tt][8 * pc], kk + ((r0 + tt) * g.H + h) * kGdnD + 8 * pc);
-  }
-  for (int i = tid; i < n * (kScanRows / 4); i += kScanThreads) {  // U' of this CTA's rows
-    const int tt = i / (kScanRows / 4), pc = i % (kScanRows / 4);
-    cp_async16(&b.U[tt][4 * pc], cd + kOffU + tt * kGdnD + blockIdx.z * kScanRows + 4 * pc);
-  }
-  for (int i = tid; i < (kGdnC + 4) / 4; i += kScanThreads) cp_async16(&b.coef[4 * i], cd + kOffCoef + 4 * i);
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
-__global__ void __launch_bounds__(kScanThreads) gdn_scan_kernel(const GdnArgs g) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  ScanSmem& sm = *reinterpret_cast<ScanSmem*>(smem_raw);
-  const int t = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
-  const int row0 = blockIdx.z * kScanRows;
+// chunk c's record (W, U', decays) and K rows into the raw buffer; K rows past
+// the chunk's n tokens are zero-filled
+__device__ __forceinline__ void scan_prefetch(ScanRaw& raw, const GdnArgs& g, int t, int h, int c, int tid) {
+  const int T = g.tp.trunk_len[t];
+  const int n = min(kGdnC, T - c * kGdnC);
+  const float* cd = chunk_ptr(g, g.ch_off[t] + c, h);
+  const __nv_bfloat16* kk = static_cast<const __nv_bfloat16*>(g.k);
+  const long long r0 = g.tp.row_base[t] + (long long)c * kGdnC;
+  float* wu = &raw.w[0][0];  // W and U' are adjacent in the record and in the buffer
+  for (int i = tid; i < 2 * kGdnC * kGdnD / 4; i += kScanThreads) cp_async16(wu + 4 * i, cd + kOffW + 4 * i);
+  for (int i = tid; i < (kGdnC + 4) / 4; i += kScanThreads) cp_async16(&raw.coef[4 * i], cd + kOffCoef + 4 * i);
+  for (int i = tid; i < kGdnC * (kGdnD / 8); i += kScanThreads) {
+    const int tt = i >> 4, j = i & 15;
+    if (tt < n)
+      cp_async16(&raw.k[tt][8 * j], kk + ((r0 + tt) * g.H + h) * kGdnD + 8 * j);
+    else
+      *reinterpret_cast<uint4*>(&raw.k[tt][8 * j]) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  cp_async_commit();
+}
+
+__global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(const GdnArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  ScanSmem& sm = *reinterpret_cast<ScanSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int t = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int T = g.tp.trunk_len[t];
   const int nch = (T + kGdnC - 1) / kGdnC;
-  // step-1 tile: tokens 4 ut .. 4 ut + 3, rows 2 ur, 2 ur + 1
-  const int ut = tid / 16, ur = tid % 16;
-  // step-2 tile: key elements 4 se .. 4 se + 3, rows 4 sr .. 4 sr + 3
-  const int se = tid / 8, sr = tid % 8;
-  for (int i = tid; i < kGdnD * kSR; i += kScanThreads) (&sm.St[0][0])[i] = 0.f;
-  auto store_ckpt = [&](int j) {  // rows 4 sr .. 4 sr + 3, elements 4 se .. 4 se + 3 of the state after token C j - 1
-    float* dst = g.ckpt + ((long long)(g.ck_off[t] + j - 1) * g.H + h) * kGdnD * kGdnD;
+  if (tid == 0) {
+    mbar_init(&sm.bar1, 1);
+    mbar_init(&sm.bar2, 1);
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&sm.tmem, 512);
+    tmem_relinquish();
+  }
+  if (nch > 0) scan_prefetch(sm.raw, g, t, h, 0, tid);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem;
+  const int r = 32 * (warp & 3) + lane;  // warps 0-3: state row r = TMEM lane r
+  const uint32_t trow = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+  bool ok = true;
+  // thread r's row of the state after token C j - 1, 32 elements from column 32 q
+  auto store_ckpt_row = [&](int j, int q, const uint32_t (&v)[32]) {
+    float* dst = g.ckpt + ((long long)(g.ck_off[t] + j - 1) * g.H + h) * kGdnD * kGdnD + (long long)r * kGdnD + 32 * q;
 #pragma unroll
-    for (int y = 0; y < 4; ++y) {
-      const int r = 4 * sr + y;
-      *reinterpret_cast<float4*>(dst + (long long)(row0 + r) * kGdnD + 4 * se) =
-          make_float4(sm.St[4 * se][r], sm.St[4 * se + 1][r], sm.St[4 * se + 2][r], sm.St[4 * se + 3][r]);
-    }
+    for (int e = 0; e < 32; e += 4)
+      *reinterpret_cast<float4*>(dst + e) = make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                                                        __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
   };
-  if (nch > 0) scan_fetch(sm.buf[0], g, t, h, 0, tid);
-  cp_async_commit();
   for (int c = 0; c < nch; ++c) {
-    __syncthreads();  // St of the previous chunk is final
-    if (c > 0) store_ckpt(c);
-    if (c + 1 < nch) scan_fetch(sm.buf[(c + 1) & 1], g, t, h, c + 1, tid);
-    cp_async_commit();
-    cp_async_wait<1>();  // chunk c has landed
-    __syncthreads();
-    ScanBuf& b = sm.buf[c & 1];
     const int n = min(kGdnC, T - c * kGdnC);
-    float* Ug = chunk_ptr(g, g.ch_off[t] + c, h) + kOffU;
-    // step 1: U = U' - W S^T for tokens 4 ut .., rows 2 ur ..
-    {
-      float acc[4][2] = {};
-#pragma unroll 8
-      for (int e = 0; e < kGdnD; ++e) {
-        const float4 w = *reinterpret_cast<const float4*>(&b.Wt[e][4 * ut]);
-        const float2 sv = *reinterpret_cast<const float2*>(&sm.St[e][2 * ur]);
-        const float wv[4] = {w.x, w.y, w.z, w.w};
+    float* cd = chunk_ptr(g, g.ch_off[t] + c, h);
+    cp_async_wait<0>();
+    __syncthreads();  // chunk c's raw data is in shared memory
+    float up[kGdnC];  // warps 0-3: column r of U'
+    if (warp < 4) {
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          acc[x][0] = fmaf(wv[x], sv.x, acc[x][0]);
-          acc[x][1] = fmaf(wv[x], sv.y, acc[x][1]);
+      for (int tt = 0; tt < kGdnC; ++tt) up[tt] = sm.raw.u[tt][r];
+      if (c > 0 && ok) {
+        // the state at the chunk start: checkpoint, bf16 split, scale by g_n in place
+        const float gn = sm.raw.coef[kGdnC];
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          uint32_t v[32];
+          tmem_ld32(trow + kScS + 32 * q, v);
+          tmem_ld_wait();
+          store_ckpt_row(c, q, v);
+          uint32_t hi[16], lo[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float x0 = __uint_as_float(v[2 * e]), x1 = __uint_as_float(v[2 * e + 1]);
+            hi[e] = pack_bf16x2(x0, x1);
+            lo[e] = pack_bf16x2(x0 - __uint_as_float(hi[e] << 16), x1 - __uint_as_float(hi[e] & 0xFFFF0000u));
+          }
+          // 32 fp32 columns -> 16 bf16-pair columns of Shi and of Slo
+          tmem_st16(trow + kScShi + 16 * q, hi);
+          tmem_st16(trow + kScSlo + 16 * q, lo);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(gn * __uint_as_float(v[e]));
+          tmem_st32(trow + kScS + 32 * q, v);
+        }
+        tmem_st_wait();
+      }
+    } else {
+      const int u = tid - 128;
+      if (c > 0) {  // W rows (tokens) split into bf16 pairs; rows past n are zero in the record
+#pragma unroll 2
+        for (int idx = u; idx < kGdnC * 16; idx += 128) {
+          const int tt = idx >> 4, j = idx & 15;
+          const float4 a = *reinterpret_cast<const float4*>(&sm.raw.w[tt][8 * j]);
+          const float4 b = *reinterpret_cast<const float4*>(&sm.raw.w[tt][8 * j + 4]);
+          const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+          uint4 hi, lo;
+          split8(x, hi, lo);
+          const uint32_t off = (j >> 3) * kHalfPanel + swz(tt, j & 7);
+          *reinterpret_cast<uint4*>(sm.w_hi + off) = hi;
+          *reinterpret_cast<uint4*>(sm.w_lo + off) = lo;
         }
       }
+      // K^T: row e, tokens 8 j .. 8 j + 7
+      for (int idx = u; idx < kGdnD * 8; idx += 128) {
+        const int e = idx & 127, j = idx >> 7;
+        uint32_t w[4];
 #pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        const int tt = 4 * ut + x;
-        if (tt < n) {
-          const float u0 = b.U[tt][2 * ur] - acc[x][0], u1 = b.U[tt][2 * ur + 1] - acc[x][1];
-          *reinterpret_cast<float2*>(Ug + tt * kGdnD + row0 + 2 * ur) = make_float2(u0, u1);
-          // keep coef_t U_t for the state update
-          b.U[tt][2 * ur] = b.coef[tt] * u0;
-          b.U[tt][2 * ur + 1] = b.coef[tt] * u1;
-        } else {
-          b.U[tt][2 * ur] = 0.f;
-          b.U[tt][2 * ur + 1] = 0.f;
-        }
+        for (int p = 0; p < 4; ++p)
+          w[p] = (uint32_t)__bfloat16_as_ushort(sm.raw.k[8 * j + 2 * p][e]) |
+                 ((uint32_t)__bfloat16_as_ushort(sm.raw.k[8 * j + 2 * p + 1][e]) << 16);
+        *reinterpret_cast<uint4*>(sm.kt + swz(e, j)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
+      if (u < kGdnC) sm.coef[u] = u < n ? sm.raw.coef[u] : 0.f;
     }
+    fence_proxy_async_smem();
+    tc_fence_before();
     __syncthreads();
-    // step 2: S^T[e][r] = g_n S^T[e][r] + sum_t K[t][e] (coef_t U[t][r])
-    {
-      float acc[4][4];
-      const float gnv = b.coef[kGdnC];
+    tc_fence_after();
+    if (c > 0 && tid == 0) {
+      constexpr uint32_t idesc1 = idesc_bf16_f32(128, 64, false);
+      const uint32_t wh = smem_u32(sm.w_hi), wl = smem_u32(sm.w_lo);
 #pragma unroll
-      for (int x = 0; x < 4; ++x)
-#pragma unroll
-        for (int y = 0; y < 4; ++y) acc[x][y] = gnv * sm.St[4 * se + x][4 * sr + y];
-#pragma unroll 4
-      for (int tt = 0; tt < n; ++tt) {
-        const uint2 kw = *reinterpret_cast<const uint2*>(&b.K[tt][4 * se]);
-        const float kv[4] = {__uint_as_float(kw.x << 16), __uint_as_float(kw.x & 0xFFFF0000u),
-                             __uint_as_float(kw.y << 16), __uint_as_float(kw.y & 0xFFFF0000u)};
-        const float4 u = *reinterpret_cast<const float4*>(&b.U[tt][4 * sr]);
-        const float uv[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int x = 0; x < 4; ++x)
-#pragma unroll
-          for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(kv[x], uv[y], acc[x][y]);
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t bo = (ks >> 2) * kHalfPanel + (ks & 3) * 32;
+        const uint64_t b_hi = smem_desc_sw128(wh + bo, 16, 1024), b_lo = smem_desc_sw128(wl + bo, 16, 1024);
+        mma_ts(tmem + kScD, tmem + kScShi + ks * 8, b_hi, idesc1, ks > 0 ? 1u : 0u);
+        mma_ts(tmem + kScD, tmem + kScShi + ks * 8, b_lo, idesc1, 1u);
+        mma_ts(tmem + kScD, tmem + kScSlo + ks * 8, b_hi, idesc1, 1u);
       }
-#pragma unroll
-      for (int x = 0; x < 4; ++x)
-        *reinterpret_cast<float4*>(&sm.St[4 * se + x][4 * sr]) = make_float4(acc[x][0], acc[x][1], acc[x][2], acc[x][3]);
+      mma_commit(&sm.bar1);
     }
+    // the raw buffer is consumed: fetch the next chunk during this one's MMAs
+    if (c + 1 < nch) scan_prefetch(sm.raw, g, t, h, c + 1, tid);
+    if (warp < 4) {
+      // U = U' - (S W^T)^T for thread r's row, stored in place of U'; coef_t U_t split for group 2
+      if (c > 0) {
+        ok = ok && mbar_wait_warp(&sm.bar1, (uint32_t)(c - 1) & 1u, &sm.abort_flag);
+        tc_fence_after();
+      }
+      uint32_t hi[32], lo[32];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        uint32_t v[32];
+        if (c > 0 && ok) {
+          tmem_ld32(trow + kScD + 32 * q, v);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0u;
+        }
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int tt = 32 * q + e;
+          const float u0 = tt < n ? up[tt] - __uint_as_float(v[e]) : 0.f;
+          const float u1 = tt + 1 < n ? up[tt + 1] - __uint_as_float(v[e + 1]) : 0.f;
+          if (tt < n) cd[kOffU + tt * kGdnD + r] = u0;
+          if (tt + 1 < n) cd[kOffU + (tt + 1) * kGdnD + r] = u1;
+          const float c0 = sm.coef[tt] * u0, c1 = sm.coef[tt + 1] * u1;
+          const uint32_t hh = pack_bf16x2(c0, c1);
+          hi[16 * q + e / 2] = hh;
+          lo[16 * q + e / 2] = pack_bf16x2(c0 - __uint_as_float(hh << 16), c1 - __uint_as_float(hh & 0xFFFF0000u));
+        }
+      }
+      tmem_st32(trow + kScUhi, hi);
+      tmem_st32(trow + kScUlo, lo);
+      tmem_st_wait();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+      constexpr uint32_t idesc2 = idesc_bf16_f32(128, 128, false);
+      const uint32_t kb = smem_u32(sm.kt);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint64_t b = smem_desc_sw128(kb + ks * 32, 16, 1024);
+        mma_ts(tmem + kScS, tmem + kScUhi + ks * 8, b, idesc2, (c > 0 || ks > 0) ? 1u : 0u);
+        mma_ts(tmem + kScS, tmem + kScUlo + ks * 8, b, idesc2, 1u);
+      }
+      mma_commit(&sm.bar2);
+    }
+    // every thread: group 2 (and with it group 1) has finished with the panels and TMEM
+    if (!mbar_wait_warp(&sm.bar2, (uint32_t)c & 1u, &sm.abort_flag)) ok = false;
+    tc_fence_after();
   }
   cp_async_wait<0>();
+  if (!ok && lane == 0) atomicOr(reinterpret_cast<unsigned*>(g.status), SPECOPD_FLAG_TIMEOUT);
+  if (warp < 4 && ok && T % kGdnC == 0 && nch > 0) {  // the state after the last token
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+      uint32_t v[32];
+      tmem_ld32(trow + kScS + 32 * q, v);
+      tmem_ld_wait();
+      store_ckpt_row(nch, q, v);
+    }
+  }
+  tc_fence_before();
   __syncthreads();
-  if (T % kGdnC == 0 && nch > 0) store_ckpt(nch);
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
 }
 
 // Phase C: outputs of the trunk rows on the tensor cores, one CTA per (chunk,
@@ -494,9 +642,6 @@ __global__ void __launch_bounds__(kScanThreads) gdn_scan_kernel(const GdnArgs g)
 // issues the MMAs (kind::f16, bf16 in, fp32 accumulate) and commits each
 // group to an mbarrier; the warps that own TMEM lanes 0..63 form g_t R1 + R2.
 constexpr int kOutThreads = 256;
-constexpr uint32_t kPanel = 128 * 128;  // [128 rows][64 bf16] swizzled panel, bytes
-constexpr uint32_t kHalfPanel = 64 * 128;
-
 struct OutTcSmem {
   // GEMM 1: Q (two panels, K = 128) | S0 rows of the half, hi and lo (two 64-row panels each)
   // GEMM 2: P hi, lo (one panel each, K = 64) | U^T rows of the half, hi and lo (one 64-row panel each)
@@ -508,20 +653,6 @@ struct OutTcSmem {
 };
 constexpr uint32_t kOutAq = 0, kOutBsHi = 2 * kPanel, kOutBsLo = 3 * kPanel;
 constexpr uint32_t kOutApHi = 0, kOutApLo = kPanel, kOutBuHi = 2 * kPanel, kOutBuLo = 2 * kPanel + kHalfPanel;
-
-__device__ __forceinline__ uint32_t swz(int r, int j) { return (uint32_t)r * 128u + (uint32_t)((j ^ (r & 7)) << 4); }
-
-// eight fp32 values -> bf16 hi (rounded) and lo (rounded remainder), packed
-__device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
-  uint32_t h[4], l[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    h[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
-    l[i] = pack_bf16x2(x[2 * i] - __uint_as_float(h[i] << 16), x[2 * i + 1] - __uint_as_float(h[i] & 0xFFFF0000u));
-  }
-  hi = make_uint4(h[0], h[1], h[2], h[3]);
-  lo = make_uint4(l[0], l[1], l[2], l[3]);
-}
 
 __global__ void __launch_bounds__(kOutThreads) gdn_out_kernel(const GdnArgs g) {
   extern __shared__ uint8_t smem_raw[];
@@ -779,14 +910,14 @@ cudaError_t launch_gdn_tree(GdnArgs g, cudaStream_t stream) {
   }
   g.ch_off[g.tp.num_trees] = coff;
   cudaError_t e = cudaFuncSetAttribute(gdn_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)sizeof(PrepSmem));
+                                       (int)sizeof(PrepSmem) + 1024);
   if (e != cudaSuccess) return e;
-  gdn_prep_kernel<<<dim3(coff, g.H), kPrepThreads, sizeof(PrepSmem), stream>>>(g);
+  gdn_prep_kernel<<<dim3(coff, g.H), kPrepThreads, sizeof(PrepSmem) + 1024, stream>>>(g);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(gdn_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ScanSmem));
+  e = cudaFuncSetAttribute(gdn_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ScanSmem) + 1024);
   if (e != cudaSuccess) return e;
-  gdn_scan_kernel<<<dim3(g.tp.num_trees, g.H, kGdnD / kScanRows), kScanThreads, sizeof(ScanSmem), stream>>>(g);
+  gdn_scan_kernel<<<dim3(g.tp.num_trees, g.H), kScanThreads, sizeof(ScanSmem) + 1024, stream>>>(g);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(gdn_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(OutTcSmem) + 1024);
