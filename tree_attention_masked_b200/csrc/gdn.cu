@@ -18,23 +18,22 @@
 // is the unit lower-triangular system
 //   (I + A) U = diag(beta) (V - diag(g) K S0^T),  A_ti = beta_t (g_t/g_i) (k_t . k_i), i < t,
 // and  O = diag(g) Q S0^T + (L o Q K^T) U,  S_C = g_C S0 + (diag(g_C/g) U)^T K.
-// Four kernels; fp32 arithmetic throughout, the output phase's products on the
-// tensor cores with fp32 operands split into bf16 pairs:
+// Four kernels, fp32 state and fp32 sums; the products run on the tensor
+// cores (tcgen05, TMEM accumulators) with bf16 inputs exact and fp32 operands
+// split into bf16 pairs (hi + lo), the triangular solves on fp32 FMAs:
 //   gdn_prep_kernel   -- per (trunk chunk, head), in parallel: A, W = (I+A)^-1 diag(beta g) K and
 //                        U' = (I+A)^-1 diag(beta) V (so U = U' - W S0^T), the decay-
 //                        weighted Q K^T and the decay ratios;
-//   gdn_scan_kernel   -- per (tree, head, 32 state rows): the only sequential part,
-//                        chunk by chunk: the checkpoint at each chunk start,
+//   gdn_scan_kernel   -- per (tree, head): the only sequential part, chunk by
+//                        chunk: the checkpoint at each chunk start,
 //                        U = U' - W S0^T, S <- g_C S + (diag(g_C/g) U)^T K;
 //   gdn_out_kernel    -- per (trunk chunk, head, half of the columns), in parallel:
-//                        the trunk rows' outputs (tcgen05 MMAs, TMEM accumulators);
-//   gdn_branch_kernel -- per (branch, head, 32 state rows): the state after the
+//                        the trunk rows' outputs;
+//   gdn_branch_kernel -- per (branch, head), in parallel: the state after the
 //                        anchor from the checkpoint of its chunk plus that chunk's
 //                        first m + 1 update vectors (the indexed state replay of the
 //                        figure, without a token-by-token pass), then the branch's
-//                        own tokens one by one (four threads own a row, 32 of its
-//                        columns each, features staged kGdnDepth tokens ahead with
-//                        cp.async).
+//                        own samples as one chunk from that state.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -44,26 +43,10 @@ namespace specopd {
 namespace {
 
 constexpr int kGdnD = 128;            // dk = dv
-constexpr int kGdnTpr = 4;            // threads per state row
-constexpr int kGdnCols = kGdnD / kGdnTpr;
-constexpr int kGdnRows = 32;           // state rows per CTA: a head's rows spread over kGdnD / kGdnRows CTAs
-constexpr int kGdnThreads = kGdnRows * kGdnTpr;
 constexpr int kGdnC = 64;             // checkpoint interval
-
-// Features of one token and head in shared memory: k, q, v (bf16, 256 bytes
-// each), alpha, beta.
-constexpr int kGdnDepth = 16;                  // tokens in flight
-constexpr int kGdnFeatBytes = 3 * kGdnD * 2 + 16;
-struct GdnRing {
-  alignas(16) uint8_t slot[kGdnDepth][kGdnFeatBytes];
-};
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
                : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
@@ -72,119 +55,8 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// token r's features of head h into a slot: 48 threads copy 16-byte pieces of
-// k, q and v, two more copy alpha and beta
-__device__ __forceinline__ void gdn_fetch(uint8_t* slot, const GdnArgs& g, long long r, int h) {
-  const int t = threadIdx.x;
-  const long long off = (r * g.H + h) * kGdnD;
-  if (t < 48) {
-    const int which = t >> 4, piece = t & 15;
-    const void* src = static_cast<const uint8_t*>(which == 0 ? g.k : which == 1 ? g.q : g.v) + off * 2 + piece * 16;
-    cp_async16(slot + which * kGdnD * 2 + piece * 16, src);
-  } else if (t == 48) {
-    cp_async4(slot + 3 * kGdnD * 2, g.alpha + r * g.H + h);
-  } else if (t == 49) {
-    cp_async4(slot + 3 * kGdnD * 2 + 4, g.beta + r * g.H + h);
-  }
-}
-
-__device__ __forceinline__ void unpack16(const uint4 (&w)[kGdnCols / 8], float (&x)[kGdnCols]) {
-#pragma unroll
-  for (int i = 0; i < kGdnCols / 8; ++i) {
-    const uint32_t u[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      x[8 * i + 2 * j] = __uint_as_float(u[j] << 16);
-      x[8 * i + 2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
-    }
-  }
-}
-
-// one token from its slot: update this thread's 32 columns of row `row`,
-// return o_row (valid in every thread of the row's quad)
-__device__ __forceinline__ float gdn_step(float (&S)[kGdnCols], const uint8_t* slot, int row, int part) {
-  uint4 kw[kGdnCols / 8], qw[kGdnCols / 8];
-#pragma unroll
-  for (int i = 0; i < kGdnCols / 8; ++i) {
-    kw[i] = reinterpret_cast<const uint4*>(slot + part * kGdnCols * 2)[i];
-    qw[i] = reinterpret_cast<const uint4*>(slot + kGdnD * 2 + part * kGdnCols * 2)[i];
-  }
-  float k[kGdnCols], q[kGdnCols];
-  unpack16(kw, k);
-  unpack16(qw, q);
-  const float v = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(slot + 2 * kGdnD * 2)[row]);
-  const float a = *reinterpret_cast<const float*>(slot + 3 * kGdnD * 2);
-  const float b = *reinterpret_cast<const float*>(slot + 3 * kGdnD * 2 + 4);
-  float u0 = 0.f, u1 = 0.f, u2 = 0.f, u3 = 0.f;
-#pragma unroll
-  for (int j = 0; j < kGdnCols; j += 4) {
-    u0 = fmaf(S[j], k[j], u0);
-    u1 = fmaf(S[j + 1], k[j + 1], u1);
-    u2 = fmaf(S[j + 2], k[j + 2], u2);
-    u3 = fmaf(S[j + 3], k[j + 3], u3);
-  }
-  float u = (u0 + u1) + (u2 + u3);
-  u += __shfl_xor_sync(0xffffffffu, u, 1);
-  u += __shfl_xor_sync(0xffffffffu, u, 2);
-  const float c = b * (v - a * u);
-  float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
-#pragma unroll
-  for (int j = 0; j < kGdnCols; j += 4) {
-    S[j] = fmaf(c, k[j], a * S[j]);
-    S[j + 1] = fmaf(c, k[j + 1], a * S[j + 1]);
-    S[j + 2] = fmaf(c, k[j + 2], a * S[j + 2]);
-    S[j + 3] = fmaf(c, k[j + 3], a * S[j + 3]);
-    o0 = fmaf(S[j], q[j], o0);
-    o1 = fmaf(S[j + 1], q[j + 1], o1);
-    o2 = fmaf(S[j + 2], q[j + 2], o2);
-    o3 = fmaf(S[j + 3], q[j + 3], o3);
-  }
-  float o = (o0 + o1) + (o2 + o3);
-  o += __shfl_xor_sync(0xffffffffu, o, 1);
-  o += __shfl_xor_sync(0xffffffffu, o, 2);
-  return o;
-}
-
-// rows r0 .. r1-1 (packed, consecutive) through the recurrence, their
-// features staged kGdnDepth tokens ahead in the CTA's ring (one cp.async group
-// per token; a slot is refilled only after every thread has passed the next
-// step's barrier, so no thread still reads it); outputs of rows >= out_from
-// written; with ck non-null a checkpoint after every row whose trunk position
-// p has (p + 1) % C == 0.  Every thread of the CTA calls it with the same
-// arguments.
-__device__ __forceinline__ void gdn_run(float (&S)[kGdnCols], GdnRing* ring, const GdnArgs& g, int h, int row,
-                                        int part, long long r0, long long r1, long long out_from, float* ck,
-                                        long long ck_pos0) {
-  if (r0 >= r1) return;
-  __syncthreads();  // the ring may still be read by an earlier call
-#pragma unroll 1
-  for (int d = 0; d < kGdnDepth - 1; ++d) {
-    if (r0 + d < r1) gdn_fetch(ring->slot[(r0 + d) % kGdnDepth], g, r0 + d, h);
-    cp_async_commit();
-  }
-  for (long long r = r0; r < r1; ++r) {
-    cp_async_wait<kGdnDepth - 2>();
-    __syncthreads();
-    const long long rn = r + kGdnDepth - 1;
-    if (rn < r1) gdn_fetch(ring->slot[rn % kGdnDepth], g, rn, h);
-    cp_async_commit();
-    const float o = gdn_step(S, ring->slot[r % kGdnDepth], row, part);
-    if (r >= out_from && part == 0) g.out[(r * g.H + h) * kGdnD + row] = o;
-    if (ck) {
-      const long long p = ck_pos0 + (r - r0);
-      if ((p + 1) % kGdnC == 0) {
-        float* dst = ck + ((p + 1) / kGdnC - 1) * (long long)g.H * kGdnD * kGdnD + row * kGdnD + part * kGdnCols;
-#pragma unroll
-        for (int j = 0; j < kGdnCols; j += 4)
-          *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
-      }
-    }
-  }
-  cp_async_wait<0>();
-}
-
 // ---------------------------------------------------------------- chunked trunk pass
-// Per (trunk chunk, head) the workspace holds (fp32): W^T [128][64], U [64][128]
+// Per (trunk chunk, head) the workspace holds (fp32): W [64][128], U [64][128]
 // (U' from phase A, then U from phase B), P [64][64], log2 decays [64], the
 // chunk-end decay ratios g_n/g_t [64] and g_n (padded to 4): kGdnChunkFloats.
 constexpr int kOffW = 0;
@@ -805,84 +677,376 @@ __global__ void __launch_bounds__(kOutThreads) gdn_out_kernel(const GdnArgs g) {
   }
 }
 
-// Phase D: branches, one CTA per (branch, head, 32 state rows).  The state
-// after the anchor a (in chunk c, m = a - C c) comes from the chunk's cached
-// data without a token-by-token replay: S = g_m S0 + sum_{t<=m} (g_m/g_t) U_t k_t^T,
-// S0 the chunk's start state; then the branch's own tokens run through the
-// recurrence one by one, writing their outputs.
-__global__ void __launch_bounds__(kGdnThreads) gdn_branch_kernel(const GdnArgs g) {
-  __shared__ GdnRing ring;
-  const int gb = blockIdx.x, h = blockIdx.y;
-  const int row = blockIdx.z * kGdnRows + threadIdx.x / kGdnTpr, part = threadIdx.x % kGdnTpr;
+// Phase D: branches on the tensor cores, one CTA per (branch, head), 256
+// threads.  A branch's nb <= 64 samples form one chunk whose start state is
+// S_a, the state after the anchor a (in trunk chunk c, m = a - C c), formed
+// without a token-by-token replay (the indexed state replay of the figure):
+//   S_a = g_m S_c + sum_{t<=m} (g_m/g_t) U_t k_t^T       (S_c: the chunk's checkpoint)
+// then the chunked form from S_a, as for a trunk chunk:
+//   Gram [K_b; Q_b] K_b^T -> A_b, P_b;   (I + A_b) [W_b | U'_b] = [diag(beta g) K_b | diag(beta) V_b];
+//   U_b = U'_b - W_b S_a^T;    O_b = diag(g) Q_b S_a^T + P_b U_b.
+// Products on the tensor cores (fp32 operands as bf16 pairs, bf16 inputs
+// exact), the triangular solve on fp32 FMAs (one column per thread).  TMEM
+// (256 columns): S_a [0, 128), then D1 = S_a W_b^T [0, 64) and D2 = S_a Q_b^T
+// [64, 128); the Gram [128, 192), then S_a's split Shi [128, 192) and Slo
+// [192, 256), then U_b^T's split [128, 192) and D3 = U_b^T P_b^T [192, 256).
+constexpr int kBrThreads = 256;
+constexpr uint32_t kBrRA = 48 * 1024;  // (coef U)^T and K_c^T panels, then W_b and P_b staging, then P_b panels
+constexpr uint32_t kBrRB = 32 * 1024;  // [K_b; Q_b] panels
+constexpr uint32_t kBrRC = 34 * 1024;  // V_b and A_b, then W_b panels
+
+struct BranchSmem {
+  uint8_t ra[kBrRA];
+  uint8_t kq[kBrRB];
+  uint8_t rc[kBrRC];
+  float lgb[kGdnC], betab[kGdnC], bgb[kGdnC];  // the branch's log2 g_t, beta_t, beta_t g_t
+  uint64_t bar;
+  uint32_t tmem;
+  int abort_flag;
+};
+// region RA
+constexpr uint32_t kBrUtHi = 0, kBrUtLo = kPanel, kBrKct = 2 * kPanel;  // phase 0-1
+constexpr uint32_t kBrWst = 0, kBrPst = 2 * kPanel;                     // phase 2 (fp32 [64][128], [64][64])
+constexpr uint32_t kBrPHi = 0, kBrPLo = kPanel / 2;                     // phase 4-5
+// region RC
+constexpr uint32_t kBrV = 0, kBrAs = kPanel;                            // phase 0-2 (bf16 [64][128], fp32 [64][kAsP])
+constexpr uint32_t kBrWHi = 0, kBrWLo = kPanel;                         // phase 2-3
+static_assert(kPanel + kGdnC * kAsP * 4 <= kBrRC, "branch region C too small");
+static_assert(2 * kPanel + kGdnC * kGdnC * 4 <= kBrRA, "branch region A too small");
+
+__global__ void __launch_bounds__(kBrThreads, 1) gdn_branch_kernel(const GdnArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  BranchSmem& sm = *reinterpret_cast<BranchSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int gb = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nb = g.tp.rows_per_branch;
+  if (nb <= 0) return;  // uniform: no samples to score
   int lo = 0, hi = g.tp.num_trees - 1;  // the tree holding global branch gb
   while (lo < hi) {
     const int mid = (lo + hi + 1) / 2;
     if (g.tp.branch_base[mid] <= gb) lo = mid; else hi = mid - 1;
   }
   const int t = lo;
-  const int T = g.tp.trunk_len[t], P = g.tp.prompt_len[t];
+  const int T = g.tp.trunk_len[t], Pl = g.tp.prompt_len[t];
   int a = g.anchors[gb];
-  if (a < P || a > T - 1) {
-    if (threadIdx.x == 0) atomicOr(reinterpret_cast<unsigned*>(g.status), SPECOPD_FLAG_ANCHOR);
-    a = a < P ? P : T - 1;
+  if (a < Pl || a > T - 1) {
+    if (tid == 0) atomicOr(reinterpret_cast<unsigned*>(g.status), SPECOPD_FLAG_ANCHOR);
+    a = a < Pl ? Pl : T - 1;
   }
   const long long base = g.tp.row_base[t];
   const int c = a / kGdnC, m = a - c * kGdnC;
-  float S[kGdnCols];
-  if (c > 0) {
-    const float* src = g.ckpt + ((long long)(g.ck_off[t] + c - 1) * g.H + h) * kGdnD * kGdnD + row * kGdnD +
-                       part * kGdnCols;
+  const long long first = base + T + (long long)(gb - g.tp.branch_base[t]) * nb;
+  const float* cdc = chunk_ptr(g, g.ch_off[t] + c, h);
+  const __nv_bfloat16* kk = static_cast<const __nv_bfloat16*>(g.k);
+  const __nv_bfloat16* qq = static_cast<const __nv_bfloat16*>(g.q);
+  const __nv_bfloat16* vv = static_cast<const __nv_bfloat16*>(g.v);
+  uint8_t* ra = sm.ra;
+  uint8_t* rc = sm.rc;
+  if (tid == 0) {
+    mbar_init(&sm.bar, 1);
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&sm.tmem, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem;
+  const int r = 32 * (warp & 3) + lane;   // the TMEM lane (state row) this thread may access
+  const int hc = warp >> 2;               // which half of the columns
+  const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+  const float lgm = cdc[kOffLg + m];
+  // ---- phase 0: staging
+  for (int idx = tid; idx < kGdnD * 8; idx += kBrThreads) {  // (coef U)^T: row r, tokens 8 j ..
+    const int rr = idx & 127, j = idx >> 7;
+    float x[8];
 #pragma unroll
-    for (int j = 0; j < kGdnCols; j += 4) {
-      const float4 x = *reinterpret_cast<const float4*>(src + j);
-      S[j] = x.x;
-      S[j + 1] = x.y;
-      S[j + 2] = x.z;
-      S[j + 3] = x.w;
+    for (int q = 0; q < 8; ++q) {
+      const int tt = 8 * j + q;
+      x[q] = tt <= m ? exp2f(lgm - cdc[kOffLg + tt]) * cdc[kOffU + tt * kGdnD + rr] : 0.f;
+    }
+    uint4 xh, xl;
+    split8(x, xh, xl);
+    *reinterpret_cast<uint4*>(ra + kBrUtHi + swz(rr, j)) = xh;
+    *reinterpret_cast<uint4*>(ra + kBrUtLo + swz(rr, j)) = xl;
+  }
+  for (int idx = tid; idx < kGdnD * 8; idx += kBrThreads) {  // K_c^T: row e, tokens 8 j .. (exact)
+    const int e = idx & 127, j = idx >> 7;
+    uint32_t w[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const int t0 = 8 * j + 2 * p;
+      const long long rw = base + (long long)c * kGdnC + t0;
+      const uint32_t l16 = t0 <= m ? __bfloat16_as_ushort(kk[(rw * g.H + h) * kGdnD + e]) : 0u;
+      const uint32_t h16 = t0 + 1 <= m ? __bfloat16_as_ushort(kk[((rw + 1) * g.H + h) * kGdnD + e]) : 0u;
+      w[p] = l16 | (h16 << 16);
+    }
+    *reinterpret_cast<uint4*>(ra + kBrKct + swz(e, j)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  for (int idx = tid; idx < kGdnC * 16; idx += kBrThreads) {  // K_b, Q_b, V_b rows (zero past nb)
+    const int tt = idx >> 4, j = idx & 15;
+    uint4 kw = make_uint4(0u, 0u, 0u, 0u), qw = kw, vw = kw;
+    if (tt < nb) {
+      const long long off = ((first + tt) * g.H + h) * kGdnD + 8 * j;
+      kw = *reinterpret_cast<const uint4*>(kk + off);
+      qw = *reinterpret_cast<const uint4*>(qq + off);
+      vw = *reinterpret_cast<const uint4*>(vv + off);
+    }
+    *reinterpret_cast<uint4*>(sm.kq + (j >> 3) * kPanel + swz(tt, j & 7)) = kw;
+    *reinterpret_cast<uint4*>(sm.kq + (j >> 3) * kPanel + swz(kGdnC + tt, j & 7)) = qw;
+    *reinterpret_cast<uint4*>(rc + kBrV + (tt * kGdnD + 8 * j) * 2) = vw;
+  }
+  if (tid < kGdnC) {
+    const bool in = tid < nb;
+    sm.lgb[tid] = in ? log2f(g.alpha[(first + tid) * g.H + h]) : 0.f;
+    sm.betab[tid] = in ? g.beta[(first + tid) * g.H + h] : 0.f;
+  }
+  if (c > 0) {  // g_m S_c into the accumulator: row r, columns 64 hc ..
+    const float gm = exp2f(lgm);
+    const float* src = g.ckpt + ((long long)(g.ck_off[t] + c - 1) * g.H + h) * kGdnD * kGdnD + r * kGdnD + 64 * hc;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      uint32_t v[32];
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(src + 32 * q + e);
+        v[e] = __float_as_uint(gm * x.x);
+        v[e + 1] = __float_as_uint(gm * x.y);
+        v[e + 2] = __float_as_uint(gm * x.z);
+        v[e + 3] = __float_as_uint(gm * x.w);
+      }
+      tmem_st32(tl + 64 * hc + 32 * q, v);
+    }
+    tmem_st_wait();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // ---- phase 1: S_a += (coef U)^T K_c;  Gram [K_b; Q_b] K_b^T
+  if (tid == 0) {
+    constexpr uint32_t id128 = idesc_bf16_f32(128, 128, false), id64 = idesc_bf16_f32(128, 64, false);
+    const uint32_t sra = smem_u32(ra), skq = smem_u32(sm.kq);
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      const uint64_t b = smem_desc_sw128(sra + kBrKct + ks * 32, 16, 1024);
+      mma_ss(tmem, smem_desc_sw128(sra + kBrUtHi + ks * 32, 16, 1024), b, id128, (c > 0 || ks > 0) ? 1u : 0u);
+      mma_ss(tmem, smem_desc_sw128(sra + kBrUtLo + ks * 32, 16, 1024), b, id128, 1u);
+    }
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint64_t d = smem_desc_sw128(skq + (ks >> 2) * kPanel + (ks & 3) * 32, 16, 1024);
+      mma_ss(tmem + 128, d, d, id64, ks > 0 ? 1u : 0u);
+    }
+    mma_commit(&sm.bar);
+  }
+  if (tid == 32)
+    for (int tt = 1; tt < kGdnC; ++tt) sm.lgb[tt] += sm.lgb[tt - 1];
+  __syncthreads();
+  if (tid < kGdnC) sm.bgb[tid] = sm.betab[tid] * exp2f(sm.lgb[tid]);
+  bool ok = mbar_wait_warp(&sm.bar, 0, &sm.abort_flag);
+  tc_fence_after();
+  // ---- phase 2a: A_b and P_b from the Gram (TMEM lanes 0..63: K_b K_b^T, 64..127: Q_b K_b^T)
+  float* As = reinterpret_cast<float*>(rc + kBrAs);
+  float* Pst = reinterpret_cast<float*>(ra + kBrPst);
+  if (warp < 4 && ok) {
+    const int tt = r & (kGdnC - 1);
+    const bool qrow = warp >= 2;
+    const float lgt = sm.lgb[tt], bt = sm.betab[tt];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint32_t v[32];
+      tmem_ld32(tl + 128 + 32 * half, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        float o[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = 32 * half + e + u;
+          const float ratio = exp2f(lgt - sm.lgb[i]);
+          const float x = __uint_as_float(v[e + u]);
+          o[u] = qrow ? ((i <= tt && tt < nb) ? ratio * x : 0.f) : ((i < tt && tt < nb) ? bt * ratio * x : 0.f);
+        }
+        const float4 o4 = make_float4(o[0], o[1], o[2], o[3]);
+        if (qrow)
+          *reinterpret_cast<float4*>(Pst + tt * kGdnC + 32 * half + e) = o4;
+        else
+          *reinterpret_cast<float4*>(As + tt * kAsP + 32 * half + e) = o4;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // ---- phase 2b: S_a's bf16 split into TMEM (row r, columns 64 hc ..); the solve
+  if (ok) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      uint32_t v[32], sh[16], sl[16];
+      tmem_ld32(tl + 64 * hc + 32 * q, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float x0 = __uint_as_float(v[2 * e]), x1 = __uint_as_float(v[2 * e + 1]);
+        sh[e] = pack_bf16x2(x0, x1);
+        sl[e] = pack_bf16x2(x0 - __uint_as_float(sh[e] << 16), x1 - __uint_as_float(sh[e] & 0xFFFF0000u));
+      }
+      tmem_st16(tl + 128 + 32 * hc + 16 * q, sh);
+      tmem_st16(tl + 192 + 32 * hc + 16 * q, sl);
+    }
+    tmem_st_wait();
+  }
+  const int j = tid;  // column j of [W_b | U'_b]
+  float X[kGdnC];
+#pragma unroll
+  for (int tt = 0; tt < kGdnC; ++tt) {
+    if (tt >= nb) {
+      X[tt] = 0.f;
+      continue;
+    }
+    const float bv = j < kGdnD
+                         ? sm.bgb[tt] * __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm.kq + swz_elem(tt, j)))
+                         : sm.betab[tt] * __bfloat162float(
+                                              reinterpret_cast<const __nv_bfloat16*>(rc + kBrV)[tt * kGdnD + j - kGdnD]);
+    float a0 = bv, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+    for (int i = 0; i + 3 < tt; i += 4) {
+      const float4 av = *reinterpret_cast<const float4*>(As + tt * kAsP + i);
+      a0 = fmaf(-av.x, X[i], a0);
+      a1 = fmaf(-av.y, X[i + 1], a1);
+      a2 = fmaf(-av.z, X[i + 2], a2);
+      a3 = fmaf(-av.w, X[i + 3], a3);
+    }
+#pragma unroll
+    for (int i = tt & ~3; i < tt; ++i) a0 = fmaf(-As[tt * kAsP + i], X[i], a0);
+    X[tt] = (a0 + a1) + (a2 + a3);
+  }
+  __syncthreads();  // the solve is done with V_b and A_b
+  // ---- phase 2c: W_b rows (tokens) to fp32 staging, then into bf16 panels
+  float* Wst = reinterpret_cast<float*>(ra + kBrWst);
+  if (j < kGdnD) {
+#pragma unroll
+    for (int tt = 0; tt < kGdnC; ++tt) Wst[tt * kGdnD + j] = X[tt];
+  }
+  __syncthreads();
+  for (int idx = tid; idx < kGdnC * 16; idx += kBrThreads) {
+    const int tt = idx >> 4, jj = idx & 15;
+    const float4 p0 = *reinterpret_cast<const float4*>(Wst + tt * kGdnD + 8 * jj);
+    const float4 p1 = *reinterpret_cast<const float4*>(Wst + tt * kGdnD + 8 * jj + 4);
+    const float x[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    uint4 xh, xl;
+    split8(x, xh, xl);
+    const uint32_t off = (jj >> 3) * kHalfPanel + swz(tt, jj & 7);
+    *reinterpret_cast<uint4*>(rc + kBrWHi + off) = xh;
+    *reinterpret_cast<uint4*>(rc + kBrWLo + off) = xl;
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // ---- phase 3: D1 = S_a W_b^T (3 MMAs per step), D2 = S_a Q_b^T (2 per step), A from TMEM
+  if (tid == 0) {
+    constexpr uint32_t id64 = idesc_bf16_f32(128, 64, false);
+    const uint32_t src_ = smem_u32(rc), skq = smem_u32(sm.kq);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint32_t bo = (ks >> 2) * kHalfPanel + (ks & 3) * 32;
+      const uint64_t wh = smem_desc_sw128(src_ + kBrWHi + bo, 16, 1024);
+      const uint64_t wl = smem_desc_sw128(src_ + kBrWLo + bo, 16, 1024);
+      const uint64_t bq = smem_desc_sw128(skq + (ks >> 2) * kPanel + kGdnC * 128 + (ks & 3) * 32, 16, 1024);
+      const uint32_t ah = tmem + 128 + ks * 8, al = tmem + 192 + ks * 8;
+      mma_ts(tmem, ah, wh, id64, ks > 0 ? 1u : 0u);
+      mma_ts(tmem, ah, wl, id64, 1u);
+      mma_ts(tmem, al, wh, id64, 1u);
+      mma_ts(tmem + 64, ah, bq, id64, ks > 0 ? 1u : 0u);
+      mma_ts(tmem + 64, al, bq, id64, 1u);
+    }
+    mma_commit(&sm.bar);
+  }
+  ok = mbar_wait_warp(&sm.bar, 1, &sm.abort_flag) && ok;
+  tc_fence_after();
+  // ---- phase 4: U_b = U'_b - D1^T (warps 4-7: U'_b column r is this thread's X), its split into
+  // TMEM; P_b into bf16 panels (warps 0-3)
+  if (warp >= 4) {
+    if (ok) {
+      uint32_t uh[32], ul[32];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        uint32_t v[32];
+        tmem_ld32(tl + 32 * q, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int tt = 32 * q + e;
+          const float u0 = tt < nb ? X[tt] - __uint_as_float(v[e]) : 0.f;
+          const float u1 = tt + 1 < nb ? X[tt + 1] - __uint_as_float(v[e + 1]) : 0.f;
+          const uint32_t hh = pack_bf16x2(u0, u1);
+          uh[16 * q + e / 2] = hh;
+          ul[16 * q + e / 2] = pack_bf16x2(u0 - __uint_as_float(hh << 16), u1 - __uint_as_float(hh & 0xFFFF0000u));
+        }
+      }
+      tmem_st32(tl + 128, uh);
+      tmem_st32(tl + 160, ul);
+      tmem_st_wait();
     }
   } else {
-#pragma unroll
-    for (int j = 0; j < kGdnCols; ++j) S[j] = 0.f;
+    for (int idx = tid; idx < kGdnC * 8; idx += 128) {
+      const int tt = idx >> 3, jj = idx & 7;
+      const float4 p0 = *reinterpret_cast<const float4*>(Pst + tt * kGdnC + 8 * jj);
+      const float4 p1 = *reinterpret_cast<const float4*>(Pst + tt * kGdnC + 8 * jj + 4);
+      const float x[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+      uint4 xh, xl;
+      split8(x, xh, xl);
+      *reinterpret_cast<uint4*>(ra + kBrPHi + swz(tt, jj)) = xh;
+      *reinterpret_cast<uint4*>(ra + kBrPLo + swz(tt, jj)) = xl;
+    }
   }
-  // the chunk's first m + 1 keys, update-vector entries of this CTA's rows and
-  // decays, staged in shared memory by all threads at once
-  __shared__ __align__(16) __nv_bfloat16 kst[kGdnC][kGdnD];
-  __shared__ float ust[kGdnC][kGdnRows];
-  __shared__ float lgs[kGdnC];
-  const long long chunk = g.ch_off[t] + c;
-  const float* lg = chunk_ptr(g, chunk, h) + kOffLg;
-  const float* Uc = chunk_ptr(g, chunk, h) + kOffU;
-  const __nv_bfloat16* kk = static_cast<const __nv_bfloat16*>(g.k);
-  for (int i = threadIdx.x; i <= m * (kGdnD / 8) + (kGdnD / 8 - 1); i += kGdnThreads) {
-    const int tt = i / (kGdnD / 8), pc = i % (kGdnD / 8);
-    cp_async16(&kst[tt][8 * pc], kk + ((base + (long long)c * kGdnC + tt) * g.H + h) * kGdnD + 8 * pc);
-  }
-  for (int i = threadIdx.x; i <= m * (kGdnRows / 4) + (kGdnRows / 4 - 1); i += kGdnThreads) {
-    const int tt = i / (kGdnRows / 4), pc = i % (kGdnRows / 4);
-    cp_async16(&ust[tt][4 * pc], Uc + tt * kGdnD + blockIdx.z * kGdnRows + 4 * pc);
-  }
-  for (int i = threadIdx.x; i <= m; i += kGdnThreads) cp_async4(&lgs[i], lg + i);
-  cp_async_commit();
-  cp_async_wait<0>();
+  fence_proxy_async_smem();
+  tc_fence_before();
   __syncthreads();
-  const int lrow = threadIdx.x / kGdnTpr;
-  const float lgm = lgs[m];
-  const float gm = exp2f(lgm);
+  tc_fence_after();
+  // ---- phase 5: D3 = U_b^T P_b^T (3 MMAs per step)
+  if (tid == 0) {
+    constexpr uint32_t id64 = idesc_bf16_f32(128, 64, false);
+    const uint32_t sra = smem_u32(ra);
 #pragma unroll
-  for (int j = 0; j < kGdnCols; ++j) S[j] *= gm;
-  for (int tt = 0; tt <= m; ++tt) {
-    const float coef = exp2f(lgm - lgs[tt]) * ust[tt][lrow];
-    uint4 kw[kGdnCols / 8];
-#pragma unroll
-    for (int i = 0; i < kGdnCols / 8; ++i) kw[i] = reinterpret_cast<const uint4*>(&kst[tt][part * kGdnCols])[i];
-    float kf[kGdnCols];
-    unpack16(kw, kf);
-#pragma unroll
-    for (int j = 0; j < kGdnCols; ++j) S[j] = fmaf(coef, kf[j], S[j]);
+    for (int ks = 0; ks < 4; ++ks) {
+      const uint64_t ph = smem_desc_sw128(sra + kBrPHi + ks * 32, 16, 1024);
+      const uint64_t pl = smem_desc_sw128(sra + kBrPLo + ks * 32, 16, 1024);
+      const uint32_t ah = tmem + 128 + ks * 8, al = tmem + 160 + ks * 8;
+      mma_ts(tmem + 192, ah, ph, id64, ks > 0 ? 1u : 0u);
+      mma_ts(tmem + 192, ah, pl, id64, 1u);
+      mma_ts(tmem + 192, al, ph, id64, 1u);
+    }
+    mma_commit(&sm.bar);
   }
-  // the branch's own rows
-  const long long first = base + T + (long long)(gb - g.tp.branch_base[t]) * g.tp.rows_per_branch;
-  gdn_run(S, &ring, g, h, row, part, first, first + g.tp.rows_per_branch, first, nullptr, 0);
+  ok = mbar_wait_warp(&sm.bar, 0, &sm.abort_flag) && ok;
+  tc_fence_after();
+  // ---- phase 6: O_b[t][r] = g_t D2[r][t] + D3[r][t], tokens 32 hc ..
+  if (ok) {
+    uint32_t d2[32], d3[32];
+    tmem_ld32(tl + 64 + 32 * hc, d2);
+    tmem_ld32(tl + 192 + 32 * hc, d3);
+    tmem_ld_wait();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int tt = 32 * hc + e;
+      if (tt < nb)
+        g.out[((first + tt) * g.H + h) * kGdnD + r] =
+            fmaf(exp2f(sm.lgb[tt]), __uint_as_float(d2[e]), __uint_as_float(d3[e]));
+    }
+  } else if (lane == 0) {
+    atomicOr(reinterpret_cast<unsigned*>(g.status), SPECOPD_FLAG_TIMEOUT);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
 }
 
 }  // namespace
@@ -926,7 +1090,9 @@ cudaError_t launch_gdn_tree(GdnArgs g, cudaStream_t stream) {
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (g.tp.total_branches == 0) return cudaSuccess;
-  gdn_branch_kernel<<<dim3(g.tp.total_branches, g.H, kGdnD / kGdnRows), kGdnThreads, 0, stream>>>(g);
+  e = cudaFuncSetAttribute(gdn_branch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(BranchSmem) + 1024);
+  if (e != cudaSuccess) return e;
+  gdn_branch_kernel<<<dim3(g.tp.total_branches, g.H), kBrThreads, sizeof(BranchSmem) + 1024, stream>>>(g);
   return cudaGetLastError();
 }
 
