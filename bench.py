@@ -50,9 +50,9 @@ KERNEL_SOURCES = {
                        "tree_attention_masked_b200/csrc/ptx.cuh"],
 }
 MEASURED_TRAFFIC = {  # {(workload, kernel): {"bytes": B, "sha": digest, "profile": file}}
-    (5, "tree_attention"): {"bytes": 3482385664.0 + 453979392.0, "sha": "ec93944992a931ed",
+    (5, "tree_attention"): {"bytes": 3460822272.0 + 454361856.0, "sha": "4bdfe3fbb81768aa",
                             "profile": "profiles/dram_traffic_scale27b.md"},
-    (5, "tv_overlap_e2e"): {"bytes": 17671086848.0 + 8334844672.0, "sha": "05ea75c9d2c9d63c",
+    (5, "tv_overlap_e2e"): {"bytes": 17651496192.0 + 8334336512.0, "sha": "2b82289312ce03e1",
                             "profile": "profiles/dram_traffic_scale27b.md"},
 }
 

@@ -686,12 +686,13 @@ __global__ void __launch_bounds__(kOutThreads) gdn_out_kernel(const GdnArgs g) {
 //   Gram [K_b; Q_b] K_b^T -> A_b, P_b;   (I + A_b) [W_b | U'_b] = [diag(beta g) K_b | diag(beta) V_b];
 //   U_b = U'_b - W_b S_a^T;    O_b = diag(g) Q_b S_a^T + P_b U_b.
 // Products on the tensor cores (fp32 operands as bf16 pairs, bf16 inputs
-// exact), the triangular solve on fp32 FMAs (one column per thread).  TMEM
-// (256 columns): S_a [0, 128), then D1 = S_a W_b^T [0, 64) and D2 = S_a Q_b^T
-// [64, 128); the Gram [128, 192), then S_a's split Shi [128, 192) and Slo
-// [192, 256), then U_b^T's split [128, 192) and D3 = U_b^T P_b^T [192, 256).
+// exact; token dimensions padded to 64), the triangular solve on fp32 FMAs
+// (one column per thread, NMAX >= nb steps unrolled).  TMEM (256 columns):
+// S_a [0, 128), then D1 = S_a W_b^T [0, 64) and D2 = S_a Q_b^T [64, 128); the
+// Gram [128, 192) and (coef U)^T's split [192, 256), then S_a's split [128,
+// 256), then U_b^T's split [128, 192) and D3 = U_b^T P_b^T [192, 256).
 constexpr int kBrThreads = 256;
-constexpr uint32_t kBrRA = 48 * 1024;  // (coef U)^T and K_c^T panels, then W_b and P_b staging, then P_b panels
+constexpr uint32_t kBrRA = 16 * 1024;  // K_c^T panel, then P_b panels
 constexpr uint32_t kBrRB = 32 * 1024;  // [K_b; Q_b] panels
 constexpr uint32_t kBrRC = 34 * 1024;  // V_b and A_b, then W_b panels
 
@@ -704,22 +705,19 @@ struct BranchSmem {
   uint32_t tmem;
   int abort_flag;
 };
-// region RA
-constexpr uint32_t kBrUtHi = 0, kBrUtLo = kPanel, kBrKct = 2 * kPanel;  // phase 0-1
-constexpr uint32_t kBrWst = 0, kBrPst = 2 * kPanel;                     // phase 2 (fp32 [64][128], [64][64])
-constexpr uint32_t kBrPHi = 0, kBrPLo = kPanel / 2;                     // phase 4-5
-// region RC
-constexpr uint32_t kBrV = 0, kBrAs = kPanel;                            // phase 0-2 (bf16 [64][128], fp32 [64][kAsP])
-constexpr uint32_t kBrWHi = 0, kBrWLo = kPanel;                         // phase 2-3
+constexpr uint32_t kBrKct = 0;                                      // region A, phase 0-1
+constexpr uint32_t kBrPHi = 0, kBrPLo = kPanel / 2;                 // region A, phase 2-5
+constexpr uint32_t kBrV = 0, kBrAs = kPanel;                        // region C, phase 0-2
+constexpr uint32_t kBrWHi = 0, kBrWLo = kPanel;                     // region C, phase 2-3
 static_assert(kPanel + kGdnC * kAsP * 4 <= kBrRC, "branch region C too small");
-static_assert(2 * kPanel + kGdnC * kGdnC * 4 <= kBrRA, "branch region A too small");
 
-__global__ void __launch_bounds__(kBrThreads, 1) gdn_branch_kernel(const GdnArgs g) {
+template <int NMAX>
+__global__ void __launch_bounds__(kBrThreads, NMAX <= 32 ? 2 : 1) gdn_branch_kernel(const GdnArgs g) {
   extern __shared__ uint8_t smem_raw[];
   BranchSmem& sm = *reinterpret_cast<BranchSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int gb = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nb = g.tp.rows_per_branch;
-  if (nb <= 0) return;  // uniform: no samples to score
+  if (nb <= 0 || nb > NMAX) return;  // uniform (the launcher picks NMAX >= nb)
   int lo = 0, hi = g.tp.num_trees - 1;  // the tree holding global branch gb
   while (lo < hi) {
     const int mid = (lo + hi + 1) / 2;
@@ -755,22 +753,23 @@ __global__ void __launch_bounds__(kBrThreads, 1) gdn_branch_kernel(const GdnArgs
   tc_fence_after();
   const uint32_t tmem = sm.tmem;
   const int r = 32 * (warp & 3) + lane;   // the TMEM lane (state row) this thread may access
-  const int hc = warp >> 2;               // which half of the columns
+  const int hc = warp >> 2;               // which half of the columns / tokens
   const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
   const float lgm = cdc[kOffLg + m];
   // ---- phase 0: staging
-  for (int idx = tid; idx < kGdnD * 8; idx += kBrThreads) {  // (coef U)^T: row r, tokens 8 j ..
-    const int rr = idx & 127, j = idx >> 7;
-    float x[8];
+  {  // (coef U)^T row r, tokens 32 hc .. 32 hc + 31, split into TMEM [192, 256)
+    uint32_t uh[16], ul[16];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int tt = 8 * j + q;
-      x[q] = tt <= m ? exp2f(lgm - cdc[kOffLg + tt]) * cdc[kOffU + tt * kGdnD + rr] : 0.f;
+    for (int e = 0; e < 32; e += 2) {
+      const int t0 = 32 * hc + e;
+      const float x0 = t0 <= m ? exp2f(lgm - cdc[kOffLg + t0]) * cdc[kOffU + t0 * kGdnD + r] : 0.f;
+      const float x1 = t0 + 1 <= m ? exp2f(lgm - cdc[kOffLg + t0 + 1]) * cdc[kOffU + (t0 + 1) * kGdnD + r] : 0.f;
+      const uint32_t hh = pack_bf16x2(x0, x1);
+      uh[e / 2] = hh;
+      ul[e / 2] = pack_bf16x2(x0 - __uint_as_float(hh << 16), x1 - __uint_as_float(hh & 0xFFFF0000u));
     }
-    uint4 xh, xl;
-    split8(x, xh, xl);
-    *reinterpret_cast<uint4*>(ra + kBrUtHi + swz(rr, j)) = xh;
-    *reinterpret_cast<uint4*>(ra + kBrUtLo + swz(rr, j)) = xl;
+    tmem_st16(tl + 192 + 16 * hc, uh);
+    tmem_st16(tl + 224 + 16 * hc, ul);
   }
   for (int idx = tid; idx < kGdnD * 8; idx += kBrThreads) {  // K_c^T: row e, tokens 8 j .. (exact)
     const int e = idx & 127, j = idx >> 7;
@@ -796,7 +795,7 @@ __global__ void __launch_bounds__(kBrThreads, 1) gdn_branch_kernel(const GdnArgs
     }
     *reinterpret_cast<uint4*>(sm.kq + (j >> 3) * kPanel + swz(tt, j & 7)) = kw;
     *reinterpret_cast<uint4*>(sm.kq + (j >> 3) * kPanel + swz(kGdnC + tt, j & 7)) = qw;
-    *reinterpret_cast<uint4*>(rc + kBrV + (tt * kGdnD + 8 * j) * 2) = vw;
+    if (tt < NMAX) *reinterpret_cast<uint4*>(rc + kBrV + (tt * kGdnD + 8 * j) * 2) = vw;
   }
   if (tid < kGdnC) {
     const bool in = tid < nb;
@@ -819,21 +818,21 @@ __global__ void __launch_bounds__(kBrThreads, 1) gdn_branch_kernel(const GdnArgs
       }
       tmem_st32(tl + 64 * hc + 32 * q, v);
     }
-    tmem_st_wait();
   }
+  tmem_st_wait();
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // ---- phase 1: S_a += (coef U)^T K_c;  Gram [K_b; Q_b] K_b^T
+  // ---- phase 1: S_a += (coef U)^T K_c (A from TMEM);  Gram [K_b; Q_b] K_b^T
   if (tid == 0) {
     constexpr uint32_t id128 = idesc_bf16_f32(128, 128, false), id64 = idesc_bf16_f32(128, 64, false);
     const uint32_t sra = smem_u32(ra), skq = smem_u32(sm.kq);
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
       const uint64_t b = smem_desc_sw128(sra + kBrKct + ks * 32, 16, 1024);
-      mma_ss(tmem, smem_desc_sw128(sra + kBrUtHi + ks * 32, 16, 1024), b, id128, (c > 0 || ks > 0) ? 1u : 0u);
-      mma_ss(tmem, smem_desc_sw128(sra + kBrUtLo + ks * 32, 16, 1024), b, id128, 1u);
+      mma_ts(tmem, tmem + 192 + ks * 8, b, id128, (c > 0 || ks > 0) ? 1u : 0u);
+      mma_ts(tmem, tmem + 224 + ks * 8, b, id128, 1u);
     }
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
@@ -848,9 +847,9 @@ __global__ void __launch_bounds__(kBrThreads, 1) gdn_branch_kernel(const GdnArgs
   if (tid < kGdnC) sm.bgb[tid] = sm.betab[tid] * exp2f(sm.lgb[tid]);
   bool ok = mbar_wait_warp(&sm.bar, 0, &sm.abort_flag);
   tc_fence_after();
-  // ---- phase 2a: A_b and P_b from the Gram (TMEM lanes 0..63: K_b K_b^T, 64..127: Q_b K_b^T)
+  // ---- phase 2a: from the Gram (TMEM lanes 0..63: K_b K_b^T, 64..127: Q_b K_b^T),
+  // A_b to shared memory and P_b straight into its bf16 panels (region A is free)
   float* As = reinterpret_cast<float*>(rc + kBrAs);
-  float* Pst = reinterpret_cast<float*>(ra + kBrPst);
   if (warp < 4 && ok) {
     const int tt = r & (kGdnC - 1);
     const bool qrow = warp >= 2;
@@ -861,20 +860,25 @@ __global__ void __launch_bounds__(kBrThreads, 1) gdn_branch_kernel(const GdnArgs
       tmem_ld32(tl + 128 + 32 * half, v);
       tmem_ld_wait();
 #pragma unroll
-      for (int e = 0; e < 32; e += 4) {
-        float o[4];
+      for (int e8 = 0; e8 < 32; e8 += 8) {
+        float o[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int i = 32 * half + e + u;
+        for (int u = 0; u < 8; ++u) {
+          const int i = 32 * half + e8 + u;
           const float ratio = exp2f(lgt - sm.lgb[i]);
-          const float x = __uint_as_float(v[e + u]);
+          const float x = __uint_as_float(v[e8 + u]);
           o[u] = qrow ? ((i <= tt && tt < nb) ? ratio * x : 0.f) : ((i < tt && tt < nb) ? bt * ratio * x : 0.f);
         }
-        const float4 o4 = make_float4(o[0], o[1], o[2], o[3]);
-        if (qrow)
-          *reinterpret_cast<float4*>(Pst + tt * kGdnC + 32 * half + e) = o4;
-        else
-          *reinterpret_cast<float4*>(As + tt * kAsP + 32 * half + e) = o4;
+        if (qrow) {
+          uint4 xh, xl;
+          split8(o, xh, xl);
+          const int j = (32 * half + e8) >> 3;
+          *reinterpret_cast<uint4*>(ra + kBrPHi + swz(tt, j)) = xh;
+          *reinterpret_cast<uint4*>(ra + kBrPLo + swz(tt, j)) = xl;
+        } else if (tt < NMAX) {
+          *reinterpret_cast<float4*>(As + tt * kAsP + 32 * half + e8) = make_float4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<float4*>(As + tt * kAsP + 32 * half + e8 + 4) = make_float4(o[4], o[5], o[6], o[7]);
+        }
       }
     }
   }
@@ -900,9 +904,9 @@ __global__ void __launch_bounds__(kBrThreads, 1) gdn_branch_kernel(const GdnArgs
     tmem_st_wait();
   }
   const int j = tid;  // column j of [W_b | U'_b]
-  float X[kGdnC];
+  float X[NMAX];
 #pragma unroll
-  for (int tt = 0; tt < kGdnC; ++tt) {
+  for (int tt = 0; tt < NMAX; ++tt) {
     if (tt >= nb) {
       X[tt] = 0.f;
       continue;
@@ -925,23 +929,19 @@ __global__ void __launch_bounds__(kBrThreads, 1) gdn_branch_kernel(const GdnArgs
     X[tt] = (a0 + a1) + (a2 + a3);
   }
   __syncthreads();  // the solve is done with V_b and A_b
-  // ---- phase 2c: W_b rows (tokens) to fp32 staging, then into bf16 panels
-  float* Wst = reinterpret_cast<float*>(ra + kBrWst);
+  // ---- phase 2c: W_b column j straight into its bf16 panels (rows = tokens, zero past NMAX)
   if (j < kGdnD) {
+    __nv_bfloat16* wh = reinterpret_cast<__nv_bfloat16*>(rc + kBrWHi);
+    __nv_bfloat16* wl = reinterpret_cast<__nv_bfloat16*>(rc + kBrWLo);
 #pragma unroll
-    for (int tt = 0; tt < kGdnC; ++tt) Wst[tt * kGdnD + j] = X[tt];
-  }
-  __syncthreads();
-  for (int idx = tid; idx < kGdnC * 16; idx += kBrThreads) {
-    const int tt = idx >> 4, jj = idx & 15;
-    const float4 p0 = *reinterpret_cast<const float4*>(Wst + tt * kGdnD + 8 * jj);
-    const float4 p1 = *reinterpret_cast<const float4*>(Wst + tt * kGdnD + 8 * jj + 4);
-    const float x[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-    uint4 xh, xl;
-    split8(x, xh, xl);
-    const uint32_t off = (jj >> 3) * kHalfPanel + swz(tt, jj & 7);
-    *reinterpret_cast<uint4*>(rc + kBrWHi + off) = xh;
-    *reinterpret_cast<uint4*>(rc + kBrWLo + off) = xl;
+    for (int tt = 0; tt < kGdnC; ++tt) {
+      const float x = tt < NMAX ? X[tt < NMAX ? tt : 0] : 0.f;
+      const __nv_bfloat16 xh = __float2bfloat16_rn(x);
+      const __nv_bfloat16 xl = __float2bfloat16_rn(x - __bfloat162float(xh));
+      const uint32_t off = ((j >> 6) * kHalfPanel + swz(tt, (j & 63) >> 3) + (j & 7) * 2) / 2;
+      wh[off] = xh;
+      wl[off] = xl;
+    }
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -968,43 +968,30 @@ __global__ void __launch_bounds__(kBrThreads, 1) gdn_branch_kernel(const GdnArgs
   }
   ok = mbar_wait_warp(&sm.bar, 1, &sm.abort_flag) && ok;
   tc_fence_after();
-  // ---- phase 4: U_b = U'_b - D1^T (warps 4-7: U'_b column r is this thread's X), its split into
-  // TMEM; P_b into bf16 panels (warps 0-3)
-  if (warp >= 4) {
-    if (ok) {
-      uint32_t uh[32], ul[32];
+  // ---- phase 4: U_b = U'_b - D1^T (warps 4-7: U'_b column r is this thread's X), split into TMEM
+  if (warp >= 4 && ok) {
+    uint32_t uh[32], ul[32];
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t v[32];
+    for (int q = 0; q < 2; ++q) {
+      uint32_t v[32];
+      if (32 * q < NMAX) {
         tmem_ld32(tl + 32 * q, v);
         tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int tt = 32 * q + e;
-          const float u0 = tt < nb ? X[tt] - __uint_as_float(v[e]) : 0.f;
-          const float u1 = tt + 1 < nb ? X[tt + 1] - __uint_as_float(v[e + 1]) : 0.f;
-          const uint32_t hh = pack_bf16x2(u0, u1);
-          uh[16 * q + e / 2] = hh;
-          ul[16 * q + e / 2] = pack_bf16x2(u0 - __uint_as_float(hh << 16), u1 - __uint_as_float(hh & 0xFFFF0000u));
-        }
       }
-      tmem_st32(tl + 128, uh);
-      tmem_st32(tl + 160, ul);
-      tmem_st_wait();
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        const int tt = 32 * q + e;
+        const float u0 = (tt < NMAX && tt < nb) ? X[tt < NMAX ? tt : 0] - __uint_as_float(v[e]) : 0.f;
+        const float u1 = (tt + 1 < NMAX && tt + 1 < nb) ? X[tt + 1 < NMAX ? tt + 1 : 0] - __uint_as_float(v[e + 1]) : 0.f;
+        const uint32_t hh = pack_bf16x2(u0, u1);
+        uh[16 * q + e / 2] = hh;
+        ul[16 * q + e / 2] = pack_bf16x2(u0 - __uint_as_float(hh << 16), u1 - __uint_as_float(hh & 0xFFFF0000u));
+      }
     }
-  } else {
-    for (int idx = tid; idx < kGdnC * 8; idx += 128) {
-      const int tt = idx >> 3, jj = idx & 7;
-      const float4 p0 = *reinterpret_cast<const float4*>(Pst + tt * kGdnC + 8 * jj);
-      const float4 p1 = *reinterpret_cast<const float4*>(Pst + tt * kGdnC + 8 * jj + 4);
-      const float x[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-      uint4 xh, xl;
-      split8(x, xh, xl);
-      *reinterpret_cast<uint4*>(ra + kBrPHi + swz(tt, jj)) = xh;
-      *reinterpret_cast<uint4*>(ra + kBrPLo + swz(tt, jj)) = xl;
-    }
+    tmem_st32(tl + 128, uh);
+    tmem_st32(tl + 160, ul);
+    tmem_st_wait();
   }
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1027,16 +1014,18 @@ __global__ void __launch_bounds__(kBrThreads, 1) gdn_branch_kernel(const GdnArgs
   tc_fence_after();
   // ---- phase 6: O_b[t][r] = g_t D2[r][t] + D3[r][t], tokens 32 hc ..
   if (ok) {
-    uint32_t d2[32], d3[32];
-    tmem_ld32(tl + 64 + 32 * hc, d2);
-    tmem_ld32(tl + 192 + 32 * hc, d3);
-    tmem_ld_wait();
+    if (32 * hc < nb) {
+      uint32_t d2[32], d3[32];
+      tmem_ld32(tl + 64 + 32 * hc, d2);
+      tmem_ld32(tl + 192 + 32 * hc, d3);
+      tmem_ld_wait();
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const int tt = 32 * hc + e;
-      if (tt < nb)
-        g.out[((first + tt) * g.H + h) * kGdnD + r] =
-            fmaf(exp2f(sm.lgb[tt]), __uint_as_float(d2[e]), __uint_as_float(d3[e]));
+      for (int e = 0; e < 32; ++e) {
+        const int tt = 32 * hc + e;
+        if (tt < nb)
+          g.out[((first + tt) * g.H + h) * kGdnD + r] =
+              fmaf(exp2f(sm.lgb[tt]), __uint_as_float(d2[e]), __uint_as_float(d3[e]));
+      }
     }
   } else if (lane == 0) {
     atomicOr(reinterpret_cast<unsigned*>(g.status), SPECOPD_FLAG_TIMEOUT);
@@ -1047,6 +1036,15 @@ __global__ void __launch_bounds__(kBrThreads, 1) gdn_branch_kernel(const GdnArgs
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }
+}
+
+template <int NMAX>
+cudaError_t launch_branch(const GdnArgs& g, cudaStream_t stream) {
+  const int smem = (int)sizeof(BranchSmem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(gdn_branch_kernel<NMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  gdn_branch_kernel<NMAX><<<dim3(g.tp.total_branches, g.H), kBrThreads, smem, stream>>>(g);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -1090,10 +1088,10 @@ cudaError_t launch_gdn_tree(GdnArgs g, cudaStream_t stream) {
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (g.tp.total_branches == 0) return cudaSuccess;
-  e = cudaFuncSetAttribute(gdn_branch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(BranchSmem) + 1024);
-  if (e != cudaSuccess) return e;
-  gdn_branch_kernel<<<dim3(g.tp.total_branches, g.H), kBrThreads, sizeof(BranchSmem) + 1024, stream>>>(g);
-  return cudaGetLastError();
+  // the branch kernel unrolls its triangular solve to the branch length
+  const int nb = g.tp.rows_per_branch;
+  if (nb <= 0) return cudaSuccess;
+  return nb <= 16 ? launch_branch<16>(g, stream) : nb <= 32 ? launch_branch<32>(g, stream) : launch_branch<64>(g, stream);
 }
 
 }  // namespace specopd
