@@ -247,15 +247,17 @@ __global__ void __launch_bounds__(kPrepThreads) gdn_prep_kernel(const GdnArgs g)
 // columns: S [0, 128), its bf16 split Shi [128, 192) and Slo [192, 256) (two
 // bf16 per column), D = S W^T [256, 320), the split of (coef U)^T: Uhi
 // [320, 352) and Ulo [352, 384).  Per chunk c of n tokens:
-//   warps 0-3, one state row per thread: store the checkpoint (the state at
-//     the chunk start), split S into Shi + Slo, scale S in place by g_n, the
-//     chunk's total decay, and take the row's U' column into registers;
-//   warps 4-7: split the chunk's W into bf16 panels, transpose K into a bf16
-//     panel (exact);
+//   every warp, one state row per thread (warps 0-3 and 4-7 share the TMEM
+//     lanes and take half of the columns each): store the checkpoint (the
+//     state at the chunk start), split S into Shi + Slo, scale S in place by
+//     g_n, the chunk's total decay, and take half of the row's U' column into
+//     registers; all threads split the chunk's W into bf16 panels and
+//     transpose K into a bf16 panel (exact);
 //   MMA group 1 (A from TMEM):  D = Shi Whi^T + Shi Wlo^T + Slo Whi^T    (M 128, N 64, K 128);
 //   meanwhile every thread prefetches the next chunk's W, U', K and decays
 //     (cp.async) into a raw staging buffer;
-//   warps 0-3:    U = U' - D^T (stored for phases C and D), then coef_t U_t split into Uhi + Ulo;
+//   every warp, half of the tokens: U = U' - D^T (stored for phases C and D),
+//     then coef_t U_t split into Uhi + Ulo;
 //   MMA group 2 (A from TMEM):  S += Uhi^T K + Ulo^T K                   (M 128, N 128, K 64).
 // The fp32 operands enter as bf16 pairs x = hi + lo (about 16 mantissa bits;
 // the dropped lo x lo term is about 2^-16 of a product); K is exact in bf16.
@@ -335,7 +337,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(const GdnArgs
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem;
-  const int r = 32 * (warp & 3) + lane;  // warps 0-3: state row r = TMEM lane r
+  const int r = 32 * (warp & 3) + lane;  // state row r = TMEM lane r
+  const int hc = warp >> 2;
   const uint32_t trow = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
   bool ok = true;
   // thread r's row of the state after token C j - 1, 32 elements from column 32 q
@@ -351,63 +354,62 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(const GdnArgs
     float* cd = chunk_ptr(g, g.ch_off[t] + c, h);
     cp_async_wait<0>();
     __syncthreads();  // chunk c's raw data is in shared memory
-    float up[kGdnC];  // warps 0-3: column r of U'
-    if (warp < 4) {
+    // every warp: state row r = TMEM lane r; warps 0-3 take the state's columns
+    // 0..63 and tokens 0..31, warps 4-7 columns 64..127 and tokens 32..63
+    float up[kGdnC / 2];  // U'[32 hc + i][r]
 #pragma unroll
-      for (int tt = 0; tt < kGdnC; ++tt) up[tt] = sm.raw.u[tt][r];
-      if (c > 0 && ok) {
-        // the state at the chunk start: checkpoint, bf16 split, scale by g_n in place
-        const float gn = sm.raw.coef[kGdnC];
+    for (int i = 0; i < kGdnC / 2; ++i) up[i] = sm.raw.u[32 * hc + i][r];
+    if (c > 0 && ok) {
+      // the state at the chunk start: checkpoint, bf16 split, scale by g_n in place
+      const float gn = sm.raw.coef[kGdnC];
 #pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          uint32_t v[32];
-          tmem_ld32(trow + kScS + 32 * q, v);
-          tmem_ld_wait();
-          store_ckpt_row(c, q, v);
-          uint32_t hi[16], lo[16];
+      for (int qq = 0; qq < 2; ++qq) {
+        const int q = 2 * hc + qq;
+        uint32_t v[32];
+        tmem_ld32(trow + kScS + 32 * q, v);
+        tmem_ld_wait();
+        store_ckpt_row(c, q, v);
+        uint32_t hi[16], lo[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float x0 = __uint_as_float(v[2 * e]), x1 = __uint_as_float(v[2 * e + 1]);
-            hi[e] = pack_bf16x2(x0, x1);
-            lo[e] = pack_bf16x2(x0 - __uint_as_float(hi[e] << 16), x1 - __uint_as_float(hi[e] & 0xFFFF0000u));
-          }
-          // 32 fp32 columns -> 16 bf16-pair columns of Shi and of Slo
-          tmem_st16(trow + kScShi + 16 * q, hi);
-          tmem_st16(trow + kScSlo + 16 * q, lo);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(gn * __uint_as_float(v[e]));
-          tmem_st32(trow + kScS + 32 * q, v);
+        for (int e = 0; e < 16; ++e) {
+          const float x0 = __uint_as_float(v[2 * e]), x1 = __uint_as_float(v[2 * e + 1]);
+          hi[e] = pack_bf16x2(x0, x1);
+          lo[e] = pack_bf16x2(x0 - __uint_as_float(hi[e] << 16), x1 - __uint_as_float(hi[e] & 0xFFFF0000u));
         }
-        tmem_st_wait();
-      }
-    } else {
-      const int u = tid - 128;
-      if (c > 0) {  // W rows (tokens) split into bf16 pairs; rows past n are zero in the record
-#pragma unroll 2
-        for (int idx = u; idx < kGdnC * 16; idx += 128) {
-          const int tt = idx >> 4, j = idx & 15;
-          const float4 a = *reinterpret_cast<const float4*>(&sm.raw.w[tt][8 * j]);
-          const float4 b = *reinterpret_cast<const float4*>(&sm.raw.w[tt][8 * j + 4]);
-          const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-          uint4 hi, lo;
-          split8(x, hi, lo);
-          const uint32_t off = (j >> 3) * kHalfPanel + swz(tt, j & 7);
-          *reinterpret_cast<uint4*>(sm.w_hi + off) = hi;
-          *reinterpret_cast<uint4*>(sm.w_lo + off) = lo;
-        }
-      }
-      // K^T: row e, tokens 8 j .. 8 j + 7
-      for (int idx = u; idx < kGdnD * 8; idx += 128) {
-        const int e = idx & 127, j = idx >> 7;
-        uint32_t w[4];
+        // 32 fp32 columns -> 16 bf16-pair columns of Shi and of Slo
+        tmem_st16(trow + kScShi + 16 * q, hi);
+        tmem_st16(trow + kScSlo + 16 * q, lo);
 #pragma unroll
-        for (int p = 0; p < 4; ++p)
-          w[p] = (uint32_t)__bfloat16_as_ushort(sm.raw.k[8 * j + 2 * p][e]) |
-                 ((uint32_t)__bfloat16_as_ushort(sm.raw.k[8 * j + 2 * p + 1][e]) << 16);
-        *reinterpret_cast<uint4*>(sm.kt + swz(e, j)) = make_uint4(w[0], w[1], w[2], w[3]);
+        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(gn * __uint_as_float(v[e]));
+        tmem_st32(trow + kScS + 32 * q, v);
       }
-      if (u < kGdnC) sm.coef[u] = u < n ? sm.raw.coef[u] : 0.f;
+      tmem_st_wait();
     }
+    if (c > 0) {  // W rows (tokens) split into bf16 pairs; rows past n are zero in the record
+#pragma unroll 2
+      for (int idx = tid; idx < kGdnC * 16; idx += kScanThreads) {
+        const int tt = idx >> 4, j = idx & 15;
+        const float4 a = *reinterpret_cast<const float4*>(&sm.raw.w[tt][8 * j]);
+        const float4 b = *reinterpret_cast<const float4*>(&sm.raw.w[tt][8 * j + 4]);
+        const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        uint4 hi, lo;
+        split8(x, hi, lo);
+        const uint32_t off = (j >> 3) * kHalfPanel + swz(tt, j & 7);
+        *reinterpret_cast<uint4*>(sm.w_hi + off) = hi;
+        *reinterpret_cast<uint4*>(sm.w_lo + off) = lo;
+      }
+    }
+    // K^T: row e, tokens 8 j .. 8 j + 7
+    for (int idx = tid; idx < kGdnD * 8; idx += kScanThreads) {
+      const int e = idx & 127, j = idx >> 7;
+      uint32_t w[4];
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+        w[p] = (uint32_t)__bfloat16_as_ushort(sm.raw.k[8 * j + 2 * p][e]) |
+               ((uint32_t)__bfloat16_as_ushort(sm.raw.k[8 * j + 2 * p + 1][e]) << 16);
+      *reinterpret_cast<uint4*>(sm.kt + swz(e, j)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    if (tid < kGdnC) sm.coef[tid] = tid < n ? sm.raw.coef[tid] : 0.f;
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -427,38 +429,36 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(const GdnArgs
     }
     // the raw buffer is consumed: fetch the next chunk during this one's MMAs
     if (c + 1 < nch) scan_prefetch(sm.raw, g, t, h, c + 1, tid);
-    if (warp < 4) {
-      // U = U' - (S W^T)^T for thread r's row, stored in place of U'; coef_t U_t split for group 2
+    {
+      // U = U' - (S W^T)^T for row r and this warp's 32 tokens, stored in place of
+      // U'; coef_t U_t split for group 2
       if (c > 0) {
         ok = ok && mbar_wait_warp(&sm.bar1, (uint32_t)(c - 1) & 1u, &sm.abort_flag);
         tc_fence_after();
       }
-      uint32_t hi[32], lo[32];
+      uint32_t v[32];
+      if (c > 0 && ok) {
+        tmem_ld32(trow + kScD + 32 * hc, v);
+        tmem_ld_wait();
+      } else {
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t v[32];
-        if (c > 0 && ok) {
-          tmem_ld32(trow + kScD + 32 * q, v);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = 0u;
-        }
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int tt = 32 * q + e;
-          const float u0 = tt < n ? up[tt] - __uint_as_float(v[e]) : 0.f;
-          const float u1 = tt + 1 < n ? up[tt + 1] - __uint_as_float(v[e + 1]) : 0.f;
-          if (tt < n) cd[kOffU + tt * kGdnD + r] = u0;
-          if (tt + 1 < n) cd[kOffU + (tt + 1) * kGdnD + r] = u1;
-          const float c0 = sm.coef[tt] * u0, c1 = sm.coef[tt + 1] * u1;
-          const uint32_t hh = pack_bf16x2(c0, c1);
-          hi[16 * q + e / 2] = hh;
-          lo[16 * q + e / 2] = pack_bf16x2(c0 - __uint_as_float(hh << 16), c1 - __uint_as_float(hh & 0xFFFF0000u));
-        }
+        for (int e = 0; e < 32; ++e) v[e] = 0u;
       }
-      tmem_st32(trow + kScUhi, hi);
-      tmem_st32(trow + kScUlo, lo);
+      uint32_t hi[16], lo[16];
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        const int tt = 32 * hc + e;
+        const float u0 = tt < n ? up[e] - __uint_as_float(v[e]) : 0.f;
+        const float u1 = tt + 1 < n ? up[e + 1] - __uint_as_float(v[e + 1]) : 0.f;
+        if (tt < n) cd[kOffU + tt * kGdnD + r] = u0;
+        if (tt + 1 < n) cd[kOffU + (tt + 1) * kGdnD + r] = u1;
+        const float c0 = sm.coef[tt] * u0, c1 = sm.coef[tt + 1] * u1;
+        const uint32_t hh = pack_bf16x2(c0, c1);
+        hi[e / 2] = hh;
+        lo[e / 2] = pack_bf16x2(c0 - __uint_as_float(hh << 16), c1 - __uint_as_float(hh & 0xFFFF0000u));
+      }
+      tmem_st16(trow + kScUhi + 16 * hc, hi);
+      tmem_st16(trow + kScUlo + 16 * hc, lo);
       tmem_st_wait();
     }
     tc_fence_before();
@@ -481,9 +481,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(const GdnArgs
   }
   cp_async_wait<0>();
   if (!ok && lane == 0) atomicOr(reinterpret_cast<unsigned*>(g.status), SPECOPD_FLAG_TIMEOUT);
-  if (warp < 4 && ok && T % kGdnC == 0 && nch > 0) {  // the state after the last token
+  if (ok && T % kGdnC == 0 && nch > 0) {  // the state after the last token
 #pragma unroll 1
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 2 * hc; q < 2 * hc + 2; ++q) {
       uint32_t v[32];
       tmem_ld32(trow + kScS + 32 * q, v);
       tmem_ld_wait();

@@ -144,7 +144,7 @@ struct SparseArgs {
   void* out;            // [N, Hq, 128] bf16
   void* rq;             // workspace: rotated q
   void* rk;             // workspace: rotated k
-  float* gkey;          // workspace: [trunk groups][Hkv][di] fp32
+  float* gkey;          // workspace: per tree [Hkv][di][trunk groups of the tree] fp32
   int64_t N;
   int Hq, Hkv, di, g, topk;
   float theta, scale, scale_log2;  // softmax scale and scale * log2(e)

@@ -14,10 +14,11 @@
 //   sparse_gkey_kernel   -- the keys of every complete trunk group (shared by
 //                           all rows of the tree): fp32 mean in position order;
 //   sparse_select_kernel -- one warp per (row, KV head): scores of the row's
-//                           complete groups (trunk keys from the table, keys of
-//                           groups holding branch tokens formed on the spot, in
-//                           the same order; the lanes split a key's elements and
-//                           a fixed shuffle tree sums the products), top-k by
+//                           complete groups (trunk keys from the table, one group
+//                           per lane with a sequential FMA chain; keys of groups
+//                           holding branch tokens formed on the spot, in
+//                           position order, the lanes splitting a key's elements
+//                           and a fixed shuffle tree summing the products), top-k by
 //                           repeated warp argmax; it
 //                           writes the chosen groups as an ascending list and
 //                           as bits of the row's selection words;
@@ -91,7 +92,10 @@ __global__ void sparse_gkey_kernel(const SparseArgs s) {
   const __nv_bfloat16* ki = static_cast<const __nv_bfloat16*>(s.ki);
   float sum = 0.f;
   for (int j = 0; j < s.g; ++j) sum += ldbf(ki + ((base + (long long)m * s.g + j) * s.Hkv + kvh) * s.di + e);
-  s.gkey[((long long)gidx * s.Hkv + kvh) * s.di + e] = sum / (float)s.g;
+  // element-major per (tree, KV head): element e of group m at (kvh di + e) ng + m,
+  // so that the lanes of the selection warp, one group each, read consecutive words
+  const int ng = s.gk_off[t + 1] - s.gk_off[t];
+  s.gkey[(long long)s.gk_off[t] * s.Hkv * s.di + ((long long)kvh * s.di + e) * ng + m] = sum / (float)s.g;
 }
 
 __global__ void __launch_bounds__(32 * kSpWarps) sparse_select_kernel(const SparseArgs s) {
@@ -108,36 +112,44 @@ __global__ void __launch_bounds__(32 * kSpWarps) sparse_select_kernel(const Spar
   const __nv_bfloat16* qi = static_cast<const __nv_bfloat16*>(s.qi) + (r * s.Hkv + kvh) * s.di;
   const __nv_bfloat16* ki = static_cast<const __nv_bfloat16*>(s.ki);
 
-  // ---- indexer scores of the complete groups: the lanes split each key's
-  // elements (lane + 32 i), then a fixed xor-shuffle tree sums the products
-  constexpr int kQi = 8;  // di <= 256
-  float qv[kQi];
-#pragma unroll
-  for (int i = 0; i < kQi; ++i) qv[i] = (lane + 32 * i < s.di) ? ldbf(qi + lane + 32 * i) : 0.f;
-  for (int m = 0; m < nc; ++m) {
-    float part = 0.f;
-    if (m * s.g + s.g - 1 <= x.a) {  // trunk group: the shared key
-      const float* key = s.gkey + ((long long)(s.gk_off[t] + m) * s.Hkv + kvh) * s.di;
-#pragma unroll
-      for (int i = 0; i < kQi; ++i)
-        if (lane + 32 * i < s.di) part = fmaf(qv[i], key[lane + 32 * i], part);
-    } else {                          // holds branch tokens: this branch's key, members summed in order
-      float sum[kQi];
-#pragma unroll
-      for (int i = 0; i < kQi; ++i) sum[i] = 0.f;
-      for (int j = 0; j < s.g; ++j) {
-        const __nv_bfloat16* kr = ki + (hist_row(x, m * s.g + j) * s.Hkv + kvh) * s.di;
-#pragma unroll
-        for (int i = 0; i < kQi; ++i)
-          if (lane + 32 * i < s.di) sum[i] += ldbf(kr + lane + 32 * i);
-      }
-#pragma unroll
-      for (int i = 0; i < kQi; ++i)
-        if (lane + 32 * i < s.di) part = fmaf(qv[i], sum[i] / (float)s.g, part);
+  // ---- indexer scores of the complete groups.  Groups wholly in the trunk
+  // part of the history use the shared keys: one group per lane, a sequential
+  // fp32 FMA chain over the di products in element order (the query from
+  // shared memory).  A group holding branch tokens gets this branch's key:
+  // the lanes split its elements (lane + 32 i), sum the members in position
+  // order, and a fixed xor-shuffle tree sums the products.
+  __shared__ float qsm[kSpWarps][256];
+  for (int e = lane; e < s.di; e += 32) qsm[w][e] = ldbf(qi + e);
+  __syncwarp();
+  const int nct = min(nc, (x.a + 1) / s.g);  // complete groups inside the trunk part
+  {
+    const int ng = s.gk_off[t + 1] - s.gk_off[t];
+    const float* gk0 = s.gkey + (long long)s.gk_off[t] * s.Hkv * s.di + (long long)kvh * s.di * ng;
+    for (int m = lane; m < nct; m += 32) {
+      float part = 0.f;
+#pragma unroll 8
+      for (int e = 0; e < s.di; ++e) part = fmaf(qsm[w][e], gk0[(long long)e * ng + m], part);
+      score[w][m] = part;
     }
+  }
+  constexpr int kQi = 8;  // di <= 256
+  for (int m = nct; m < nc; ++m) {
+    float sum[kQi];
+#pragma unroll
+    for (int i = 0; i < kQi; ++i) sum[i] = 0.f;
+    for (int j = 0; j < s.g; ++j) {
+      const __nv_bfloat16* kr = ki + (hist_row(x, m * s.g + j) * s.Hkv + kvh) * s.di;
+#pragma unroll
+      for (int i = 0; i < kQi; ++i)
+        if (lane + 32 * i < s.di) sum[i] += ldbf(kr + lane + 32 * i);
+    }
+    float part = 0.f;
+#pragma unroll
+    for (int i = 0; i < kQi; ++i)
+      if (lane + 32 * i < s.di) part = fmaf(qsm[w][lane + 32 * i], sum[i] / (float)s.g, part);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-    if (lane == (m & 31)) score[w][m] = part;
+    if (lane == 0) score[w][m] = part;
   }
   __syncwarp();
 
