@@ -274,6 +274,7 @@ struct ScanRaw {  // one chunk record's W, U', decays, and the chunk's K rows, a
   __nv_bfloat16 k[kGdnC][kGdnD];
 };
 struct ScanSmem {
+  float ct[kScanThreads / 32][32][33];                 // per warp: a 32 x 32 state tile on its way to the checkpoint
   uint8_t w_hi[2 * kHalfPanel], w_lo[2 * kHalfPanel];  // B of group 1: W rows (tokens), K = 128
   uint8_t kt[kPanel];                                  // B of group 2: K^T rows (key elements), K = 64 tokens
   ScanRaw raw;
@@ -341,13 +342,19 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(const GdnArgs
   const int hc = warp >> 2;
   const uint32_t trow = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
   bool ok = true;
-  // thread r's row of the state after token C j - 1, 32 elements from column 32 q
+  // the warp's 32 state rows (TMEM lanes), 32 elements from column 32 q, of the
+  // state after token C j - 1 into the checkpoint: transposed through shared
+  // memory so that every store writes 128 contiguous bytes of one row
   auto store_ckpt_row = [&](int j, int q, const uint32_t (&v)[32]) {
-    float* dst = g.ckpt + ((long long)(g.ck_off[t] + j - 1) * g.H + h) * kGdnD * kGdnD + (long long)r * kGdnD + 32 * q;
+    float (*tile)[33] = sm.ct[warp];
 #pragma unroll
-    for (int e = 0; e < 32; e += 4)
-      *reinterpret_cast<float4*>(dst + e) = make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                                                        __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+    for (int e = 0; e < 32; ++e) tile[lane][e] = __uint_as_float(v[e]);
+    __syncwarp();
+    float* dst = g.ckpt + ((long long)(g.ck_off[t] + j - 1) * g.H + h) * kGdnD * kGdnD +
+                 (long long)(32 * (warp & 3)) * kGdnD + 32 * q + lane;
+#pragma unroll 8
+    for (int rr = 0; rr < 32; ++rr) dst[rr * kGdnD] = tile[rr][lane];
+    __syncwarp();
   };
   for (int c = 0; c < nch; ++c) {
     const int n = min(kGdnC, T - c * kGdnC);
