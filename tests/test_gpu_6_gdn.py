@@ -71,6 +71,9 @@ CASES = [
     dict(trees=[(150, 20, 4), (70, 3, 2), (64, 0, 1)], W=3, H=1),  # several trees; a trunk of exactly 64
     dict(trees=[(130, 10, 5)], W=1, H=2),                     # one-token branches
     dict(trees=[(130, 10, 5)], W=5, H=2, pack_terminal=False),  # terminal rows not packed
+    dict(trees=[(200, 10, 4)], W=20, H=2),                    # 20-sample branches: the 32-step branch solve
+    dict(trees=[(150, 10, 3)], W=64, H=1),                    # 64-sample branches: the 64-step branch solve
+    dict(trees=[(300, 50, 3)], W=40, H=1, pack_terminal=False),  # 39 rows per branch, padded to 64
 ]
 
 
