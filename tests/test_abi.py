@@ -159,12 +159,13 @@ def test_sparse_argument_errors_before_launch(S):
     N = S.specopd_tree_packed_rows(trees)
     tiles = S.specopd_tree_num_tiles(trees)
     need = S.specopd_sparse_workspace_bytes(trees, 4, 2, 32, 8, 4)
-    # rotated Q, K; trunk group keys; chosen groups [N][Hkv][topk]; selection words
+    # rotated Q, K; trunk group keys; branch group keys (4 branches x (4 // 8 + 1) slots);
+    # chosen groups [N][Hkv][topk]; selection words
     # (the deepest row has (200 + 4) // 8 = 25 complete groups: one word)
-    rq, rk, gk = N * 4 * 128 * 2, N * 2 * 128 * 2, (200 // 8) * 2 * 32 * 4
+    rq, rk, gk, bk = N * 4 * 128 * 2, N * 2 * 128 * 2, (200 // 8) * 2 * 32 * 4, 4 * 1 * 2 * 32 * 4
     lst, words = N * 2 * 4 * 4, N * 2 * 1 * 4
     up = lambda x: (x + 255) // 256 * 256
-    assert need == up(rq) + up(rk) + up(gk) + up(lst) + up(words)
+    assert need == up(rq) + up(rk) + up(gk) + up(bk) + up(lst) + up(words)
     assert S.specopd_sparse_workspace_bytes(trees, 4, 2, 32, 8, 0) == 0
     f = S._c["specopd_sparse_tree_attention"]
     args = lambda **kw: [trees.ref(), kw.get("q", 16), 16, 16, 16, 16, 16, kw.get("N", N), 4, kw.get("Hkv", 2),

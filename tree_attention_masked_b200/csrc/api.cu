@@ -408,10 +408,11 @@ int specopd_gdn_tree(const specopd_tree_desc* desc, const void* q, const void* k
 }
 
 // Sparse attention workspace (all regions 256-byte aligned): rotated Q [N][Hq][128]
-// and K [N][Hkv][128] bf16, trunk group keys [groups][Hkv][di] fp32, the chosen
+// and K [N][Hkv][128] bf16, trunk group keys [groups][Hkv][di] fp32, the keys of
+// the groups holding branch tokens [branches][slots][Hkv][di] fp32, the chosen
 // groups [N][Hkv][topk] int32 and the selection words [N][Hkv][words] uint32.
 struct SparseLayout {
-  size_t rk, gk, list, mask, total;
+  size_t rk, gk, bk, list, mask, total;
   int words;
 };
 
@@ -421,7 +422,8 @@ static SparseLayout sparse_layout(const TreeParams& p, int Hq, int Hkv, int di, 
   L.words = sparse_selection_words(p, g);
   L.rk = align_up((size_t)N * Hq * 128 * 2);
   L.gk = L.rk + align_up((size_t)N * Hkv * 128 * 2);
-  L.list = L.gk + align_up(sparse_group_keys(p, g) * Hkv * di * sizeof(float));
+  L.bk = L.gk + align_up(sparse_group_keys(p, g) * Hkv * di * sizeof(float));
+  L.list = L.bk + align_up((size_t)p.total_branches * sparse_branch_slots(p, g) * Hkv * di * sizeof(float));
   L.mask = L.list + align_up((size_t)N * Hkv * topk * sizeof(int32_t));
   L.total = L.mask + align_up((size_t)N * Hkv * L.words * sizeof(uint32_t));
   return L;
@@ -467,6 +469,8 @@ int specopd_sparse_tree_attention(const specopd_tree_desc* desc, const void* q, 
   a.rq = ws;
   a.rk = ws + L.rk;
   a.gkey = reinterpret_cast<float*>(ws + L.gk);
+  a.bkey = reinterpret_cast<float*>(ws + L.bk);
+  a.bslots = sparse_branch_slots(a.tp, g);
   a.sel_list = reinterpret_cast<int32_t*>(ws + L.list);
   a.sel_mask = reinterpret_cast<uint32_t*>(ws + L.mask);
   a.sel_words = L.words;

@@ -145,6 +145,8 @@ struct SparseArgs {
   void* rq;             // workspace: rotated q
   void* rk;             // workspace: rotated k
   float* gkey;          // workspace: per tree [Hkv][di][trunk groups of the tree] fp32
+  float* bkey;          // workspace: [branches][bslots][Hkv][di] fp32, keys of groups holding branch tokens
+  int bslots;           // rows_per_branch / g + 1: groups holding branch tokens per branch, at most
   int64_t N;
   int Hq, Hkv, di, g, topk;
   float theta, scale, scale_log2;  // softmax scale and scale * log2(e)
@@ -163,6 +165,8 @@ struct SparseArgs {
   int32_t gk_off[SPECOPD_MAX_TREES + 1];  // first trunk group of each tree (set by the launcher)
 };
 size_t sparse_group_keys(const TreeParams& tp, int g);
+// slots per branch for the keys of complete groups that hold branch tokens
+inline int sparse_branch_slots(const TreeParams& tp, int g) { return tp.rows_per_branch / g + 1; }
 int sparse_selection_words(const TreeParams& tp, int g);
 cudaError_t launch_sparse_attention(SparseArgs s, cudaStream_t stream);
 

@@ -13,12 +13,13 @@
 //
 //   sparse_gkey_kernel   -- the keys of every complete trunk group (shared by
 //                           all rows of the tree): fp32 mean in position order;
+//   sparse_bkey_kernel   -- the keys of the complete groups holding branch
+//                           tokens, once per branch (members in position order);
 //   sparse_select_kernel -- one warp per (row, KV head): scores of the row's
 //                           complete groups (trunk keys from the table, one group
-//                           per lane with a sequential FMA chain; keys of groups
-//                           holding branch tokens formed on the spot, in
-//                           position order, the lanes splitting a key's elements
-//                           and a fixed shuffle tree summing the products), top-k by
+//                           per lane with a sequential FMA chain; the branch's
+//                           keys with the lanes splitting a key's elements and
+//                           a fixed shuffle tree summing the products), top-k by
 //                           repeated warp argmax; it
 //                           writes the chosen groups as an ascending list and
 //                           as bits of the row's selection words;
@@ -41,6 +42,7 @@ constexpr int kSpD = 128;             // head dim
 constexpr int kSpWarps = 4;           // (row, KV head) items per CTA
 
 struct RowPlace {
+  int gb;           // global branch (branch rows)
   int t;            // tree
   long long base;   // first packed row of the tree
   long long bfirst; // first packed row of the branch (branch rows)
@@ -64,6 +66,7 @@ __device__ __forceinline__ RowPlace place_row(const SparseArgs& s, long long r) 
     x.p = (int)local;
     x.a = x.p;
     x.bfirst = 0;
+    x.gb = -1;
   } else {
     const long long bl = (local - T) / rpb;
     const int i = (int)((local - T) % rpb);
@@ -72,6 +75,7 @@ __device__ __forceinline__ RowPlace place_row(const SparseArgs& s, long long r) 
     x.a = a;
     x.p = a + 1 + i;
     x.bfirst = x.base + T + bl * rpb;
+    x.gb = s.tp.branch_base[t] + (int)bl;
   }
   return x;
 }
@@ -98,6 +102,36 @@ __global__ void sparse_gkey_kernel(const SparseArgs s) {
   s.gkey[(long long)s.gk_off[t] * s.Hkv * s.di + ((long long)kvh * s.di + e) * ng + m] = sum / (float)s.g;
 }
 
+// Keys of the complete groups that hold branch tokens, once per (branch, slot,
+// KV head): group m0 + slot with m0 = (a + 1) / g, members in position order
+// (trunk rows up to the anchor, then the branch's rows), an fp32 sum divided by
+// g; every row of the branch that sees the group complete shares its key.
+__global__ void sparse_bkey_kernel(const SparseArgs s) {
+  const int gb = blockIdx.x / s.bslots, slot = blockIdx.x % s.bslots, kvh = blockIdx.y, e = threadIdx.x;
+  if (e >= s.di) return;
+  int lo = 0, hi = s.tp.num_trees - 1;  // the tree holding global branch gb
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) / 2;
+    if (s.tp.branch_base[mid] <= gb) lo = mid; else hi = mid - 1;
+  }
+  const int t = lo;
+  const int T = s.tp.trunk_len[t], P = s.tp.prompt_len[t], rpb = s.tp.rows_per_branch;
+  int a = s.anchors[gb];
+  a = a < P ? P : (a > T - 1 ? T - 1 : a);
+  const int m = (a + 1) / s.g + slot;
+  if ((long long)m * s.g + s.g - 1 > a + rpb) return;  // no row of the branch sees it complete
+  const long long base = s.tp.row_base[t];
+  const long long bfirst = base + T + (long long)(gb - s.tp.branch_base[t]) * rpb;
+  const __nv_bfloat16* ki = static_cast<const __nv_bfloat16*>(s.ki);
+  float sum = 0.f;
+  for (int j = 0; j < s.g; ++j) {
+    const int q = m * s.g + j;
+    const long long row = q <= a ? base + q : bfirst + (q - a - 1);
+    sum += ldbf(ki + (row * s.Hkv + kvh) * s.di + e);
+  }
+  s.bkey[(((long long)gb * s.bslots + slot) * s.Hkv + kvh) * s.di + e] = sum / (float)s.g;
+}
+
 __global__ void __launch_bounds__(32 * kSpWarps) sparse_select_kernel(const SparseArgs s) {
   __shared__ float score[kSpWarps][kSpMaxGroups];
   __shared__ int sel[kSpWarps][kSpMaxTopk];
@@ -110,7 +144,6 @@ __global__ void __launch_bounds__(32 * kSpWarps) sparse_select_kernel(const Spar
   const int t = x.t;
   const int nc = (x.p + 1) / s.g;  // complete groups
   const __nv_bfloat16* qi = static_cast<const __nv_bfloat16*>(s.qi) + (r * s.Hkv + kvh) * s.di;
-  const __nv_bfloat16* ki = static_cast<const __nv_bfloat16*>(s.ki);
 
   // ---- indexer scores of the complete groups.  Groups wholly in the trunk
   // part of the history use the shared keys: one group per lane, a sequential
@@ -133,20 +166,12 @@ __global__ void __launch_bounds__(32 * kSpWarps) sparse_select_kernel(const Spar
     }
   }
   constexpr int kQi = 8;  // di <= 256
-  for (int m = nct; m < nc; ++m) {
-    float sum[kQi];
-#pragma unroll
-    for (int i = 0; i < kQi; ++i) sum[i] = 0.f;
-    for (int j = 0; j < s.g; ++j) {
-      const __nv_bfloat16* kr = ki + (hist_row(x, m * s.g + j) * s.Hkv + kvh) * s.di;
-#pragma unroll
-      for (int i = 0; i < kQi; ++i)
-        if (lane + 32 * i < s.di) sum[i] += ldbf(kr + lane + 32 * i);
-    }
+  for (int m = nct; m < nc; ++m) {  // groups holding branch tokens: this branch's keys, formed once per branch
+    const float* key = s.bkey + (((long long)x.gb * s.bslots + (m - nct)) * s.Hkv + kvh) * s.di;
     float part = 0.f;
 #pragma unroll
     for (int i = 0; i < kQi; ++i)
-      if (lane + 32 * i < s.di) part = fmaf(qsm[w][lane + 32 * i], sum[i] / (float)s.g, part);
+      if (lane + 32 * i < s.di) part = fmaf(qsm[w][lane + 32 * i], key[lane + 32 * i], part);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
     if (lane == 0) score[w][m] = part;
@@ -290,6 +315,11 @@ cudaError_t launch_sparse_attention(SparseArgs s, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   if (off > 0) {
     sparse_gkey_kernel<<<dim3(off, s.Hkv), (s.di + 31) / 32 * 32, 0, stream>>>(s);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (s.tp.total_branches > 0 && s.tp.rows_per_branch > 0) {
+    sparse_bkey_kernel<<<dim3(s.tp.total_branches * s.bslots, s.Hkv), (s.di + 31) / 32 * 32, 0, stream>>>(s);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
