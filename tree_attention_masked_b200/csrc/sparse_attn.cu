@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(32 * kSpWarps) sparse_select_kernel(const Spar
   // shared memory).  A group holding branch tokens gets this branch's key:
   // the lanes split its elements (lane + 32 i), sum the members in position
   // order, and a fixed xor-shuffle tree sums the products.
-  __shared__ float qsm[kSpWarps][256];
+  __shared__ __align__(16) float qsm[kSpWarps][256];
   for (int e = lane; e < s.di; e += 32) qsm[w][e] = ldbf(qi + e);
   __syncwarp();
   const int nct = min(nc, (x.a + 1) / s.g);  // complete groups inside the trunk part
@@ -159,9 +159,19 @@ __global__ void __launch_bounds__(32 * kSpWarps) sparse_select_kernel(const Spar
     const int ng = s.gk_off[t + 1] - s.gk_off[t];
     const float* gk0 = s.gkey + (long long)s.gk_off[t] * s.Hkv * s.di + (long long)kvh * s.di * ng;
     for (int m = lane; m < nct; m += 32) {
+      const float* col = gk0 + m;  // element e of group m at col[e ng]
       float part = 0.f;
-#pragma unroll 8
-      for (int e = 0; e < s.di; ++e) part = fmaf(qsm[w][e], gk0[(long long)e * ng + m], part);
+      int e = 0;
+#pragma unroll 2
+      for (; e + 4 <= s.di; e += 4) {
+        const float4 q4 = *reinterpret_cast<const float4*>(&qsm[w][e]);
+        part = fmaf(q4.x, col[0], part);
+        part = fmaf(q4.y, col[ng], part);
+        part = fmaf(q4.z, col[2 * ng], part);
+        part = fmaf(q4.w, col[3 * ng], part);
+        col += 4 * ng;
+      }
+      for (; e < s.di; ++e, col += ng) part = fmaf(qsm[w][e], *col, part);
       score[w][m] = part;
     }
   }
@@ -206,17 +216,20 @@ __global__ void __launch_bounds__(32 * kSpWarps) sparse_select_kernel(const Spar
       }
       __syncwarp();
     }
-    if (lane == 0) {  // groups in ascending order
-      for (int i = 1; i < K; ++i) {
-        const int v = sel[w][i];
-        int j = i - 1;
-        while (j >= 0 && sel[w][j] > v) {
-          sel[w][j + 1] = sel[w][j];
-          --j;
-        }
-        sel[w][j + 1] = v;
-      }
+    // groups in ascending order: every lane ranks the choices it holds (the
+    // groups are distinct, so the ranks are a permutation)
+    __syncwarp();
+    const int v0 = lane < K ? sel[w][lane] : 0x7fffffff;
+    const int v1 = lane + 32 < K ? sel[w][lane + 32] : 0x7fffffff;
+    int r0 = 0, r1 = 0;
+    for (int i = 0; i < K; ++i) {
+      const int u = sel[w][i];
+      r0 += u < v0 ? 1 : 0;
+      r1 += u < v1 ? 1 : 0;
     }
+    __syncwarp();
+    if (lane < K) sel[w][r0] = v0;
+    if (lane + 32 < K) sel[w][r1] = v1;
   } else if (lane == 0) {
     for (int i = 0; i < K; ++i) sel[w][i] = i;
   }
