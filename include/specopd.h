@@ -297,8 +297,9 @@ int specopd_tree_causal_conv(const void* x, void* out, specopd_dtype dtype, int6
                              const int32_t* cu_rows, int num_trees, specopd_stream_t stream);
 
 /* Bytes of workspace specopd_gdn_tree needs: the fp32 trunk checkpoints,
- * (sum over trees of T / 64) * H * 128 * 128 * 4 rounded up to 256 (0 for an
- * invalid description). */
+ * (sum over trees of T / 64) * H * 128 * 128 * 4, then the chunked form's
+ * record of every trunk chunk and head, (sum over trees of ceil(T / 64)) * H
+ * * 20,612 * 4, each rounded up to 256 (0 for an invalid description). */
 size_t specopd_gdn_workspace_bytes(const specopd_tree_desc* desc, int H);
 
 /*
@@ -316,6 +317,12 @@ size_t specopd_gdn_workspace_bytes(const specopd_tree_desc* desc, int H);
  *   o_t = S_t q_t.
  * A branch's history is the trunk through its anchor, then its own earlier
  * tokens (the packing of specopd_build_tree_mask for the same description).
+ * The library computes the same outputs in the chunked form of the rule (64
+ * tokens per chunk: a per-chunk triangular solve and products, the state
+ * carried from chunk to chunk in fp32), with the products on the tensor cores
+ * and fp32 operands split into bf16 pairs; a branch's state at its anchor is
+ * formed from the checkpoint and that chunk's cached update vectors, and its
+ * samples run as one chunk from there.
  *
  * q, k, v [N, H, 128] bf16 (dk = dv = 128; k normalised upstream), alpha,
  * beta [N, H] fp32, out [N, H, 128] fp32: device, row-major, 16-byte aligned.
@@ -332,9 +339,10 @@ int specopd_gdn_tree(const specopd_tree_desc* desc, const void* q, const void* k
                      void* workspace, size_t workspace_bytes, int32_t* status, specopd_stream_t stream);
 
 /* Bytes of workspace specopd_sparse_tree_attention needs: rotated Q and K
- * (bf16), the trunk group keys (fp32), the chosen groups [N][Hkv][topk]
- * (int32) and the per-row selection words (uint32), each rounded up to 256
- * bytes (0 for an invalid description). */
+ * (bf16), the trunk group keys and the keys of the groups holding branch
+ * tokens (fp32), the chosen groups [N][Hkv][topk] (int32) and the per-row
+ * selection words (uint32), each rounded up to 256 bytes (0 for an invalid
+ * description). */
 size_t specopd_sparse_workspace_bytes(const specopd_tree_desc* desc, int Hq, int Hkv, int di, int g, int topk);
 
 /*
